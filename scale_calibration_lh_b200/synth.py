@@ -1,0 +1,298 @@
+"""Seeded synthetic inputs for the calibration hot path.
+
+This module is shared by the CUDA path's tests and benchmark and by the CPU
+oracle's tests. It holds no step of the calibration method itself (no Hessian,
+no scale sweep, no loss): only random draws, their shaping into the layer
+workloads below, and bf16 rounding of the drawn values.
+
+Workloads (token-major activations X[T, C], weights W[G, R, C]):
+
+* ``tiny``  : X fp32 [256, 64] ~ N(0, 1); W fp32 [32, 64] ~ N(0, 0.02^2); full H.
+* ``dense`` : X bf16 [16384, 4096], per-column std sigma_i = exp(N(0, 1)) with
+  round(1% of C) distinct columns (chosen uniformly) multiplied by 20;
+  W bf16 [4096, 4096] ~ N(0, (1/sqrt(4096))^2); full H.
+* ``act``   : X as ``dense`` at [32768, 4096]; X_q = NVFP4 max fake-quant of X
+  (see ``nvfp4_act_fake_quant``); W bf16 [12288, 4096]; activation-aware H and P.
+* ``wmse``  : X bf16 [65536, 12288], sigma_i = exp(N(0, 1.5^2)), no outliers;
+  W bf16 [4096, 12288] ~ N(0, 1/12288); diagonal importance.
+* ``moe``   : X bf16 [16384, 2560] drawn as ``dense``; each token routed to 10
+  distinct experts of 512 chosen uniformly; CSR sorted by expert with token ids
+  ascending; W bf16 [512, 1280, 2560] ~ N(0, 1/2560); grouped full H with a
+  global scale per expert.
+
+The pages name the workloads' shapes and distributions but never the
+calibration data itself, so these draws stand in for captured activations.
+
+Random numbers come from numpy PCG64 streams, one per 2^22-element chunk and per
+tensor tag, seeded by ``SeedSequence([seed, tag, chunk])``; chunks are filled on
+a thread pool, so the values do not depend on the thread count.
+"""
+from __future__ import annotations
+
+import os
+from concurrent.futures import ThreadPoolExecutor
+from dataclasses import dataclass, field
+
+import numpy as np
+
+CHUNK = 1 << 22
+_TAGS = {"sigma": 1, "outlier": 2, "x": 3, "w": 4, "route": 5}
+
+WORKLOADS = ("tiny", "dense", "act", "wmse", "moe")
+
+# Full sizes of each workload: (tokens, cin, rows, groups).
+FULL_SIZES = {
+    "tiny": (256, 64, 32, 1),
+    "dense": (16384, 4096, 4096, 1),
+    "act": (32768, 4096, 12288, 1),
+    "wmse": (65536, 12288, 4096, 1),
+    "moe": (16384, 2560, 1280, 512),
+}
+MODES = {"tiny": "full", "dense": "full", "act": "act", "wmse": "diag", "moe": "full"}
+MOE_TOP_K = 10
+
+
+def _pool():
+    return ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1))
+
+
+def _normal_f32(n: int, seed: int, tag: str) -> np.ndarray:
+    """n standard normal float32 draws, chunked into independent streams."""
+    out = np.empty(n, dtype=np.float32)
+    nchunks = (n + CHUNK - 1) // CHUNK
+
+    def fill(i):
+        g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, _TAGS[tag], i])))
+        lo, hi = i * CHUNK, min(n, (i + 1) * CHUNK)
+        g.standard_normal(out=out[lo:hi], dtype=np.float32)
+
+    if nchunks == 1:
+        fill(0)
+    else:
+        with _pool() as ex:
+            list(ex.map(fill, range(nchunks)))
+    return out
+
+
+def _rng(seed: int, tag: str) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, _TAGS[tag], 0])))
+
+
+def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """Round float32 to bfloat16 (nearest, ties to even); returns uint16 bit patterns.
+
+    Inputs are finite by construction, so NaN handling is not needed.
+    """
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    u = a.view(np.uint32)
+    out = np.empty(u.shape, dtype=np.uint16)
+    flat_u, flat_o = u.reshape(-1), out.reshape(-1)
+
+    def rnd(lo_hi):
+        lo, hi = lo_hi
+        v = flat_u[lo:hi]
+        r = v + np.uint32(0x7FFF) + ((v >> np.uint32(16)) & np.uint32(1))
+        flat_o[lo:hi] = (r >> np.uint32(16)).astype(np.uint16)
+
+    spans = [(i, min(flat_u.size, i + CHUNK)) for i in range(0, flat_u.size, CHUNK)]
+    if len(spans) <= 1:
+        for s in spans:
+            rnd(s)
+    else:
+        with _pool() as ex:
+            list(ex.map(rnd, spans))
+    return out
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    """Widen bfloat16 bit patterns to float32 exactly."""
+    return (np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def _scaled_columns(tokens: int, cin: int, sigma: np.ndarray, seed: int) -> np.ndarray:
+    z = _normal_f32(tokens * cin, seed, "x").reshape(tokens, cin)
+    # Multiply in place chunk by chunk to bound temporaries.
+    rows_per = max(1, CHUNK // max(cin, 1))
+    spans = [(r, min(tokens, r + rows_per)) for r in range(0, tokens, rows_per)]
+
+    def mul(span):
+        lo, hi = span
+        z[lo:hi] *= sigma[None, :]
+
+    with _pool() as ex:
+        list(ex.map(mul, spans))
+    return z
+
+
+def _column_sigma(cin: int, seed: int, log_std: float, outlier_frac: float) -> np.ndarray:
+    sigma = np.exp(_rng(seed, "sigma").normal(0.0, log_std, size=cin)).astype(np.float32)
+    n_out = int(round(outlier_frac * cin))
+    if n_out:
+        cols = _rng(seed, "outlier").choice(cin, size=n_out, replace=False)
+        sigma[cols] *= np.float32(20.0)
+    return sigma
+
+
+# --- activation quantizer for the ``act`` workload (input data, not the method) ---------
+
+_E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def _e4m3_round_positive(x: np.ndarray) -> np.ndarray:
+    """Nearest E4M3 value (ties to even), saturating at 448, for x >= 0 (fp64)."""
+    x = np.minimum(np.asarray(x, dtype=np.float64), 448.0)
+    out = np.zeros_like(x)
+    nz = x > 0
+    xe = x[nz]
+    # E4M3: 3 mantissa bits, min normal 2^-6, subnormal step 2^-9.
+    _, ex = np.frexp(xe)  # xe = m * 2^ex with m in [0.5, 1): floor(log2 xe) = ex - 1
+    e = np.maximum(ex.astype(np.float64) - 1.0, -6.0)
+    step = np.exp2(e - 3.0)
+    q = xe / step
+    fl = np.floor(q)
+    frac = q - fl
+    up = (frac > 0.5) | ((frac == 0.5) & (np.mod(fl, 2.0) == 1.0))
+    out[nz] = np.minimum((fl + up) * step, 448.0)
+    return out
+
+
+def _e2m1_round(u: np.ndarray) -> np.ndarray:
+    u = np.minimum(u, 6.0)
+    d = np.abs(u[..., None] - _E2M1_GRID)
+    best = d.min(axis=-1, keepdims=True)
+    tie_ok = d == best
+    # Among equally near grid points take the one with an even code (index).
+    even_ok = tie_ok & (np.arange(8) % 2 == 0)
+    idx = np.where(even_ok.any(-1), np.argmax(even_ok, -1), np.argmax(tie_ok, -1))
+    return _E2M1_GRID[idx]
+
+
+def nvfp4_act_fake_quant(x_bits: np.ndarray) -> np.ndarray:
+    """NVFP4 max fake-quant of bf16 activations X[T, C]; returns bf16 bits of X_q.
+
+    Per-tensor global scale gx = fp32(amax|X| / 2688); per (token, 16-wide block)
+    scale = E4M3(amax_blk / (6 gx)) * gx in fp32; each value rounds to E2M1
+    (nearest, ties to even, clamped at 6) and is rescaled, keeping its sign.
+    This only produces input data for the activation-aware workload.
+    """
+    x = bf16_bits_to_f32(x_bits).astype(np.float64)
+    t, c = x.shape
+    gx = np.float32(np.abs(x).max() / 2688.0)
+    out = np.empty((t, c), dtype=np.uint16)
+    rows_per = max(1, (1 << 18) // c)
+
+    def one(span):
+        lo, hi = span
+        xb = x[lo:hi].reshape(hi - lo, c // 16, 16)
+        amax_blk = np.abs(xb).max(-1)
+        if gx > 0:
+            code = _e4m3_round_positive(amax_blk / (6.0 * np.float64(gx)))
+        else:
+            code = np.zeros_like(amax_blk)
+        s = (code * np.float64(gx)).astype(np.float32).astype(np.float64)[..., None]
+        with np.errstate(divide="ignore", invalid="ignore"):
+            u = np.where(s > 0, np.abs(xb) / np.where(s > 0, s, 1.0), 0.0)
+        q = _e2m1_round(u)
+        xq = np.copysign((q * s).astype(np.float32), xb.astype(np.float32))
+        out[lo:hi] = f32_to_bf16_bits(xq.reshape(hi - lo, c))
+
+    spans = [(r, min(t, r + rows_per)) for r in range(0, t, rows_per)]
+    with _pool() as ex:
+        list(ex.map(one, spans))
+    return out
+
+
+# --- workloads ------------------------------------------------------------------------------
+
+
+@dataclass
+class Layer:
+    """One synthetic layer. bf16 tensors are uint16 bit patterns."""
+
+    name: str
+    mode: str  # "full" | "act" | "diag"
+    dtype: str  # "f32" | "bf16"
+    x: np.ndarray  # [T, C]
+    w: np.ndarray  # [G, R, C]
+    xq: np.ndarray | None = None
+    group_offsets: np.ndarray | None = None  # int32 [G + 1]
+    token_ids: np.ndarray | None = None  # int32 [group_offsets[-1]]
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def tokens(self) -> int:
+        return int(self.x.shape[0])
+
+    @property
+    def cin(self) -> int:
+        return int(self.x.shape[1])
+
+    @property
+    def groups(self) -> int:
+        return int(self.w.shape[0])
+
+    @property
+    def rows(self) -> int:
+        return int(self.w.shape[1])
+
+    def x_f32(self) -> np.ndarray:
+        return self.x if self.dtype == "f32" else bf16_bits_to_f32(self.x)
+
+    def xq_f32(self) -> np.ndarray:
+        return bf16_bits_to_f32(self.xq)
+
+    def w_f32(self) -> np.ndarray:
+        return self.w if self.dtype == "f32" else bf16_bits_to_f32(self.w)
+
+
+def moe_routing(tokens: int, experts: int, top_k: int, seed: int):
+    """Uniform top-k routing: each token picks top_k distinct experts.
+
+    Returns CSR (offsets[experts + 1], token ids sorted by expert, ascending within).
+    """
+    g = _rng(seed, "route")
+    keys = g.random((tokens, experts), dtype=np.float32) if experts > 1 else np.zeros((tokens, 1), np.float32)
+    top_k = min(top_k, experts)
+    picks = np.argpartition(keys, top_k - 1, axis=1)[:, :top_k] if top_k < experts else np.tile(np.arange(experts), (tokens, 1))
+    exp_flat = picks.reshape(-1).astype(np.int64)
+    tok_flat = np.repeat(np.arange(tokens, dtype=np.int64), top_k)
+    order = np.lexsort((tok_flat, exp_flat))
+    token_ids = tok_flat[order].astype(np.int32)
+    counts = np.bincount(exp_flat, minlength=experts)
+    offsets = np.zeros(experts + 1, dtype=np.int32)
+    offsets[1:] = np.cumsum(counts)
+    return offsets, token_ids
+
+
+def make_layer(name: str, seed: int = 0, tokens: int | None = None, cin: int | None = None,
+               rows: int | None = None, groups: int | None = None, top_k: int = MOE_TOP_K) -> Layer:
+    """Build workload ``name`` at its full size, or at the given smaller sizes."""
+    if name not in FULL_SIZES:
+        raise ValueError(f"unknown workload {name!r}")
+    T0, C0, R0, G0 = FULL_SIZES[name]
+    T = T0 if tokens is None else tokens
+    C = C0 if cin is None else cin
+    R = R0 if rows is None else rows
+    G = G0 if groups is None else groups
+    if C % 16:
+        raise ValueError("cin must be a multiple of 16")
+    mode = MODES[name]
+    if name == "tiny":
+        x = _normal_f32(T * C, seed, "x").reshape(T, C)
+        w = (_normal_f32(G * R * C, seed, "w") * np.float32(0.02)).reshape(G, R, C)
+        return Layer(name, mode, "f32", x, w)
+    log_std, outl = (1.5, 0.0) if name == "wmse" else (1.0, 0.01)
+    sigma = _column_sigma(C, seed, log_std, outl)
+    xf = _scaled_columns(T, C, sigma, seed)
+    x = f32_to_bf16_bits(xf)
+    del xf
+    wf = _normal_f32(G * R * C, seed, "w").reshape(G, R, C)
+    wf *= np.float32(1.0 / np.sqrt(C))
+    w = f32_to_bf16_bits(wf)
+    del wf
+    layer = Layer(name, mode, "bf16", x, w, meta={"sigma": sigma})
+    if name == "act":
+        layer.xq = nvfp4_act_fake_quant(x)
+    if name == "moe":
+        layer.group_offsets, layer.token_ids = moe_routing(T, G, top_k, seed)
+    return layer

@@ -1,0 +1,267 @@
+"""Pins for the CPU oracle: format facts, closed forms, brute force and invariants.
+
+Each test ties the oracle to something other than itself: a library's own
+number-format conversion, exact rational arithmetic, an identity the pages
+state, or a brute-force evaluation on a tiny input.
+"""
+from fractions import Fraction
+
+import ml_dtypes
+import numpy as np
+import pytest
+import torch
+
+from oracle import lhcal_oracle as O
+
+E2M1 = [Fraction(v) for v in (0, 0.5, 1, 1.5, 2, 3, 4, 6)]
+
+
+# --------------------------------------------------------------------------- formats
+
+def test_e4m3_candidates_match_torch_float8():
+    codes = O.candidate_codes()
+    assert len(codes) == 126 and codes[0] == 1 and codes[-1] == 0x7E
+    lib = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    np.testing.assert_array_equal(O.e4m3_value(codes), lib[codes])
+    v = O.e4m3_value(codes)
+    assert np.all(np.diff(v) > 0)
+    assert v[0] == 2.0 ** -9 and v[-1] == 448.0
+    # The set is every positive finite non-zero E4M3 value.
+    finite = lib[np.isfinite(lib) & (lib > 0)]
+    assert sorted(finite.tolist()) == v.tolist()
+
+
+@pytest.mark.parametrize("u,q", [(0.25, 0), (0.75, 1), (1.25, 1), (1.75, 2), (2.5, 2), (3.5, 4), (5.0, 4),
+                                 (6.0, 6), (7.0, 6), (100.0, 6), (0.0, 0), (0.2499, 0), (0.2501, 0.5)])
+def test_e2m1_midpoints_ties_to_even(u, q):
+    assert O.e2m1_round(np.array([u]))[0] == q
+
+
+def test_e2m1_matches_ml_dtypes_on_fp32_values():
+    rng = np.random.default_rng(1)
+    u = np.concatenate([rng.uniform(0, 8, 200000), np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])])
+    u = u.astype(np.float32)
+    lib = u.astype(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    np.testing.assert_array_equal(O.e2m1_round(u.astype(np.float64)), lib)
+
+
+def _fq_exact(w: float, s: float) -> float:
+    """Fake quant by exact rationals: nearest grid point to |w|/s, ties to even code."""
+    if s == 0:
+        return float(np.copysign(0.0, w))
+    u = min(Fraction(abs(w)) / Fraction(s), Fraction(6))
+    d = [abs(u - g) for g in E2M1]
+    m = min(d)
+    idx = [i for i, x in enumerate(d) if x == m]
+    i = idx[0] if len(idx) == 1 else [j for j in idx if j % 2 == 0][0]
+    mag = np.float32(float(E2M1[i] * Fraction(s)))  # exact product rounded once to fp32
+    return float(np.copysign(mag, w))
+
+
+def test_fake_quant_exact_ties_and_neighbours():
+    # s with few mantissa bits so m * s is an exact fp32 midpoint.
+    rng = np.random.default_rng(2)
+    ws, ss = [], []
+    for s in (np.float32(0.0078125), np.float32(3.0 * 2 ** -12), np.float32(0.1)):
+        for m in (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0):
+            t = np.float32(m * float(s))
+            for w in (t, np.nextafter(t, np.float32(0)), np.nextafter(t, np.float32(1))):
+                for sign in (1, -1):
+                    ws.append(np.float32(sign * w))
+                    ss.append(s)
+    ws += list(rng.normal(0, 0.05, 2000).astype(np.float32))
+    ss += list(np.float32(rng.uniform(1e-4, 1e-2, 2000)))
+    ws, ss = np.array(ws, np.float32), np.array(ss, np.float32)
+    got = O.fake_quant(ws, ss)
+    want = np.array([_fq_exact(float(w), float(s)) for w, s in zip(ws, ss)], np.float32)
+    np.testing.assert_array_equal(got.view(np.int32), want.view(np.int32))
+
+
+def test_fake_quant_negative_zero_and_zero_scale():
+    out = O.fake_quant(np.array([-1e-6, 1e-6, -0.5], np.float32), np.float32(1.0))
+    assert out.view(np.int32)[0] == np.float32(-0.0).view(np.int32)
+    assert out[1] == 0.0 and out[2] == -0.5
+    z = O.fake_quant(np.array([0.3, -0.3], np.float32), np.float32(0.0))
+    assert z.view(np.int32).tolist() == [0, np.float32(-0.0).view(np.int32)]
+
+
+def test_global_scale_is_448_normalized():
+    w = np.array([[0.5, -1.75, 0.25]], np.float32)
+    assert O.global_scale(w) == np.float32(1.75 / 2688.0)
+    s = O.candidate_scales(O.global_scale(w))
+    # The largest candidate maps amax onto the top of the FP4 grid: 448 * g * 6 ~ amax.
+    assert abs(float(s[-1]) * 6 - 1.75) < 1e-6
+    assert O.global_scale(np.zeros((2, 3), np.float32)) == 0.0
+
+
+# --------------------------------------------------------------------------- Hessians
+
+def _tiny_x(t=7, c=32, seed=3):
+    return np.random.default_rng(seed).normal(size=(t, c)).astype(np.float32)
+
+
+def test_full_hessian_brute_force():
+    x = _tiny_x()
+    h = O.hessian_sum_full(x)
+    for n in range(2):
+        for i in range(16):
+            for j in range(16):
+                ref = sum(Fraction(float(x[t, 16 * n + i])) * Fraction(float(x[t, 16 * n + j])) for t in range(x.shape[0]))
+                assert abs(h[n, i, j] - float(ref)) <= 1e-12 * max(1.0, abs(float(ref)))
+
+
+def test_act_hessians_brute_force_and_properties():
+    x = _tiny_x(9, 32, 4)
+    xq = (x + np.random.default_rng(5).normal(0, 0.1, x.shape)).astype(np.float32)
+    h, p = O.hessian_sum_act(x, xq)
+    for n, i, j in [(0, 0, 0), (0, 3, 11), (1, 15, 2), (1, 7, 7)]:
+        refh = sum(float(xq[t, 16 * n + i]) * float(xq[t, 16 * n + j]) for t in range(9))
+        refp = sum(float(xq[t, 16 * n + i]) * (float(xq[t, 16 * n + j]) - float(x[t, 16 * n + j])) for t in range(9))
+        assert abs(h[n, i, j] - refh) < 1e-12 and abs(p[n, i, j] - refp) < 1e-12
+    assert not np.allclose(p, p.transpose(0, 2, 1))  # P is not symmetric: its index order matters
+    h0, p0 = O.hessian_sum_act(x, x)
+    assert np.all(p0 == 0.0)
+    np.testing.assert_array_equal(h0, O.hessian_sum_full(x))
+
+
+def test_hessian_symmetric_psd_and_diag_is_importance():
+    x = _tiny_x(40, 64, 6)
+    h = O.hessian_sum_full(x)
+    np.testing.assert_array_equal(h, h.transpose(0, 2, 1))
+    ev = np.linalg.eigvalsh(h)
+    assert ev.min() >= -1e-12 * np.abs(ev).max()
+    np.testing.assert_allclose(np.diagonal(h, axis1=1, axis2=2), O.importance_sum(x), rtol=1e-14)
+
+
+def test_grouped_accumulate_and_zero_group_fallback():
+    x = _tiny_x(12, 32, 7)
+    off = np.array([0, 3, 3, 8], np.int32)
+    ids = np.array([0, 5, 11, 1, 2, 3, 4, 9], np.int32)
+    h, _, counts = O.accumulate("full", x, group_offsets=off, token_ids=ids)
+    assert counts.tolist() == [3, 0, 5]
+    np.testing.assert_array_equal(h[0], O.hessian_sum_full(x[[0, 5, 11]]))
+    np.testing.assert_array_equal(h[2], O.hessian_sum_full(x[[1, 2, 3, 4, 9]]))
+    assert np.all(h[1] == 0)
+    hf, _ = O.finalize("full", h, None, counts)
+    np.testing.assert_array_equal(hf[1], np.broadcast_to(np.eye(16), (2, 16, 16)))
+    np.testing.assert_allclose(hf[2], h[2] / 5.0, rtol=1e-15)
+    hd, _, cd = O.accumulate("diag", x, group_offsets=off, token_ids=ids)
+    hdf, _ = O.finalize("diag", hd, None, cd)
+    assert np.all(hdf[1] == 1.0)
+    np.testing.assert_array_equal(hdf[0], hd[0])  # importance stays a raw sum
+
+
+# --------------------------------------------------------------------------- losses and sweep
+
+def _layer(seed, rows=6, cin=16, t=64):
+    rng = np.random.default_rng(seed)
+    x = rng.normal(size=(t, cin)).astype(np.float32) * rng.lognormal(0, 1, cin).astype(np.float32)
+    w = rng.normal(0, 0.05, (1, rows, cin)).astype(np.float32)
+    return x, w
+
+
+def test_act_expanded_loss_equals_output_mse_including_negative():
+    """On one block (cin = 16): L_k + w^T D^T D w / B == ||X_q wq_k - X w||^2 / B for every k."""
+    x, w = _layer(8, rows=1)
+    t = x.shape[0]
+    g = O.global_scale(w[0])
+    s = O.candidate_scales(g)
+    # X_q = 0.9 X and w chosen so that one candidate's quantized weights equal w / 0.9:
+    # the output error then vanishes and the expanded objective is negative there.
+    k0 = 100
+    qv = np.array([6, 4, 3, 2, 1.5, 1, 0.5, 6, 4, 3, 2, 1.5, 1, 0.5, 6, 4], np.float64)
+    sign = np.where(np.arange(16) % 3 == 0, -1.0, 1.0)
+    wrow = (0.9 * qv * float(s[k0]) * sign).astype(np.float32)
+    xq = (0.9 * x.astype(np.float64)).astype(np.float32)
+    for wr in (w[0, 0], wrow):
+        hs, ps = O.hessian_sum_act(x, xq)
+        h, p = hs[0] / t, ps[0] / t
+        loss, wq, _ = O.candidate_losses("act", wr[None], h[None], p[None], g)
+        d = xq.astype(np.float64) - x.astype(np.float64)
+        const = float(np.sum((d @ wr.astype(np.float64)) ** 2)) / t
+        for k in range(126):
+            out = xq.astype(np.float64) @ wq[0, k].astype(np.float64) - x.astype(np.float64) @ wr.astype(np.float64)
+            mse = float(np.sum(out ** 2)) / t
+            assert abs(loss[0, k] + const - mse) <= 1e-9 * max(mse, const, 1e-30)
+    assert loss[0, k0] < 0  # the deliberately negative objective of the last row
+
+
+def test_act_with_xq_equal_x_is_local_hessian():
+    x, w = _layer(9, rows=20, cin=48)
+    full = O.calibrate("full", x, w)
+    act = O.calibrate("act", x, w, xq=x)
+    np.testing.assert_array_equal(full["codes"], act["codes"])
+    np.testing.assert_array_equal(full["wq"].view(np.int32), act["wq"].view(np.int32))
+    np.testing.assert_array_equal(full["loss"], act["loss"])
+
+
+def test_wmse_equals_full_with_diagonal_hessian():
+    x, w = _layer(10, rows=20, cin=48)
+    d = O.calibrate("diag", x, w)
+    imp = O.importance_sum(x)[None]
+    hdiag = np.zeros((1, imp.shape[1], 16, 16))
+    hdiag[0, :, np.arange(16), np.arange(16)] = imp[0].T
+    f = O.sweep("full", w, hdiag, None, d["g"])
+    np.testing.assert_array_equal(f["codes"], d["codes"])
+    np.testing.assert_allclose(f["loss"], d["loss"], rtol=1e-13)
+
+
+def test_identity_hessian_is_plain_block_mse_by_exact_rationals():
+    _, w = _layer(11, rows=3, cin=16)
+    g = O.global_scale(w[0])
+    s = O.candidate_scales(g)
+    h = np.eye(16)[None].repeat(3, 0)
+    loss, _, _ = O.candidate_losses("full", w[0], h, None, g)
+    for r in range(3):
+        for k in range(0, 126, 5):
+            ref = sum((Fraction(_fq_exact(float(wi), float(s[k]))) - Fraction(float(wi))) ** 2 for wi in w[0, r])
+            assert abs(loss[r, k] - float(ref)) <= 1e-12 * float(ref)
+
+
+def test_sweep_is_exhaustive_lowest_code_on_ties():
+    x, w = _layer(12, rows=8, cin=32)
+    hs, _, c = O.accumulate("full", x)
+    h, _ = O.finalize("full", hs, None, c)
+    g = np.array([O.global_scale(w[0])], np.float32)
+    out = O.sweep("full", w, h, None, g)
+    losses = O.sweep("full", w, h, None, g)["all_losses"] if "all_losses" in out else None
+    for u, (r, n) in enumerate([(r, n) for r in range(8) for n in range(2)]):
+        wb = w[0, r, 16 * n:16 * n + 16]
+        all_l, _, _ = O.candidate_losses("full", wb[None], h[0, n][None], None, g[0])
+        brute = min(range(126), key=lambda k: (all_l[0, k], k))
+        assert out["codes"][u] == brute + 1
+        assert out["loss"][u] == all_l[0, brute]
+    assert losses is None or losses.shape[1] == 126
+    # An all-zero block ties every candidate: code 1 wins.
+    w0 = w.copy()
+    w0[0, 0, :16] = 0
+    z = O.sweep("full", w0, h, None, g)
+    assert z["codes"][0] == 1 and z["loss"][0] == 0.0
+
+
+def test_sweep_invariances():
+    x, w = _layer(13, rows=16, cin=32)
+    hs, _, c = O.accumulate("full", x)
+    h, _ = O.finalize("full", hs, None, c)
+    g = np.array([O.global_scale(w[0])], np.float32)
+    base = O.sweep("full", w, h, None, g)
+    scaled = O.sweep("full", w, 4.0 * h, None, g)
+    np.testing.assert_array_equal(base["codes"], scaled["codes"])
+    np.testing.assert_allclose(scaled["loss"], 4.0 * base["loss"], rtol=1e-14)
+    neg = O.sweep("full", -w, h, None, g)
+    np.testing.assert_array_equal(base["codes"], neg["codes"])
+    np.testing.assert_array_equal(base["wq"], -neg["wq"])
+    np.testing.assert_allclose(neg["loss"], base["loss"], rtol=1e-14)
+    perm = np.random.default_rng(0).permutation(16)
+    wp = w.copy()
+    wp[0, :, :16] = w[0, :, :16][:, perm]
+    hp = h.copy()
+    hp[0, 0] = h[0, 0][np.ix_(perm, perm)]
+    pb = O.sweep("full", wp, hp, None, g)
+    np.testing.assert_array_equal(pb["codes"], base["codes"])
+    np.testing.assert_allclose(pb["loss"], base["loss"], rtol=1e-12)
+    imp = np.random.default_rng(1).uniform(0.5, 2, (1, 2, 16))
+    d1 = O.sweep("diag", w, imp, None, g)
+    d2 = O.sweep("diag", -w, imp, None, g)
+    np.testing.assert_array_equal(d1["codes"], d2["codes"])
+    np.testing.assert_array_equal(d1["loss"], d2["loss"])
