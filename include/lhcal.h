@@ -1,0 +1,162 @@
+/*
+ * lhcal.h - C ABI of liblhcal.so: local-Hessian NVFP4 weight-scale calibration on B200 (sm_100a).
+ *
+ * The method (NVIDIA Model-Optimizer pull requests, cited by page title and section):
+ *   - "add local hessian calibration" (PR #788), Overview: weight-scale candidates are
+ *     weighed by a per-16-wide-input-block Hessian H_n = X_b^T X_b / B.
+ *   - "Add activation-aware local Hessian scale calibration" (PR #1976), "What does this PR
+ *     do?": H = X_q^T X_q / B, P = X_q^T (X_q - X) / B and the loss dW^T H dW + 2 dW^T (P W0),
+ *     dW = quant(w) - w; the reviews: losses may be negative, best loss starts at +inf,
+ *     kernels validate device placement and sizes.
+ *   - "Add WMSE weight scale search calibration" (PR #2283), "What"/"How": Imp_i = ||X[:,i]||^2
+ *     kept as [n_blocks, 16], loss sum_i Imp_i dW_i^2, 126 candidate E4M3 block scales.
+ *   - "Add composable scale calibration to GPTQ" (PR #2004): 448-normalized NVFP4 scaling,
+ *     g = amax / (6 * 448).
+ *   - "[2/3] Speed up layerwise GPTQ on MoE models" (PR #2864), embedded #2840 description:
+ *     per-expert Hessians over the tokens routed to each expert; an expert that no token
+ *     reaches gets the plain search. Embedded #2877: launch on the tensors' own device.
+ *
+ * Conventions for every call:
+ *   - All tensors are caller-owned device memory on the CURRENT device; the library keeps
+ *     no state across calls, allocates nothing and never synchronises. Work is enqueued on
+ *     `stream` (a cudaStream_t; NULL = legacy default stream) and runs asynchronously.
+ *   - Sizes are element counts. Row-major, C order. cin must be a positive multiple of 16.
+ *   - Status codes: LHCAL_ERR_INVALID_ARG for a null/misaligned pointer, a bad size or a
+ *     host pointer where device memory is required; LHCAL_ERR_DEVICE_MISMATCH for memory of
+ *     another device than the current one; LHCAL_ERR_UNSUPPORTED for an unknown mode/dtype;
+ *     LHCAL_ERR_CUDA when a launch fails (the CUDA error string is kept). On any error
+ *     nothing is enqueued, except for LHCAL_ERR_CUDA, where earlier launches of the same
+ *     call may have been enqueued. lhcal_last_error_string() describes the last error of
+ *     the calling thread.
+ *   - Inputs must be finite; results for NaN/Inf inputs are unspecified.
+ */
+#ifndef LHCAL_H_
+#define LHCAL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LHCAL_OK = 0,
+  LHCAL_ERR_INVALID_ARG = 1,
+  LHCAL_ERR_UNSUPPORTED = 2,
+  LHCAL_ERR_DEVICE_MISMATCH = 3,
+  LHCAL_ERR_CUDA = 4,
+  LHCAL_ERR_TIMEOUT = 5 /* reserved for bounded device waits; no current kernel waits */
+} lhcal_status;
+
+typedef enum { LHCAL_F32 = 0, LHCAL_BF16 = 1 } lhcal_dtype;
+
+typedef enum {
+  LHCAL_FULL = 0,      /* H_n = X_b^T X_b / B                      (PR #788)  */
+  LHCAL_ACT_AWARE = 1, /* H = X_q^T X_q / B, P = X_q^T (X_q - X) / B (PR #1976) */
+  LHCAL_DIAG = 2       /* Imp_i = ||X[:, i]||^2                      (PR #2283) */
+} lhcal_mode;
+
+/* lhcal_accumulate flags. */
+#define LHCAL_ACCUM_ADD 0       /* h (and p) += this call's sums                  */
+#define LHCAL_ACCUM_OVERWRITE 1 /* h (and p) = this call's sums (no read of h / p) */
+
+/* Number of 126 candidate block scales (E4M3 codes 0x01..0x7E), PR #2283 "How". */
+#define LHCAL_N_CANDIDATES 126
+#define LHCAL_BLOCK 16
+
+/*
+ * Bytes of workspace lhcal_accumulate needs for these sizes (0 is possible). Host-only
+ * computation; needs no GPU. groups > 1 (grouped) needs none.
+ */
+lhcal_status lhcal_accumulate_workspace(lhcal_mode mode, lhcal_dtype dtype, int64_t tokens,
+                                        int64_t cin, int32_t groups, size_t* bytes);
+
+/*
+ * Hessian accumulation (raw sums, no 1/B), PR #788 Overview, PR #1976, PR #2283 "How".
+ *   x, xq   : [tokens, cin] activations, row stride ldx elements (ldx >= cin, ldx * element
+ *             size a multiple of 16 bytes, base 16-byte aligned). xq only for ACT_AWARE
+ *             (the input quantizer's output), else NULL.
+ *   groups  : 1 with group_offsets = token_ids = NULL sums over all rows of x. Grouped
+ *             (fused-MoE experts, PR #2864 / #2840): group_offsets [groups + 1] (device,
+ *             non-decreasing, offsets[0] = 0) and token_ids [offsets[groups]] (device,
+ *             each in [0, tokens)); group e sums rows token_ids[offsets[e] .. offsets[e+1]).
+ *   h       : FULL/ACT: [groups, cin/16, 16, 16] fp32, h[e][n][i][j] = sum x_{t,16n+i} x_{t,16n+j}
+ *             (x = xq for ACT). DIAG: [groups, cin/16, 16] fp32 sum of squares per column.
+ *   p       : ACT only: [groups, cin/16, 16, 16], p[e][n][i][j] = sum xq_{t,16n+i} (xq - x)_{t,16n+j};
+ *             NULL otherwise.
+ *   flags   : LHCAL_ACCUM_ADD or LHCAL_ACCUM_OVERWRITE.
+ *   workspace: device scratch of at least lhcal_accumulate_workspace() bytes, 256-byte
+ *             aligned; may be NULL when that size is 0. Its contents need no initialisation.
+ * Results are deterministic for fixed sizes (fixed summation order). bf16 products are exact
+ * in fp32; sums are fp32.
+ */
+lhcal_status lhcal_accumulate(lhcal_mode mode, lhcal_dtype dtype, const void* x, const void* xq,
+                              int64_t tokens, int64_t cin, int64_t ldx, int32_t groups,
+                              const int32_t* group_offsets, const int32_t* token_ids, int32_t flags,
+                              float* h, float* p, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Token counts B per group: counts[e] (+)= offsets[e+1] - offsets[e], or counts[0] (+)= tokens
+ * when group_offsets is NULL (groups must then be 1). counts: device int64 [groups].
+ * flags as for lhcal_accumulate.
+ */
+lhcal_status lhcal_count_tokens(int32_t groups, int64_t tokens, const int32_t* group_offsets,
+                                int32_t flags, int64_t* counts, void* stream);
+
+/*
+ * Finalisation in place (PR #1976: "/B"; PR #2864 / #2840: zero-token fallback).
+ *   FULL/ACT: h /= counts[e], p /= counts[e] (IEEE fp32 division).
+ *   DIAG: Imp is left as the raw sum (PR #2283).
+ *   counts[e] == 0: h := I (DIAG: Imp := 1) and p := 0, i.e. the plain block-MSE search.
+ *   counts: device int64 [groups]; h, p laid out as in lhcal_accumulate (p NULL unless ACT).
+ */
+lhcal_status lhcal_finalize(lhcal_mode mode, int32_t groups, int64_t cin, const int64_t* counts,
+                            float* h, float* p, void* stream);
+
+/*
+ * Global scale per group (PR #2004: 448-normalized): g[e] = fp32(max |W_e| / 2688), the
+ * maximum taken exactly and divided with IEEE round-to-nearest.
+ *   w: [groups, rows, cin] (fp32 or bf16), 16-byte aligned. g: device fp32 [groups].
+ */
+lhcal_status lhcal_global_scale(lhcal_dtype dtype, const void* w, int32_t groups, int64_t rows,
+                                int64_t cin, float* g, void* stream);
+
+/*
+ * Exhaustive FP8 scale sweep (PR #2283 "How", PR #1976 reviews). For each unit (e, r, n):
+ *   for code k = 1..126: s_k = fp32(v_k * g[e]) with v_k the E4M3 value of k;
+ *     q_i = E2M1 round-to-nearest-even of the exact |w_i| / s_k, clamped at 6;
+ *     wq_i = copysign(fp32(q_i * s_k), w_i); dW = wq - w;
+ *     L_k = dW^T H_n dW (FULL), + 2 dW^T (P_n w) (ACT), or sum_i Imp_{n,i} dW_i^2 (DIAG);
+ *   k* = the lowest k with the smallest L_k (losses may be negative).
+ * Decisions on the quotient are exact for g >= 2^-90 or g == 0 (g == 0 gives wq = +-0 and
+ * code 1). Losses are evaluated in fp32.
+ *   w     : [groups, rows, cin] fp32 or bf16, 16-byte aligned.
+ *   h     : FULL/ACT: [groups, cin/16, 16, 16] finalized H; DIAG: [groups, cin/16, 16] Imp.
+ *   p     : ACT: [groups, cin/16, 16, 16] finalized P; else NULL.
+ *   g     : device fp32 [groups].
+ *   codes : out [groups, rows, cin/16] uint8, the E4M3 bit pattern of the chosen scale.
+ *   wq    : out [groups, rows, cin] fp32 fake-quantized weights (16-byte aligned), or NULL.
+ *   loss  : out [groups, rows, cin/16] fp32 winning loss, or NULL.
+ */
+lhcal_status lhcal_scale_sweep(lhcal_mode mode, lhcal_dtype dtype, const void* w, int32_t groups,
+                               int64_t rows, int64_t cin, const float* h, const float* p,
+                               const float* g, uint8_t* codes, float* wq, float* loss, void* stream);
+
+/*
+ * Number of kernels this library enqueued from the calling thread since the last reset
+ * (reset != 0 returns the count and sets it to zero). Host-side bookkeeping only.
+ */
+int64_t lhcal_launch_count(int32_t reset);
+
+/* Message for the calling thread's last non-OK status ("" if none). */
+const char* lhcal_last_error_string(void);
+
+/* ABI version of this header (major * 100 + minor). */
+int32_t lhcal_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LHCAL_H_ */

@@ -1,0 +1,244 @@
+"""Python binding of liblhcal.so (local-Hessian NVFP4 weight-scale calibration on B200).
+
+Argument marshalling only: every step runs in the CUDA library. Functions carry the C
+names (``lhcal_accumulate`` ...) and take torch tensors, passing their device pointers,
+sizes and the current CUDA stream. A missing or unloadable library raises at import of
+the first call; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "liblhcal.so")
+
+# lhcal_status
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_DEVICE_MISMATCH, ERR_CUDA, ERR_TIMEOUT = range(6)
+STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "DEVICE_MISMATCH", 4: "CUDA", 5: "TIMEOUT"}
+# lhcal_dtype / lhcal_mode / flags
+F32, BF16 = 0, 1
+FULL, ACT_AWARE, DIAG = 0, 1, 2
+ACCUM_ADD, ACCUM_OVERWRITE = 0, 1
+N_CANDIDATES = 126
+BLOCK = 16
+MODE_IDS = {"full": FULL, "act": ACT_AWARE, "diag": DIAG}
+
+_lib = None
+
+
+class LhcalError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"lhcal {STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load liblhcal.so (built by ``python -m scale_calibration_lh_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"liblhcal.so not found at {path}; build it with "
+                           "`python -m scale_calibration_lh_b200.build`")
+    lib = ctypes.CDLL(path)
+    i32, i64, vp, sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t
+    sigs = {
+        "lhcal_accumulate_workspace": [i32, i32, i64, i64, i32, ctypes.POINTER(sz)],
+        "lhcal_accumulate": [i32, i32, vp, vp, i64, i64, i64, i32, vp, vp, i32, vp, vp, vp, sz, vp],
+        "lhcal_count_tokens": [i32, i64, vp, i32, vp, vp],
+        "lhcal_finalize": [i32, i32, i64, vp, vp, vp, vp],
+        "lhcal_global_scale": [i32, vp, i32, i64, i64, vp, vp],
+        "lhcal_scale_sweep": [i32, i32, vp, i32, i64, i64, vp, vp, vp, vp, vp, vp, vp],
+    }
+    for name, args in sigs.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = ctypes.c_int
+    lib.lhcal_last_error_string.restype = ctypes.c_char_p
+    lib.lhcal_last_error_string.argtypes = []
+    lib.lhcal_version.restype = ctypes.c_int32
+    lib.lhcal_version.argtypes = []
+    lib.lhcal_launch_count.restype = ctypes.c_int64
+    lib.lhcal_launch_count.argtypes = [ctypes.c_int32]
+    _lib = lib
+    return lib
+
+
+def _check(status: int):
+    if status != OK:
+        msg = load_library().lhcal_last_error_string().decode(errors="replace")
+        raise LhcalError(status, msg)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_id(t) -> int:
+    import torch
+
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _mode_id(mode) -> int:
+    return MODE_IDS[mode] if isinstance(mode, str) else int(mode)
+
+
+def lhcal_version() -> int:
+    return int(load_library().lhcal_version())
+
+
+def lhcal_launch_count(reset: bool = False) -> int:
+    """Kernels enqueued by the library from this thread (since the last reset)."""
+    return int(load_library().lhcal_launch_count(1 if reset else 0))
+
+
+def lhcal_accumulate_workspace(mode, dtype: int, tokens: int, cin: int, groups: int = 1) -> int:
+    out = ctypes.c_size_t(0)
+    _check(load_library().lhcal_accumulate_workspace(_mode_id(mode), dtype, tokens, cin, groups, ctypes.byref(out)))
+    return int(out.value)
+
+
+def lhcal_accumulate(mode, x, h, xq=None, p=None, group_offsets=None, token_ids=None,
+                     flags: int = ACCUM_ADD, workspace=None, stream=None):
+    """x, xq: [tokens, cin] (row stride x.stride(0)); h, p, workspace: fp32 device tensors."""
+    m = _mode_id(mode)
+    tokens, cin = int(x.shape[0]), int(x.shape[1])
+    if x.stride(1) != 1:
+        raise ValueError("x must have unit stride along cin")
+    groups = 1 if group_offsets is None else int(group_offsets.numel()) - 1
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load_library().lhcal_accumulate(
+        m, _dtype_id(x), _ptr(x), _ptr(xq), tokens, cin, int(x.stride(0)), groups,
+        _ptr(group_offsets), _ptr(token_ids), flags, _ptr(h), _ptr(p), _ptr(workspace), ws_bytes,
+        _stream(stream)))
+
+
+def lhcal_count_tokens(counts, tokens: int = 0, group_offsets=None, flags: int = ACCUM_ADD, stream=None):
+    groups = 1 if group_offsets is None else int(group_offsets.numel()) - 1
+    _check(load_library().lhcal_count_tokens(groups, tokens, _ptr(group_offsets), flags, _ptr(counts),
+                                             _stream(stream)))
+
+
+def lhcal_finalize(mode, counts, h, p=None, stream=None):
+    m = _mode_id(mode)
+    groups = int(h.shape[0])
+    cin = int(h.shape[1]) * BLOCK
+    _check(load_library().lhcal_finalize(m, groups, cin, _ptr(counts), _ptr(h), _ptr(p), _stream(stream)))
+
+
+def lhcal_global_scale(w, g, stream=None):
+    """w: [groups, rows, cin] fp32/bf16; g: fp32 [groups]."""
+    groups, rows, cin = (int(v) for v in w.shape)
+    _check(load_library().lhcal_global_scale(_dtype_id(w), _ptr(w), groups, rows, cin, _ptr(g), _stream(stream)))
+
+
+def lhcal_scale_sweep(mode, w, h, g, codes, wq=None, loss=None, p=None, stream=None):
+    """w [G, R, C]; h/p finalized; g [G]; codes uint8 [G, R, C/16]; wq fp32 [G, R, C]; loss fp32 [G, R, C/16]."""
+    groups, rows, cin = (int(v) for v in w.shape)
+    _check(load_library().lhcal_scale_sweep(
+        _mode_id(mode), _dtype_id(w), _ptr(w), groups, rows, cin, _ptr(h), _ptr(p), _ptr(g), _ptr(codes),
+        _ptr(wq), _ptr(loss), _stream(stream)))
+
+
+# ------------------------------------------------------------------------------------------------
+# Buffers and the whole hot path
+# ------------------------------------------------------------------------------------------------
+
+class Buffers:
+    """Device buffers for one layer's calibration (allocated by torch, owned by the caller)."""
+
+    def __init__(self, mode, tokens: int, cin: int, rows: int, groups: int, x_dtype: int, device,
+                 want_wq: bool = True, want_loss: bool = True):
+        import torch
+
+        self.mode = _mode_id(mode)
+        nblk = cin // BLOCK
+        hshape = (groups, nblk, BLOCK) if self.mode == DIAG else (groups, nblk, BLOCK, BLOCK)
+        self.h = torch.empty(hshape, dtype=torch.float32, device=device)
+        self.p = torch.empty(hshape, dtype=torch.float32, device=device) if self.mode == ACT_AWARE else None
+        self.counts = torch.empty(groups, dtype=torch.int64, device=device)
+        self.g = torch.empty(groups, dtype=torch.float32, device=device)
+        self.codes = torch.empty((groups, rows, nblk), dtype=torch.uint8, device=device)
+        self.wq = torch.empty((groups, rows, cin), dtype=torch.float32, device=device) if want_wq else None
+        self.loss = torch.empty((groups, rows, nblk), dtype=torch.float32, device=device) if want_loss else None
+        ws = lhcal_accumulate_workspace(self.mode, x_dtype, tokens, cin, groups)
+        self.workspace = torch.empty(max(ws // 4, 1), dtype=torch.float32, device=device) if ws else None
+
+
+def calibrate(mode, x, w, xq=None, group_offsets=None, token_ids=None, buffers: Buffers | None = None,
+              stream=None) -> Buffers:
+    """The whole hot path on one layer: accumulate, count, finalize, global scale, sweep.
+
+    x [T, C], w [G, R, C] (and xq for ``act``, CSR routing for grouped layers) are device
+    tensors. Returns the buffers holding h, p, g, codes, wq and loss.
+    """
+    m = _mode_id(mode)
+    groups, rows, cin = (int(v) for v in w.shape)
+    if buffers is None:
+        buffers = Buffers(m, int(x.shape[0]), cin, rows, groups, _dtype_id(x), x.device)
+    b = buffers
+    lhcal_accumulate(m, x, b.h, xq=xq, p=b.p, group_offsets=group_offsets, token_ids=token_ids,
+                     flags=ACCUM_OVERWRITE, workspace=b.workspace, stream=stream)
+    lhcal_count_tokens(b.counts, tokens=int(x.shape[0]), group_offsets=group_offsets, flags=ACCUM_OVERWRITE,
+                       stream=stream)
+    lhcal_finalize(m, b.counts, b.h, p=b.p, stream=stream)
+    lhcal_global_scale(w, b.g, stream=stream)
+    lhcal_scale_sweep(m, w, b.h, b.g, b.codes, wq=b.wq, loss=b.loss, p=b.p, stream=stream)
+    return b
+
+
+class HostOutputs:
+    """Pinned host copies of a calibration's results: codes, fake-quantized weights, losses."""
+
+    def __init__(self, buffers: Buffers):
+        import torch
+
+        self.codes = torch.empty(buffers.codes.shape, dtype=torch.uint8, pin_memory=True)
+        self.wq = None if buffers.wq is None else torch.empty(buffers.wq.shape, dtype=torch.float32, pin_memory=True)
+        self.loss = None if buffers.loss is None else torch.empty(buffers.loss.shape, dtype=torch.float32,
+                                                                   pin_memory=True)
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in (self.codes, self.wq, self.loss) if t is not None)
+
+
+def calibrate_host(mode, x, w, buffers: Buffers, staging: dict, hxq=None, group_offsets=None, token_ids=None,
+                   out: HostOutputs | None = None, stream=None) -> HostOutputs:
+    """The whole hot path from host tensors (pinned for asynchronous copies) to host results.
+
+    ``staging`` holds device tensors shaped like the inputs under keys "x", "w" and, when
+    used, "xq", "offs", "ids". Inputs are copied host to device on the current stream, the
+    layer is calibrated, and codes / wq / loss are copied back into ``out``. Returns ``out``
+    without synchronising.
+    """
+    if out is None:
+        out = HostOutputs(buffers)
+    staging["x"].copy_(x, non_blocking=True)
+    staging["w"].copy_(w, non_blocking=True)
+    if hxq is not None:
+        staging["xq"].copy_(hxq, non_blocking=True)
+    if group_offsets is not None:
+        staging["offs"].copy_(group_offsets, non_blocking=True)
+        staging["ids"].copy_(token_ids, non_blocking=True)
+    calibrate(mode, staging["x"], staging["w"], xq=staging.get("xq"), group_offsets=staging.get("offs"),
+              token_ids=staging.get("ids"), buffers=buffers, stream=stream)
+    out.codes.copy_(buffers.codes, non_blocking=True)
+    if out.wq is not None:
+        out.wq.copy_(buffers.wq, non_blocking=True)
+    if out.loss is not None:
+        out.loss.copy_(buffers.loss, non_blocking=True)
+    return out

@@ -1,0 +1,567 @@
+// Per-16-wide-input-block Hessian accumulation (raw sums).
+//
+// Method: "add local hessian calibration" (PR #788), Overview (H_n = X_b^T X_b per block);
+// "Add activation-aware local Hessian scale calibration" (PR #1976), "What does this PR do?"
+// (H = X_q^T X_q, P = X_q^T (X_q - X)); "Add WMSE weight scale search calibration" (PR #2283),
+// "How" (Imp = column sums of squares in a [n_blocks, 16] buffer); "[2/3] Speed up layerwise
+// GPTQ on MoE models" (PR #2864), embedded #2840 (one Hessian per expert over its routed tokens).
+//
+// Kernels (all HBM-bound):
+//  * accum_mma_kernel: bf16 FULL / ACT on tensor cores. A CTA owns a 128-column slab (8
+//    blocks, one per warp) and a token range; 64-token x 128-column tiles stream through a
+//    4-stage (FULL) or 3-stage (ACT) cp.async ring in XOR-swizzled shared memory. Each warp
+//    turns 16 tokens of its block into one ldmatrix.x4.trans, which is at once the A fragment
+//    (X_b^T) and both B fragments (X_b) of two m16n8k16 MMAs: the 16x16 block Hessian with no
+//    wasted MACs. bf16 x bf16 products are exact in the fp32 accumulator. For P the
+//    difference D = X_q - X (exact in fp32) is split into bf16 hi + lo parts, two more MMAs
+//    each. Dense: token ranges are split across CTAs and partials go to the workspace,
+//    reduced in a fixed order by reduce_partials_kernel. Grouped: one CTA per (group, slab)
+//    gathers its routed rows through the CSR and writes the group's blocks directly.
+//  * accum_diag_kernel: bf16 DIAG column sums of squares; each thread streams 8 columns
+//    (16-byte loads) over a token range; partials to the workspace, then reduce.
+//  * accum_generic_kernel: CUDA-core fp32 path for fp32 inputs (and grouped bf16 DIAG).
+#include "common.cuh"
+
+namespace lhcal {
+namespace {
+
+// ---------------------------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  const int n = valid ? 16 : 0;  // 0 source bytes: the 16 destination bytes are zero-filled
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(n));
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                                  uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// D += A (16x16 bf16, row) * B (16x8 bf16, col), fp32 accumulate.
+__device__ __forceinline__ void mma_bf16(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// bf16x2 (as uint32) -> two floats, exact.
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t v) {
+  return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+}
+
+__device__ __forceinline__ uint32_t f2_to_bf2(float lo, float hi) {
+  const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&b);
+}
+
+// D = Xq - X for a bf16x2 pair, split into bf16 hi + lo (hi + lo = D to ~2^-17 relative).
+__device__ __forceinline__ void diff_split(uint32_t xq, uint32_t x, uint32_t& hi, uint32_t& lo) {
+  const float2 q = bf2_to_f2(xq), v = bf2_to_f2(x);
+  const float d0 = q.x - v.x, d1 = q.y - v.y;
+  hi = f2_to_bf2(d0, d1);
+  const float2 hf = bf2_to_f2(hi);
+  lo = f2_to_bf2(d0 - hf.x, d1 - hf.y);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Tensor-core FULL / ACT accumulation
+// ---------------------------------------------------------------------------------------------
+
+constexpr int kMmaThreads = 256;  // 8 warps
+constexpr int kSlabCols = 128;    // 8 blocks of 16 columns
+constexpr int kTileTok = 64;
+constexpr int kRowBytes = kSlabCols * 2;              // 256 B per token row of the slab
+constexpr int kTileBytes = kTileTok * kRowBytes;      // 16 KB per tensor per stage
+
+template <bool ACT>
+struct MmaCfg {
+  static constexpr int kStages = ACT ? 3 : 4;
+  static constexpr int kTensors = ACT ? 2 : 1;
+  static constexpr int kSmem = kStages * kTensors * kTileBytes;
+};
+
+// Byte offset of 16-byte chunk c (0..15) of tile row r in the swizzled layout.
+__device__ __forceinline__ uint32_t swz(int r, int c) {
+  return static_cast<uint32_t>(r * kRowBytes + ((c ^ (r & 7)) << 4));
+}
+
+struct TokenSource {
+  // Dense: rows tok_begin .. tok_end-1. Grouped: rows ids[pos] for pos in [tok_begin, tok_end).
+  const int32_t* ids;
+  int64_t tok_begin, tok_end;
+  __device__ __forceinline__ int64_t row(int64_t pos) const { return ids ? static_cast<int64_t>(__ldg(ids + pos)) : pos; }
+};
+
+template <bool ACT>
+__device__ __forceinline__ void load_tile(uint8_t* smem_stage, const __nv_bfloat16* x,
+                                          const __nv_bfloat16* xq, int64_t ldx, int64_t col0,
+                                          int64_t cin, const TokenSource& src, int64_t pos0) {
+  const int tid = threadIdx.x;
+  const int c = tid & 15;
+  const bool col_ok = col0 + c * 8 < cin;
+#pragma unroll
+  for (int m = 0; m < kTileTok / 16; ++m) {
+    const int r = (tid >> 4) + 16 * m;
+    const int64_t pos = pos0 + r;
+    const bool ok = col_ok && pos < src.tok_end;
+    const int64_t row = ok ? src.row(pos) : 0;
+    const int64_t off = ok ? row * ldx + col0 + c * 8 : 0;
+    const uint32_t dst = smem_u32(smem_stage) + swz(r, c);
+    if (ACT) {
+      cp_async16(dst, xq + off, ok);
+      cp_async16(dst + kTileBytes, x + off, ok);
+    } else {
+      cp_async16(dst, x + off, ok);
+    }
+  }
+}
+
+// out_h / out_p point at [8 blocks][256] for this CTA's slab (already offset); nblk_valid
+// is the number of blocks of the slab inside cin. accumulate_into: out += acc, else out = acc.
+template <bool ACT>
+__global__ void __launch_bounds__(kMmaThreads)
+accum_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ xq,
+                 int64_t tokens, int64_t cin, int64_t ldx, const int32_t* __restrict__ group_offsets,
+                 const int32_t* __restrict__ token_ids, int64_t tok_per_split, float* __restrict__ out_h,
+                 float* __restrict__ out_p, int64_t out_group_stride, int64_t out_split_stride,
+                 int accumulate_into) {
+  using Cfg = MmaCfg<ACT>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t slab = blockIdx.x;
+  const int64_t col0 = slab * kSlabCols;
+  const int64_t nblk = cin / kBlock;
+
+  TokenSource src;
+  int64_t out_off;
+  if (group_offsets != nullptr) {  // grouped: blockIdx.y = group
+    src.ids = token_ids;
+    src.tok_begin = __ldg(group_offsets + blockIdx.y);
+    src.tok_end = __ldg(group_offsets + blockIdx.y + 1);
+    out_off = static_cast<int64_t>(blockIdx.y) * out_group_stride;
+  } else {  // dense: blockIdx.y = token split
+    src.ids = nullptr;
+    src.tok_begin = static_cast<int64_t>(blockIdx.y) * tok_per_split;
+    src.tok_end = imin64(tokens, src.tok_begin + tok_per_split);
+    out_off = static_cast<int64_t>(blockIdx.y) * out_split_stride;
+  }
+  const int64_t ntiles = ceil_div(imax64(src.tok_end - src.tok_begin, 0), kTileTok);
+
+  float acc_h[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  float acc_p[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+
+  constexpr int S = Cfg::kStages;
+  constexpr int stage_bytes = Cfg::kTensors * kTileBytes;
+#pragma unroll
+  for (int s = 0; s < S - 1; ++s) {
+    if (s < ntiles) load_tile<ACT>(smem + s * stage_bytes, x, xq, ldx, col0, cin, src, src.tok_begin + s * kTileTok);
+    cp_async_commit();
+  }
+
+  // ldmatrix.x4.trans addressing: lane -> (matrix mi = lane / 8, row rr = lane % 8);
+  // matrices: (tok 0-7, cols 0-7), (tok 0-7, cols 8-15), (tok 8-15, cols 0-7), (tok 8-15, cols 8-15).
+  const int mi = lane >> 3, rr = lane & 7;
+  const int lrow = ((mi >> 1) << 3) + rr;
+  const int lchunk = 2 * warp + (mi & 1);
+
+  for (int64_t it = 0; it < ntiles; ++it) {
+    cp_async_wait<S - 2>();
+    __syncthreads();
+    {
+      const int64_t nt = it + S - 1;
+      if (nt < ntiles)
+        load_tile<ACT>(smem + (nt % S) * stage_bytes, x, xq, ldx, col0, cin, src, src.tok_begin + nt * kTileTok);
+      cp_async_commit();
+    }
+    const uint32_t base = smem_u32(smem + (it % S) * stage_bytes);
+#pragma unroll
+    for (int ts = 0; ts < kTileTok / 16; ++ts) {
+      const uint32_t addr = base + swz(ts * 16 + lrow, lchunk);
+      uint32_t q0, q1, q2, q3;
+      ldmatrix_x4_trans(addr, q0, q1, q2, q3);  // X_q (ACT) or X (FULL)
+      mma_bf16(acc_h[0], q0, q1, q2, q3, q0, q2);
+      mma_bf16(acc_h[1], q0, q1, q2, q3, q1, q3);
+      if (ACT) {
+        uint32_t x0, x1, x2, x3;
+        ldmatrix_x4_trans(addr + kTileBytes, x0, x1, x2, x3);
+        uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
+        diff_split(q0, x0, h0, l0);
+        diff_split(q1, x1, h1, l1);
+        diff_split(q2, x2, h2, l2);
+        diff_split(q3, x3, h3, l3);
+        mma_bf16(acc_p[0], q0, q1, q2, q3, h0, h2);
+        mma_bf16(acc_p[0], q0, q1, q2, q3, l0, l2);
+        mma_bf16(acc_p[1], q0, q1, q2, q3, h1, h3);
+        mma_bf16(acc_p[1], q0, q1, q2, q3, l1, l3);
+      }
+    }
+  }
+  cp_async_wait<0>();
+
+  const int64_t blk = slab * 8 + warp;
+  if (blk >= nblk) return;
+  // Accumulator layout of m16n8: c0,c1 -> (i = lane/4, j = 2*(lane%4) + {0,1}); c2,c3 -> i + 8.
+  const int i0 = lane >> 2, j0 = 2 * (lane & 3);
+  float* oh = out_h + out_off + blk * 256;
+  float* op = ACT ? out_p + out_off + blk * 256 : nullptr;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int idx = (i0 + 8 * half) * 16 + nt * 8 + j0;
+      float2 vh = make_float2(acc_h[nt][2 * half], acc_h[nt][2 * half + 1]);
+      if (accumulate_into) {
+        const float2 o = *reinterpret_cast<const float2*>(oh + idx);
+        vh.x += o.x;
+        vh.y += o.y;
+      }
+      *reinterpret_cast<float2*>(oh + idx) = vh;
+      if (ACT) {
+        float2 vp = make_float2(acc_p[nt][2 * half], acc_p[nt][2 * half + 1]);
+        if (accumulate_into) {
+          const float2 o = *reinterpret_cast<const float2*>(op + idx);
+          vp.x += o.x;
+          vp.y += o.y;
+        }
+        *reinterpret_cast<float2*>(op + idx) = vp;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// bf16 DIAG accumulation (dense)
+// ---------------------------------------------------------------------------------------------
+
+constexpr int kDiagThreads = 256;
+constexpr int kDiagCols = kDiagThreads * 8;  // 2048 columns per CTA
+constexpr int kDiagUnroll = 8;
+
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ void sq_acc(float* acc, const uint4& v) {
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = bf2_to_f2(u[i]);
+    acc[2 * i] = fmaf(f.x, f.x, acc[2 * i]);
+    acc[2 * i + 1] = fmaf(f.y, f.y, acc[2 * i + 1]);
+  }
+}
+
+__global__ void __launch_bounds__(kDiagThreads)
+accum_diag_kernel(const __nv_bfloat16* __restrict__ x, int64_t tokens, int64_t cin, int64_t ldx,
+                  int64_t tok_per_split, float* __restrict__ ws) {
+  const int64_t col = static_cast<int64_t>(blockIdx.x) * kDiagCols + threadIdx.x * 8;
+  if (col >= cin) return;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.y) * tok_per_split;
+  const int64_t t1 = imin64(tokens, t0 + tok_per_split);
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  const __nv_bfloat16* p = x + t0 * ldx + col;
+  int64_t t = t0;
+  for (; t + kDiagUnroll <= t1; t += kDiagUnroll, p += kDiagUnroll * ldx) {
+    uint4 v[kDiagUnroll];
+#pragma unroll
+    for (int u = 0; u < kDiagUnroll; ++u) v[u] = ld_stream16(p + u * ldx);
+#pragma unroll
+    for (int u = 0; u < kDiagUnroll; ++u) sq_acc(acc, v[u]);
+  }
+  for (; t < t1; ++t, p += ldx) sq_acc(acc, ld_stream16(p));
+  float4* dst = reinterpret_cast<float4*>(ws + static_cast<int64_t>(blockIdx.y) * cin + col);
+  dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Generic CUDA-core accumulation (fp32 inputs; grouped bf16 DIAG)
+// ---------------------------------------------------------------------------------------------
+
+constexpr int kGenTok = 32;
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T v);
+template <>
+__device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// One CTA of 256 threads per (block n, split or group). Thread (i, j) owns H_ij (and P_ij);
+// DIAG uses threads 0..15. Partials / results go to out + (split or group) stride.
+template <typename T, int MODE>
+__global__ void __launch_bounds__(256)
+accum_generic_kernel(const T* __restrict__ x, const T* __restrict__ xq, int64_t tokens, int64_t cin,
+                     int64_t ldx, const int32_t* __restrict__ group_offsets,
+                     const int32_t* __restrict__ token_ids, int64_t tok_per_split, float* __restrict__ out_h,
+                     float* __restrict__ out_p, int64_t out_stride, int accumulate_into) {
+  __shared__ float sx[kGenTok][kBlock];
+  __shared__ float sq[kGenTok][kBlock];
+  const int64_t n = blockIdx.x;
+  const int tid = threadIdx.x, i = tid >> 4, j = tid & 15;
+  int64_t b0, b1;
+  const bool grouped = group_offsets != nullptr;
+  if (grouped) {
+    b0 = __ldg(group_offsets + blockIdx.y);
+    b1 = __ldg(group_offsets + blockIdx.y + 1);
+  } else {
+    b0 = static_cast<int64_t>(blockIdx.y) * tok_per_split;
+    b1 = imin64(tokens, b0 + tok_per_split);
+  }
+  float ah = 0.f, ap = 0.f;
+  for (int64_t pos0 = b0; pos0 < b1; pos0 += kGenTok) {
+    for (int e = tid; e < kGenTok * kBlock; e += 256) {
+      const int tt = e >> 4, cc = e & 15;
+      const int64_t pos = pos0 + tt;
+      float vx = 0.f, vq = 0.f;
+      if (pos < b1) {
+        const int64_t row = grouped ? static_cast<int64_t>(__ldg(token_ids + pos)) : pos;
+        const int64_t off = row * ldx + n * kBlock + cc;
+        vx = to_f32<T>(x[off]);
+        if (MODE == LHCAL_ACT_AWARE) vq = to_f32<T>(xq[off]);
+      }
+      sx[tt][cc] = vx;
+      sq[tt][cc] = vq;
+    }
+    __syncthreads();
+    if (MODE == LHCAL_DIAG) {
+      if (tid < kBlock)
+        for (int tt = 0; tt < kGenTok; ++tt) ah = fmaf(sx[tt][tid], sx[tt][tid], ah);
+    } else if (MODE == LHCAL_FULL) {
+      for (int tt = 0; tt < kGenTok; ++tt) ah = fmaf(sx[tt][i], sx[tt][j], ah);
+    } else {
+      for (int tt = 0; tt < kGenTok; ++tt) {
+        ah = fmaf(sq[tt][i], sq[tt][j], ah);
+        ap = fmaf(sq[tt][i], sq[tt][j] - sx[tt][j], ap);
+      }
+    }
+    __syncthreads();
+  }
+  const int64_t base = static_cast<int64_t>(blockIdx.y) * out_stride;
+  if (MODE == LHCAL_DIAG) {
+    if (tid < kBlock) {
+      float* o = out_h + base + n * kBlock + tid;
+      *o = accumulate_into ? *o + ah : ah;
+    }
+  } else {
+    float* o = out_h + base + n * 256 + tid;
+    *o = accumulate_into ? *o + ah : ah;
+    if (MODE == LHCAL_ACT_AWARE) {
+      float* q = out_p + base + n * 256 + tid;
+      *q = accumulate_into ? *q + ap : ap;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Fixed-order reduction of split partials: out[i] (+)= sum_s ws[s * stride + i]
+// ---------------------------------------------------------------------------------------------
+
+__global__ void reduce_partials_kernel(const float* __restrict__ ws, int64_t splits, int64_t stride,
+                                       int64_t count, float* __restrict__ out, int accumulate_into) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < count;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float s = 0.f;
+    for (int64_t k = 0; k < splits; ++k) s += __ldg(ws + k * stride + i);
+    out[i] = accumulate_into ? out[i] + s : s;
+  }
+}
+
+__global__ void fill_kernel(float* __restrict__ out, int64_t count, float v) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < count;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    out[i] = v;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Work split (pure function of the sizes)
+// ---------------------------------------------------------------------------------------------
+
+enum class Path { kMma, kDiagBf16, kGeneric };
+
+Path choose_path(lhcal_mode mode, lhcal_dtype dtype, int32_t groups) {
+  if (dtype == LHCAL_BF16 && mode != LHCAL_DIAG) return Path::kMma;
+  if (dtype == LHCAL_BF16 && mode == LHCAL_DIAG && groups == 1) return Path::kDiagBf16;
+  return Path::kGeneric;
+}
+
+struct Split {
+  int64_t splits;   // CTAs along tokens
+  int64_t per;      // tokens per split
+};
+
+Split token_split(int64_t tokens, int64_t ctas_per_split, int64_t target_ctas, int64_t granule) {
+  Split s;
+  if (tokens <= 0) return {1, granule};
+  int64_t want = imax64(1, ceil_div(target_ctas, imax64(ctas_per_split, 1)));
+  want = min(want, ceil_div(tokens, granule));
+  s.per = ceil_div(ceil_div(tokens, want), granule) * granule;
+  s.splits = ceil_div(tokens, s.per);
+  return s;
+}
+
+Split split_for(Path path, int64_t tokens, int64_t cin) {
+  switch (path) {
+    case Path::kMma:
+      return token_split(tokens, ceil_div(cin, kSlabCols), 3 * kNumSms, kTileTok);
+    case Path::kDiagBf16:
+      return token_split(tokens, ceil_div(cin, kDiagCols), 8 * kNumSms, kDiagUnroll);
+    default:
+      return token_split(tokens, cin / kBlock, 4 * kNumSms, kGenTok);
+  }
+}
+
+size_t floats_per_split(lhcal_mode mode, int64_t cin) {
+  const int64_t nblk = cin / kBlock;
+  if (mode == LHCAL_DIAG) return static_cast<size_t>(cin);
+  return static_cast<size_t>(nblk * 256 * (mode == LHCAL_ACT_AWARE ? 2 : 1));
+}
+
+lhcal_status launch_fill(float* out, int64_t count, float v, cudaStream_t stream) {
+  if (count <= 0) return LHCAL_OK;
+  const int64_t blocks = imin64(ceil_div(count, 256), 4 * kNumSms);
+  fill_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(out, count, v);
+  return check_launch("fill");
+}
+
+lhcal_status launch_reduce(const float* ws, int64_t splits, int64_t stride, int64_t count, float* out,
+                           int accumulate_into, cudaStream_t stream) {
+  const int64_t blocks = imin64(ceil_div(count, 256), 8 * kNumSms);
+  reduce_partials_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(ws, splits, stride, count, out,
+                                                                             accumulate_into);
+  return check_launch("reduce partials");
+}
+
+template <bool ACT>
+lhcal_status launch_mma(const void* x, const void* xq, int64_t tokens, int64_t cin, int64_t ldx,
+                        int32_t groups, const int32_t* offs, const int32_t* ids, int accumulate_into,
+                        float* h, float* p, float* ws, cudaStream_t stream) {
+  using Cfg = MmaCfg<ACT>;
+  // Set on every call: cheap, thread-safe, and correct whichever device is current.
+  const cudaError_t attr = cudaFuncSetAttribute(accum_mma_kernel<ACT>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
+  if (attr != cudaSuccess) return fail(LHCAL_ERR_CUDA, "accumulate: %s", cudaGetErrorString(attr));
+  const int64_t slabs = ceil_div(cin, kSlabCols);
+  const int64_t nblk = cin / kBlock;
+  const auto* xb = static_cast<const __nv_bfloat16*>(x);
+  const auto* xqb = static_cast<const __nv_bfloat16*>(ACT ? xq : x);
+  if (offs != nullptr) {
+    const dim3 grid(static_cast<unsigned>(slabs), static_cast<unsigned>(groups));
+    accum_mma_kernel<ACT><<<grid, kMmaThreads, Cfg::kSmem, stream>>>(
+        xb, xqb, tokens, cin, ldx, offs, ids, 0, h, p, nblk * 256, 0, accumulate_into);
+    return check_launch("accumulate (grouped, tensor cores)");
+  }
+  const Split sp = split_for(Path::kMma, tokens, cin);
+  const int64_t per_split = nblk * 256;
+  float* ws_h = ws;
+  float* ws_p = ws + sp.splits * per_split;
+  const dim3 grid(static_cast<unsigned>(slabs), static_cast<unsigned>(sp.splits));
+  accum_mma_kernel<ACT><<<grid, kMmaThreads, Cfg::kSmem, stream>>>(
+      xb, xqb, tokens, cin, ldx, nullptr, nullptr, sp.per, ws_h, ws_p, 0, per_split, 0);
+  lhcal_status st = check_launch("accumulate (tensor cores)");
+  if (st != LHCAL_OK) return st;
+  st = launch_reduce(ws_h, sp.splits, per_split, per_split, h, accumulate_into, stream);
+  if (st != LHCAL_OK || !ACT) return st;
+  return launch_reduce(ws_p, sp.splits, per_split, per_split, p, accumulate_into, stream);
+}
+
+template <typename T, int MODE>
+lhcal_status launch_generic(const void* x, const void* xq, int64_t tokens, int64_t cin, int64_t ldx,
+                            int32_t groups, const int32_t* offs, const int32_t* ids, int accumulate_into,
+                            float* h, float* p, float* ws, cudaStream_t stream) {
+  const int64_t nblk = cin / kBlock;
+  const int64_t per_group = (MODE == LHCAL_DIAG) ? cin : nblk * 256;
+  const auto* xt = static_cast<const T*>(x);
+  const auto* xqt = static_cast<const T*>(MODE == LHCAL_ACT_AWARE ? xq : x);
+  if (offs != nullptr) {
+    const dim3 grid(static_cast<unsigned>(nblk), static_cast<unsigned>(groups));
+    accum_generic_kernel<T, MODE><<<grid, 256, 0, stream>>>(xt, xqt, tokens, cin, ldx, offs, ids, 0, h, p,
+                                                            per_group, accumulate_into);
+    return check_launch("accumulate (grouped)");
+  }
+  const Split sp = split_for(Path::kGeneric, tokens, cin);
+  float* ws_h = ws;
+  float* ws_p = ws + sp.splits * per_group;
+  const dim3 grid(static_cast<unsigned>(nblk), static_cast<unsigned>(sp.splits));
+  accum_generic_kernel<T, MODE><<<grid, 256, 0, stream>>>(xt, xqt, tokens, cin, ldx, nullptr, nullptr, sp.per,
+                                                          ws_h, ws_p, per_group, 0);
+  lhcal_status st = check_launch("accumulate");
+  if (st != LHCAL_OK) return st;
+  st = launch_reduce(ws_h, sp.splits, per_group, per_group, h, accumulate_into, stream);
+  if (st != LHCAL_OK || MODE != LHCAL_ACT_AWARE) return st;
+  return launch_reduce(ws_p, sp.splits, per_group, per_group, p, accumulate_into, stream);
+}
+
+}  // namespace
+
+size_t accumulate_workspace_bytes(lhcal_mode mode, lhcal_dtype dtype, int64_t tokens, int64_t cin,
+                                  int32_t groups) {
+  if (groups != 1 || tokens <= 0) return 0;
+  const Path path = choose_path(mode, dtype, groups);
+  const Split sp = split_for(path, tokens, cin);
+  return static_cast<size_t>(sp.splits) * floats_per_split(mode, cin) * sizeof(float);
+}
+
+lhcal_status launch_accumulate(lhcal_mode mode, lhcal_dtype dtype, const void* x, const void* xq,
+                               int64_t tokens, int64_t cin, int64_t ldx, int32_t groups,
+                               const int32_t* group_offsets, const int32_t* token_ids, int32_t flags,
+                               float* h, float* p, void* workspace, cudaStream_t stream) {
+  const int acc_into = (flags & LHCAL_ACCUM_OVERWRITE) ? 0 : 1;
+  const int64_t nblk = cin / kBlock;
+  const int64_t out_count = static_cast<int64_t>(groups) * (mode == LHCAL_DIAG ? cin : nblk * 256);
+  if (group_offsets == nullptr && tokens == 0) {
+    if (acc_into) return LHCAL_OK;
+    lhcal_status st = launch_fill(h, out_count, 0.f, stream);
+    if (st != LHCAL_OK || mode != LHCAL_ACT_AWARE) return st;
+    return launch_fill(p, out_count, 0.f, stream);
+  }
+  float* ws = static_cast<float*>(workspace);
+  const Path path = choose_path(mode, dtype, groups);
+  if (path == Path::kMma) {
+    if (mode == LHCAL_ACT_AWARE)
+      return launch_mma<true>(x, xq, tokens, cin, ldx, groups, group_offsets, token_ids, acc_into, h, p, ws, stream);
+    return launch_mma<false>(x, xq, tokens, cin, ldx, groups, group_offsets, token_ids, acc_into, h, p, ws, stream);
+  }
+  if (path == Path::kDiagBf16) {
+    const Split sp = split_for(path, tokens, cin);
+    const dim3 grid(static_cast<unsigned>(ceil_div(cin, kDiagCols)), static_cast<unsigned>(sp.splits));
+    accum_diag_kernel<<<grid, kDiagThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), tokens, cin, ldx,
+                                                         sp.per, ws);
+    lhcal_status st = check_launch("accumulate (diagonal)");
+    if (st != LHCAL_OK) return st;
+    return launch_reduce(ws, sp.splits, cin, cin, h, acc_into, stream);
+  }
+#define LHCAL_GEN(T, M) \
+  return launch_generic<T, M>(x, xq, tokens, cin, ldx, groups, group_offsets, token_ids, acc_into, h, p, ws, stream)
+  if (dtype == LHCAL_F32) {
+    if (mode == LHCAL_FULL) LHCAL_GEN(float, LHCAL_FULL);
+    if (mode == LHCAL_ACT_AWARE) LHCAL_GEN(float, LHCAL_ACT_AWARE);
+    LHCAL_GEN(float, LHCAL_DIAG);
+  }
+  LHCAL_GEN(__nv_bfloat16, LHCAL_DIAG);
+#undef LHCAL_GEN
+}
+
+}  // namespace lhcal

@@ -1,0 +1,99 @@
+"""liblhcal.so builds, loads and exports the C ABI; host-side validation needs no GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import scale_calibration_lh_b200 as L
+from scale_calibration_lh_b200 import build as B
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return L.load_library()
+
+
+def declared_functions(root):
+    text = open(os.path.join(root, "include", "lhcal.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lhcal_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib, root_dir):
+    names = declared_functions(root_dir)
+    assert "lhcal_scale_sweep" in names and "lhcal_accumulate" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert L.lhcal_version() == 100
+
+
+def test_status_values_match_header(root_dir):
+    text = open(os.path.join(root_dir, "include", "lhcal.h")).read()
+    for name, val in [("LHCAL_OK", L.OK), ("LHCAL_ERR_INVALID_ARG", L.ERR_INVALID_ARG),
+                      ("LHCAL_ERR_UNSUPPORTED", L.ERR_UNSUPPORTED), ("LHCAL_ERR_DEVICE_MISMATCH", L.ERR_DEVICE_MISMATCH),
+                      ("LHCAL_ERR_CUDA", L.ERR_CUDA), ("LHCAL_ERR_TIMEOUT", L.ERR_TIMEOUT),
+                      ("LHCAL_F32", L.F32), ("LHCAL_BF16", L.BF16), ("LHCAL_FULL", L.FULL),
+                      ("LHCAL_ACT_AWARE", L.ACT_AWARE), ("LHCAL_DIAG", L.DIAG),
+                      ("LHCAL_ACCUM_ADD", L.ACCUM_ADD), ("LHCAL_ACCUM_OVERWRITE", L.ACCUM_OVERWRITE),
+                      ("LHCAL_N_CANDIDATES", L.N_CANDIDATES)]:
+        m = re.search(rf"\b{name}\s*=?\s*(\d+)", text)
+        assert m and int(m.group(1)) == val, name
+
+
+def test_workspace_query_is_host_only(lib):
+    dense = L.lhcal_accumulate_workspace("full", L.BF16, 16384, 4096, 1)
+    assert dense > 0 and dense % (256 * 4 * 256) == 0  # whole [splits, N, 16, 16] partials
+    act = L.lhcal_accumulate_workspace("act", L.BF16, 16384, 4096, 1)
+    assert act == 2 * dense
+    diag = L.lhcal_accumulate_workspace("diag", L.BF16, 65536, 12288, 1)
+    assert diag % (12288 * 4) == 0
+    assert L.lhcal_accumulate_workspace("full", L.BF16, 16384, 2560, 512) == 0
+    assert L.lhcal_accumulate_workspace("full", L.BF16, 0, 64, 1) == 0
+    with pytest.raises(L.LhcalError) as e:
+        L.lhcal_accumulate_workspace("full", L.BF16, 100, 24, 1)
+    assert e.value.status == L.ERR_INVALID_ARG and "multiple of 16" in str(e.value)
+    with pytest.raises(L.LhcalError) as e:
+        L.lhcal_accumulate_workspace(7, L.BF16, 100, 32, 1)
+    assert e.value.status == L.ERR_UNSUPPORTED
+
+
+def _call_accumulate(lib, **kw):
+    args = dict(mode=L.FULL, dtype=L.BF16, x=None, xq=None, tokens=10, cin=32, ldx=32, groups=1, offs=None,
+                ids=None, flags=0, h=None, p=None, ws=None, ws_bytes=0, stream=None)
+    args.update(kw)
+    return lib.lhcal_accumulate(args["mode"], args["dtype"], args["x"], args["xq"], args["tokens"], args["cin"],
+                                args["ldx"], args["groups"], args["offs"], args["ids"], args["flags"], args["h"],
+                                args["p"], args["ws"], args["ws_bytes"], args["stream"])
+
+
+def test_argument_validation_without_gpu(lib):
+    assert _call_accumulate(lib, cin=33) == L.ERR_INVALID_ARG
+    assert _call_accumulate(lib, ldx=16) == L.ERR_INVALID_ARG
+    assert _call_accumulate(lib, ldx=36) == L.ERR_INVALID_ARG  # 72 bytes: not a multiple of 16
+    assert _call_accumulate(lib, flags=5) == L.ERR_INVALID_ARG
+    assert _call_accumulate(lib, groups=3) == L.ERR_INVALID_ARG
+    assert _call_accumulate(lib, mode=L.ACT_AWARE) == L.ERR_INVALID_ARG  # no xq
+    assert _call_accumulate(lib, tokens=-1) == L.ERR_INVALID_ARG
+    assert _call_accumulate(lib, dtype=9) == L.ERR_UNSUPPORTED
+    assert _call_accumulate(lib, tokens=100000, cin=4096, ldx=4096) == L.ERR_INVALID_ARG  # workspace too small
+    assert b"workspace" in lib.lhcal_last_error_string()
+    # Sweep / finalize / global scale reject bad sizes before touching memory.
+    assert lib.lhcal_scale_sweep(0, 1, None, 1, 0, 32, None, None, None, None, None, None, None) == L.ERR_INVALID_ARG
+    assert lib.lhcal_scale_sweep(0, 1, None, 0, 4, 32, None, None, None, None, None, None, None) == L.ERR_INVALID_ARG
+    assert lib.lhcal_scale_sweep(1, 1, None, 1, 4, 32, None, None, None, None, None, None, None) == L.ERR_INVALID_ARG
+    assert lib.lhcal_finalize(0, 1, 20, None, None, None, None) == L.ERR_INVALID_ARG
+    assert lib.lhcal_global_scale(3, None, 1, 4, 32, None, None) == L.ERR_UNSUPPORTED
+    assert lib.lhcal_count_tokens(2, 5, None, 0, None, None) == L.ERR_INVALID_ARG
+    # A pointer that is not device memory is refused (no GPU here: the query itself fails).
+    buf = ctypes.create_string_buffer(4096)
+    addr = (ctypes.addressof(buf) + 255) // 256 * 256
+    st = lib.lhcal_global_scale(1, ctypes.c_void_p(addr), 1, 4, 32, ctypes.c_void_p(addr), None)
+    assert st in (L.ERR_INVALID_ARG, L.ERR_DEVICE_MISMATCH)
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    monkeypatch.setattr(L, "_lib", None)
+    with pytest.raises(RuntimeError, match="not found"):
+        L.load_library(str(tmp_path / "nope.so"))

@@ -1,0 +1,300 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 CPU oracle.
+
+Small cases span several tiles and ragged tails (tokens not a multiple of the 64-token
+tile, cin not a multiple of the 128-column slab or the 2048-column DIAG slab, rows not a
+multiple of the 128-row sweep tile, experts with no tokens). Full-size workloads compare
+all Hessian blocks and a sample of sweep units (plus the layer's corner units).
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import scale_calibration_lh_b200 as L  # noqa: E402
+from scale_calibration_lh_b200 import synth  # noqa: E402
+from oracle import lhcal_oracle as O  # noqa: E402
+from tests import parity as P  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from scale_calibration_lh_b200 import build
+
+    build.build()
+    L.load_library()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+
+
+def _sync():
+    torch.cuda.synchronize()
+
+
+def _oracle_hessians(layer):
+    xq = layer.xq_f32() if layer.xq is not None else None
+    hs, ps, counts = O.accumulate(layer.mode, layer.x_f32(), xq, layer.group_offsets, layer.token_ids)
+    return hs, ps, counts
+
+
+def _run_and_check(layer, units=None, check_raw=True):
+    d = P.layer_to_device(layer)
+    mode = L.MODE_IDS[layer.mode]
+    G, R, C = layer.groups, layer.rows, layer.cin
+    nblk = C // 16
+    # Raw sums first (OVERWRITE into fresh buffers), compared before finalisation.
+    b = L.Buffers(mode, layer.tokens, C, R, G, L.BF16 if layer.dtype == "bf16" else L.F32, "cuda")
+    L.lhcal_accumulate(mode, d["x"], b.h, xq=d["xq"], p=b.p, group_offsets=d["offs"], token_ids=d["ids"],
+                       flags=L.ACCUM_OVERWRITE, workspace=b.workspace)
+    _sync()
+    hs, ps, counts = _oracle_hessians(layer)
+    report = {}
+    if check_raw:
+        report["h_raw"] = P.check_hessians(b.h.cpu().numpy(), hs, f"{layer.name} raw H")
+        if ps is not None:
+            report["p_raw"] = P.check_hessians(b.p.cpu().numpy(), ps, f"{layer.name} raw P")
+    b2 = L.calibrate(mode, d["x"], d["w"], xq=d["xq"], group_offsets=d["offs"], token_ids=d["ids"], buffers=b)
+    _sync()
+    h, p = O.finalize(layer.mode, hs, ps, counts)
+    report["h"] = P.check_hessians(b2.h.cpu().numpy(), h, f"{layer.name} H")
+    if p is not None:
+        report["p"] = P.check_hessians(b2.p.cpu().numpy(), p, f"{layer.name} P")
+    np.testing.assert_array_equal(b2.counts.cpu().numpy(), counts)
+    w32 = layer.w_f32()
+    g = np.array([O.global_scale(w32[e]) for e in range(G)], np.float32)
+    np.testing.assert_array_equal(b2.g.cpu().numpy().view(np.int32), g.view(np.int32))
+    if units is None:
+        units = P.all_units(G, R, nblk)
+    ref = O.sweep(layer.mode, w32, h, p, g, units)
+    gc, gw, gl = P.gather_gpu_units(b2.codes, b2.wq, b2.loss, units)
+    report["sweep"] = P.check_sweep(gc, gw, gl, ref, layer.name)
+    return report
+
+
+# ----------------------------------------------------------------------------- small cases
+
+def test_tiny_full_size_end_to_end():
+    r = _run_and_check(synth.make_layer("tiny", 0))
+    assert r["sweep"]["units"] == 128
+
+
+@pytest.mark.parametrize("tokens,cin,rows", [(1000, 272, 300), (64, 128, 128), (1, 16, 1), (130, 400, 257)])
+def test_dense_full_bf16(tokens, cin, rows):
+    _run_and_check(synth.make_layer("dense", 1, tokens=tokens, cin=cin, rows=rows))
+
+
+@pytest.mark.parametrize("tokens,cin,rows", [(777, 160, 200), (65, 48, 129)])
+def test_act_aware_bf16(tokens, cin, rows):
+    _run_and_check(synth.make_layer("act", 2, tokens=tokens, cin=cin, rows=rows))
+
+
+@pytest.mark.parametrize("tokens,cin,rows", [(1500, 2064, 130), (9, 32, 3)])
+def test_wmse_diag_bf16(tokens, cin, rows):
+    _run_and_check(synth.make_layer("wmse", 3, tokens=tokens, cin=cin, rows=rows))
+
+
+def test_moe_grouped_with_empty_experts():
+    layer = synth.make_layer("moe", 4, tokens=40, cin=160, rows=40, groups=64, top_k=3)
+    counts = np.diff(layer.group_offsets)
+    assert (counts == 0).any() and (counts > 1).any()
+    _run_and_check(layer)
+
+
+def test_moe_grouped_diag_bf16_generic_path():
+    layer = synth.make_layer("moe", 5, tokens=50, cin=48, rows=20, groups=8, top_k=2)
+    layer.mode = "diag"
+    _run_and_check(layer)
+
+
+@pytest.mark.parametrize("mode", ["full", "act", "diag"])
+@pytest.mark.parametrize("grouped", [False, True])
+def test_fp32_inputs_all_modes(mode, grouped):
+    rng = np.random.default_rng(6)
+    T, C, R, G = 100, 48, 20, (5 if grouped else 1)
+    x = rng.normal(size=(T, C)).astype(np.float32)
+    w = rng.normal(0, 0.02, (G, R, C)).astype(np.float32)
+    layer = synth.Layer("f32-" + mode, mode, "f32", x, w)
+    if mode == "act":
+        layer.xq = (x + rng.normal(0, 0.05, x.shape)).astype(np.float32)
+    if grouped:
+        layer.group_offsets, layer.token_ids = synth.moe_routing(T, G, 2, 7)
+    _run_and_check(layer)
+
+
+# ----------------------------------------------------------------------------- sweep special cases
+
+def _sweep_gpu(mode, w, h, p, g):
+    """w fp32 [G,R,C]; h/p/g from the oracle side (fp32-rounded) -> GPU outputs (numpy)."""
+    G, R, C = w.shape
+    dw = P.to_device(w, "f32")
+    dh = P.to_device(np.asarray(h, np.float32), "f32")
+    dp = None if p is None else P.to_device(np.asarray(p, np.float32), "f32")
+    dg = P.to_device(g, "f32")
+    codes = torch.empty((G, R, C // 16), dtype=torch.uint8, device="cuda")
+    wq = torch.empty((G, R, C), dtype=torch.float32, device="cuda")
+    loss = torch.empty((G, R, C // 16), dtype=torch.float32, device="cuda")
+    L.lhcal_scale_sweep(mode, dw, dh, dg, codes, wq=wq, loss=loss, p=dp)
+    _sync()
+    return codes.cpu().numpy(), wq.cpu().numpy(), loss.cpu().numpy()
+
+
+def _special_weights(seed=8):
+    """Blocks with exact E2M1 ties, neighbours of ties, zeros, -0.0, a lone outlier, tiny values."""
+    rng = np.random.default_rng(seed)
+    G, R, C = 3, 40, 64
+    w = rng.normal(0, 0.02, (G, R, C)).astype(np.float32)
+    g0 = O.global_scale(w[0])
+    s = O.candidate_scales(g0)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    for r in range(0, 20):
+        k = rng.integers(0, 126)
+        t = (mids[rng.integers(0, 7, 16)] * np.float64(s[k])).astype(np.float32)  # may round: then a near-tie
+        sign = np.where(rng.random(16) < 0.5, -1, 1).astype(np.float32)
+        w[0, r, :16] = t * sign
+        w[0, r, 16:32] = np.nextafter(t, np.float32(1)) * sign
+        w[0, r, 32:48] = np.nextafter(t, np.float32(0)) * sign
+    w[0, 0, :] = np.float32(0.0)             # all-zero block row
+    w[0, 1, 16:32] = np.float32(-0.0)        # negative zeros
+    w[0, 2, 48:64] = 0.0
+    w[0, 2, 50] = 0.5                        # lone outlier
+    w[1] = rng.normal(0, 1e-3, (R, C)).astype(np.float32) * (rng.random((R, C)) < 0.3)
+    w[2] = 0.0                               # whole group zero: g = 0
+    return w
+
+
+@pytest.mark.parametrize("mode", ["full", "act", "diag"])
+def test_sweep_special_weights_with_oracle_hessians(mode):
+    w = _special_weights()
+    G, R, C = w.shape
+    nblk = C // 16
+    rng = np.random.default_rng(9)
+    x = (rng.normal(size=(200, C)) * rng.lognormal(0, 1, C)).astype(np.float32)
+    if mode == "diag":
+        h = np.broadcast_to(O.importance_sum(x), (G, nblk, 16)).astype(np.float32)
+        p = None
+    elif mode == "act":
+        xq = (x * 0.95 + rng.normal(0, 0.05, x.shape)).astype(np.float32)
+        hs, ps = O.hessian_sum_act(x, xq)
+        h = np.broadcast_to(hs / 200, (G, nblk, 16, 16)).astype(np.float32)
+        p = np.broadcast_to(ps / 200, (G, nblk, 16, 16)).astype(np.float32)
+    else:
+        h = np.broadcast_to(O.hessian_sum_full(x) / 200, (G, nblk, 16, 16)).astype(np.float32)
+        p = None
+    g = np.array([O.global_scale(w[e]) for e in range(G)], np.float32)
+    assert g[2] == 0
+    codes, wq, loss = _sweep_gpu(L.MODE_IDS[mode], w, h, p, g)
+    units = P.all_units(G, R, nblk)
+    ref = O.sweep(mode, w, h.astype(np.float64), None if p is None else p.astype(np.float64), g, units)
+    gc, gw, gl = P.gather_gpu_units(codes, wq, loss, units)
+    P.check_sweep(gc, gw, gl, ref, f"special {mode}")
+    # Degenerate units: every candidate ties, the lowest code wins, outputs are signed zeros.
+    assert np.all(codes[2] == 1) and np.all(codes[0, 0] == 1)
+    assert np.all(wq[2] == 0) and np.all(wq[0, 1, 16:32].view(np.int32) == np.float32(-0.0).view(np.int32))
+
+
+def test_sweep_identity_hessian_is_plain_mse():
+    rng = np.random.default_rng(10)
+    w = rng.normal(0, 0.05, (1, 64, 96)).astype(np.float32)
+    h = np.broadcast_to(np.eye(16, dtype=np.float32), (1, 6, 16, 16)).copy()
+    g = np.array([O.global_scale(w[0])], np.float32)
+    codes, wq, loss = _sweep_gpu(L.FULL, w, h, None, g)
+    # Plain block MSE of the GPU's own fake-quant output equals its reported loss.
+    mse = ((wq.astype(np.float64) - w.astype(np.float64)) ** 2).reshape(1, 64, 6, 16).sum(-1)
+    np.testing.assert_allclose(loss, mse, rtol=1e-5)
+    ref = O.sweep("full", w, h.astype(np.float64), None, g)
+    P.check_sweep(codes.reshape(-1), wq.reshape(-1, 16), loss.reshape(-1), ref, "identity H")
+
+
+# ----------------------------------------------------------------------------- accumulate semantics
+
+def test_accumulate_add_equals_one_pass_and_is_deterministic():
+    layer = synth.make_layer("act", 11, tokens=700, cin=96, rows=8)
+    d = P.layer_to_device(layer)
+    x, xq = d["x"], d["xq"]
+    nb = 96 // 16
+    ws_bytes = max(L.lhcal_accumulate_workspace("act", L.BF16, 700, 96, 1), 4)
+    ws = torch.empty(ws_bytes // 4, dtype=torch.float32, device="cuda")
+    h1 = torch.empty((1, nb, 16, 16), dtype=torch.float32, device="cuda")
+    p1 = torch.empty_like(h1)
+    L.lhcal_accumulate("act", x[:300], h1, xq=xq[:300], p=p1, flags=L.ACCUM_OVERWRITE, workspace=ws)
+    L.lhcal_accumulate("act", x[300:], h1, xq=xq[300:], p=p1, flags=L.ACCUM_ADD, workspace=ws)
+    h2 = torch.empty_like(h1)
+    p2 = torch.empty_like(h1)
+    h3 = torch.empty_like(h1)
+    p3 = torch.empty_like(h1)
+    L.lhcal_accumulate("act", x, h2, xq=xq, p=p2, flags=L.ACCUM_OVERWRITE, workspace=ws)
+    L.lhcal_accumulate("act", x, h3, xq=xq, p=p3, flags=L.ACCUM_OVERWRITE, workspace=ws)
+    _sync()
+    hs, ps, _ = _oracle_hessians(layer)
+    P.check_hessians(h1.cpu().numpy(), hs, "two-call H")
+    P.check_hessians(p1.cpu().numpy(), ps, "two-call P")
+    assert torch.equal(h2.view(torch.int32), h3.view(torch.int32))
+    assert torch.equal(p2.view(torch.int32), p3.view(torch.int32))
+
+
+def test_accumulate_strided_rows_and_zero_tokens():
+    layer = synth.make_layer("dense", 12, tokens=333, cin=64, rows=4)
+    d = P.layer_to_device(layer)
+    wide = torch.zeros((333, 96), dtype=torch.bfloat16, device="cuda")
+    wide[:, :64] = d["x"]
+    xs = wide[:, :64]  # row stride 96 elements
+    h = torch.full((1, 4, 16, 16), 7.0, dtype=torch.float32, device="cuda")
+    ws_bytes = L.lhcal_accumulate_workspace("full", L.BF16, 333, 64, 1)
+    ws = torch.empty(ws_bytes // 4, dtype=torch.float32, device="cuda")
+    L.lhcal_accumulate("full", xs, h, flags=L.ACCUM_OVERWRITE, workspace=ws)
+    _sync()
+    hs, _, _ = _oracle_hessians(layer)
+    P.check_hessians(h.cpu().numpy(), hs, "strided H")
+    # Zero tokens: OVERWRITE zeroes the sums, ADD leaves them.
+    h0 = torch.full((1, 4, 16, 16), 3.0, dtype=torch.float32, device="cuda")
+    L.lhcal_accumulate("full", xs[:0], h0, flags=L.ACCUM_ADD)
+    _sync()
+    assert torch.all(h0 == 3.0)
+    L.lhcal_accumulate("full", xs[:0], h0, flags=L.ACCUM_OVERWRITE)
+    _sync()
+    assert torch.all(h0 == 0.0)
+
+
+def test_device_and_host_pointer_errors():
+    w = torch.zeros((1, 4, 32), dtype=torch.bfloat16)
+    g = torch.zeros(1, dtype=torch.float32)
+    with pytest.raises(L.LhcalError) as e:
+        L.lhcal_global_scale(w, g)  # host tensors
+    assert e.value.status == L.ERR_INVALID_ARG
+    flat = torch.zeros(256, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(L.LhcalError) as e:
+        L.lhcal_global_scale(flat[4:68].view(1, 2, 32), g.cuda())  # 8-byte offset: misaligned
+    assert e.value.status == L.ERR_INVALID_ARG
+
+
+# ----------------------------------------------------------------------------- full-size workloads
+
+@pytest.mark.parametrize("name", ["dense", "act", "wmse", "moe"])
+def test_full_size_workload(name):
+    layer = synth.make_layer(name, 0)
+    G, R, C = layer.groups, layer.rows, layer.cin
+    units = P.sample_units(G, R, C // 16, 3000, seed=1)
+    if name == "wmse":
+        _run_and_check_wmse_full(layer, units)
+    else:
+        _run_and_check(layer, units=units, check_raw=False)
+
+
+def _run_and_check_wmse_full(layer, units):
+    """Full-size WMSE: the oracle's importance is accumulated over row chunks (fp64 sums)."""
+    d = P.layer_to_device(layer)
+    b = L.calibrate("diag", d["x"], d["w"])
+    _sync()
+    imp = np.zeros((layer.cin // 16, 16))
+    for lo in range(0, layer.tokens, 4096):
+        imp += O.importance_sum(synth.bf16_bits_to_f32(layer.x[lo:lo + 4096]))
+    h, _ = O.finalize("diag", imp[None], None, np.array([layer.tokens]))
+    P.check_hessians(b.h.cpu().numpy(), h, "wmse Imp")
+    w32 = layer.w_f32()
+    g = np.array([O.global_scale(w32[0])], np.float32)
+    np.testing.assert_array_equal(b.g.cpu().numpy().view(np.int32), g.view(np.int32))
+    ref = O.sweep("diag", w32, h, None, g, units)
+    gc, gw, gl = P.gather_gpu_units(b.codes, b.wq, b.loss, units)
+    P.check_sweep(gc, gw, gl, ref, "wmse full")
