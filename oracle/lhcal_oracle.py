@@ -253,8 +253,26 @@ def sweep_units(mode: str, w_blk, h_blk, p_blk, g):
         "loss": best,
         "second": second,
         "e0": e0,
+        "escale": loss_scale(mode, w_blk, h_blk, p_blk),
         "all_losses": loss,
     }
+
+
+def loss_scale(mode: str, w_blk, h_blk, p_blk) -> np.ndarray:
+    """|w|^T |H| |w| (+ 2 |w|^T |P| |w| for ACT; sum Imp w^2 for DIAG) per unit.
+
+    The magnitude that bounds the rounding error of any Hessian-weighted loss of this block
+    evaluated in finite precision; it is >= E0 and equals it for a diagonal H. Parity gaps
+    and loss errors are measured relative to max(|L*|, this scale).
+    """
+    a = np.abs(np.asarray(w_blk, dtype=np.float64))
+    h = np.abs(np.asarray(h_blk, dtype=np.float64))
+    if mode == "diag":
+        return np.einsum("ui,ui->u", a * a, h)
+    s = np.einsum("ui,uij,uj->u", a, h, a)
+    if mode == "act":
+        s = s + 2.0 * np.einsum("ui,uij,uj->u", a, np.abs(np.asarray(p_blk, dtype=np.float64)), a)
+    return s
 
 
 def gather_units(mode: str, w, h, p, g, units):
@@ -288,7 +306,7 @@ def sweep(mode: str, w, h, p, g, units=None, chunk: int = 512):
         sub = units[lo:lo + chunk]
         wb, hb, pb, gu = gather_units(mode, w, h, p, g, sub)
         # Units in a chunk may belong to different groups: sweep each group's slice.
-        res = {k: [] for k in ("codes", "wq", "loss", "second", "e0")}
+        res = {k: [] for k in ("codes", "wq", "loss", "second", "e0", "escale")}
         order = []
         for gv in np.unique(gu):
             sel = np.nonzero(gu == gv)[0]

@@ -102,6 +102,13 @@ def test_moe_grouped_with_empty_experts():
     _run_and_check(layer)
 
 
+def test_moe_grouped_full_rank_experts():
+    layer = synth.make_layer("moe", 13, tokens=600, cin=272, rows=150, groups=24, top_k=4)
+    assert np.diff(layer.group_offsets).min() >= 32
+    r = _run_and_check(layer)
+    assert r["sweep"]["exempt"] < 0.05 * r["sweep"]["units"]
+
+
 def test_moe_grouped_diag_bf16_generic_path():
     layer = synth.make_layer("moe", 5, tokens=50, cin=48, rows=20, groups=8, top_k=2)
     layer.mode = "diag"
