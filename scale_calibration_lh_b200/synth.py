@@ -239,7 +239,7 @@ class Layer:
         return self.x if self.dtype == "f32" else bf16_bits_to_f32(self.x)
 
     def xq_f32(self) -> np.ndarray:
-        return bf16_bits_to_f32(self.xq)
+        return self.xq if self.dtype == "f32" else bf16_bits_to_f32(self.xq)
 
     def w_f32(self) -> np.ndarray:
         return self.w if self.dtype == "f32" else bf16_bits_to_f32(self.w)
