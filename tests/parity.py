@@ -87,9 +87,9 @@ def gather_gpu_units(codes, wq, loss, units):
     u = np.asarray(units, dtype=np.int64)
     ge, r, n = u[:, 0], u[:, 1], u[:, 2]
     cols = n[:, None] * 16 + np.arange(16)[None, :]
-    if hasattr(codes, "device"):
-        import torch
+    import torch
 
+    if isinstance(codes, torch.Tensor):
         dev = codes.device
         tg, tr, tn = (torch.from_numpy(a).to(dev) for a in (ge, r, n))
         tc = torch.from_numpy(cols).to(dev)
