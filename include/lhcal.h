@@ -144,6 +144,32 @@ lhcal_status lhcal_scale_sweep(lhcal_mode mode, lhcal_dtype dtype, const void* w
                                const float* g, uint8_t* codes, float* wq, float* loss, void* stream);
 
 /*
+ * lhcal_accumulate for callers that cannot allocate device memory. The pages have no
+ * counterpart to this call: it exists for deployment. Some callers cannot call cudaMalloc:
+ * a plugin that a host framework hands only input and output pointers, a runtime whose
+ * memory planner owns every device allocation up front, or code that must not trigger the
+ * implicit device synchronisation an allocation can cause. They cannot provide the
+ * workspace lhcal_accumulate asks for.
+ *
+ * Same arguments and results as lhcal_accumulate, without workspace. The split partials go
+ * to a fixed scratch array of LHCAL_NOALLOC_SCRATCH_BYTES compiled into the library: every
+ * GPU that loads the library holds it until the process exits. Sizes whose workspace
+ * (lhcal_accumulate_workspace) exceeds it are rejected with LHCAL_ERR_INVALID_ARG before
+ * anything is enqueued. The call allocates nothing and frees nothing.
+ *   - The first call on each device looks up the scratch's device address (with that device
+ *     current); make that first call before any stream capture on the device.
+ *   - All calls on a device share the one scratch array, and it keeps the last call's
+ *     contents. The kernels overwrite every partial before reading it, so no clearing is
+ *     needed. Calls that can overlap on the GPU (on different streams, or from different
+ *     threads without ordering) race on the scratch and give wrong results: order them.
+ */
+#define LHCAL_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+lhcal_status lhcal_accumulate_noalloc(lhcal_mode mode, lhcal_dtype dtype, const void* x, const void* xq,
+                                      int64_t tokens, int64_t cin, int64_t ldx, int32_t groups,
+                                      const int32_t* group_offsets, const int32_t* token_ids, int32_t flags,
+                                      float* h, float* p, void* stream);
+
+/*
  * Number of kernels this library enqueued from the calling thread since the last reset
  * (reset != 0 returns the count and sets it to zero). Host-side bookkeeping only.
  */

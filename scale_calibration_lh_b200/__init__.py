@@ -46,6 +46,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     sigs = {
         "lhcal_accumulate_workspace": [i32, i32, i64, i64, i32, ctypes.POINTER(sz)],
         "lhcal_accumulate": [i32, i32, vp, vp, i64, i64, i64, i32, vp, vp, i32, vp, vp, vp, sz, vp],
+        "lhcal_accumulate_noalloc": [i32, i32, vp, vp, i64, i64, i64, i32, vp, vp, i32, vp, vp, vp],
         "lhcal_count_tokens": [i32, i64, vp, i32, vp, vp],
         "lhcal_finalize": [i32, i32, i64, vp, vp, vp, vp],
         "lhcal_global_scale": [i32, vp, i32, i64, i64, vp, vp],
@@ -125,6 +126,28 @@ def lhcal_accumulate(mode, x, h, xq=None, p=None, group_offsets=None, token_ids=
         m, _dtype_id(x), _ptr(x), _ptr(xq), tokens, cin, int(x.stride(0)), groups,
         _ptr(group_offsets), _ptr(token_ids), flags, _ptr(h), _ptr(p), _ptr(workspace), ws_bytes,
         _stream(stream)))
+
+
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
+
+
+def lhcal_accumulate_noalloc(mode, x, h, xq=None, p=None, group_offsets=None, token_ids=None,
+                             flags: int = ACCUM_ADD, stream=None):
+    """lhcal_accumulate for callers that cannot allocate: uses the library's fixed scratch.
+
+    For callers whose device memory is owned by someone else (a host framework's memory
+    planner, a plugin handed only its inputs and outputs) and who therefore cannot supply
+    a workspace. Sizes needing more than NOALLOC_SCRATCH_BYTES of scratch are rejected;
+    calls that may overlap on the GPU share the scratch and must be ordered.
+    """
+    m = _mode_id(mode)
+    tokens, cin = int(x.shape[0]), int(x.shape[1])
+    if x.stride(1) != 1:
+        raise ValueError("x must have unit stride along cin")
+    groups = 1 if group_offsets is None else int(group_offsets.numel()) - 1
+    _check(load_library().lhcal_accumulate_noalloc(
+        m, _dtype_id(x), _ptr(x), _ptr(xq), tokens, cin, int(x.stride(0)), groups,
+        _ptr(group_offsets), _ptr(token_ids), flags, _ptr(h), _ptr(p), _stream(stream)))
 
 
 def lhcal_count_tokens(counts, tokens: int = 0, group_offsets=None, flags: int = ACCUM_ADD, stream=None):
