@@ -19,9 +19,7 @@ import argparse
 import datetime
 import json
 import os
-import subprocess
 import sys
-import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -64,48 +62,68 @@ def load_peaks():
 # ------------------------------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Polls the SM clock and clock-event reasons (NVML, read-only) every 5 ms in a thread."""
 
-    def __init__(self, device_index: int):
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
         self.device_index = device_index
-        self.proc = None
-        self.path = None
+        self.period_s = period_s
+        self.samples = []
+        self._stop = None
+        self._thread = None
+        self.error = None
 
     def start(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
+        import threading
+
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.device_index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            import pynvml
+
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = self.device_index
+            if vis:
+                ids = [v.strip() for v in vis.split(",") if v.strip()]
+                if idx < len(ids) and ids[idx].isdigit():
+                    idx = int(ids[idx])
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self._nv = pynvml
+            self.sm_max = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.error = f"nvml unavailable: {e}"
+            return
+        self._stop = threading.Event()
+
+        def poll():
+            nv, h = self._nv, self._h
+            while not self._stop.is_set():
+                try:
+                    self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                         nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+                except Exception:
+                    pass
+                time.sleep(self.period_s)
+
+        self._thread = threading.Thread(target=poll, daemon=True)
+        self._thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = sorted(float(r[1]) for r in rows if r[1].replace(".", "").isdigit())
-        smax = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
-        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": smax, "reasons": reasons,
-                "samples": len(rows)}
+        if self._thread is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.error or "not sampled"]}
+        self._stop.set()
+        self._thread.join()
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.sm_max, "reasons": ["no samples"]}
+        sm = sorted(c for c, _ in self.samples)
+        reasons = sorted({name for _, bits in self.samples for name, const in self.REASONS
+                          if bits & getattr(self._nv, const, 0)})
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": self.sm_max, "sm_min_mhz": sm[0], "reasons": reasons,
+                "samples": len(self.samples)}
 
 
 # ------------------------------------------------------------------------------------------ helpers
@@ -254,14 +272,13 @@ def run_lhcal(args, rank, world, local_rank):
 
     # ---- device-resident timed region, with per-stage events on the launching stream
     clocks = ClockSampler(torch.cuda.current_device())
-    clocks.start()
-    time.sleep(0.3)
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     L.lhcal_launch_count(reset=True)
+    clocks.start()
     start.record(stream)
     for k in range(K):
         e = ev[k]
@@ -278,9 +295,9 @@ def run_lhcal(args, rank, world, local_rank):
         e[4].record(stream)
     end.record(stream)
     torch.cuda.synchronize()
+    clk = clocks.stop()
     barrier()
     launches = L.lhcal_launch_count()
-    clk = clocks.stop()
     ms_total = start.elapsed_time(end)
     stage = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in ev])  # ms
     t_acc, t_fin, t_g, t_sweep = (float(v) for v in stage.mean(0))
@@ -370,7 +387,7 @@ def run_lhcal(args, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["lhcal", "reference"], default="lhcal")
     ap.add_argument("--workload", choices=list(WORKLOAD_TEXT), default="dense")
