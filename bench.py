@@ -59,6 +59,23 @@ def load_peaks():
         return FALLBACK_HBM_GBS, FALLBACK_SM_MHZ, "fallback"
 
 
+def rank_max(values, device=None):
+    """Element-wise maximum of a list of floats over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def weak_scaling_value(units_per_rank: int, world: int, ms_per_step_max: float) -> float:
+    """Whole-job throughput: every rank's units over the slowest rank's step time."""
+    return units_per_rank * world / (ms_per_step_max / 1e3)
+
+
 # ------------------------------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -301,13 +318,10 @@ def run_lhcal(args, rank, world, local_rank):
     ms_total = start.elapsed_time(end)
     stage = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in ev])  # ms
     t_acc, t_fin, t_g, t_sweep = (float(v) for v in stage.mean(0))
-    if dist:
-        t = torch.tensor([ms_total, t_acc, t_sweep], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_total, t_acc, t_sweep = (float(v) for v in t.tolist())
+    ms_total, t_acc, t_sweep = rank_max([ms_total, t_acc, t_sweep], dev)
     ms = ms_total / K
     units, ops, acc_bytes = algorithmic(layer)
-    value = units * world / (ms / 1e3)
+    value = weak_scaling_value(units, world, ms)
 
     # ---- end to end through the public API from pinned host buffers
     hx = torch.empty(d["x"].shape, dtype=d["x"].dtype, pin_memory=True)
@@ -336,10 +350,7 @@ def run_lhcal(args, rank, world, local_rank):
     e2e_.record(stream)
     torch.cuda.synchronize()
     ms_e2e = e2s.elapsed_time(e2e_) / K2
-    if dist:
-        t = torch.tensor([ms_e2e], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    (ms_e2e,) = rank_max([ms_e2e], dev)
     h2d = sum(t.numel() * t.element_size() for t in (hx, hw, hxq, hoffs, hids) if t is not None)
     d2h = out_host.nbytes()
 
@@ -370,7 +381,7 @@ def run_lhcal(args, rank, world, local_rank):
                            "traffic": None, "bytes_per_step": acc_bytes,
                            "note": f"algorithmic bytes over the measured accumulation time; peak {peak_src}"},
         "stages_ms": {"accumulate": t_acc, "count_finalize": t_fin, "global_scale": t_g, "sweep": t_sweep},
-        "e2e": {"value": units * world / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": weak_scaling_value(units, world, ms_e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
         "gpu_launches": launches,
         "clocks": clk,

@@ -265,3 +265,20 @@ def test_sweep_invariances():
     d2 = O.sweep("diag", -w, imp, None, g)
     np.testing.assert_array_equal(d1["codes"], d2["codes"])
     np.testing.assert_array_equal(d1["loss"], d2["loss"])
+
+
+def test_loss_scale_bounds_e0_and_equals_it_for_diagonal_h():
+    rng = np.random.default_rng(14)
+    w = rng.normal(0, 0.05, (50, 16)).astype(np.float32)
+    a = rng.normal(size=(50, 16, 16))
+    h = a @ a.transpose(0, 2, 1)
+    _, _, e0 = O.candidate_losses("full", w, h, None, O.global_scale(w))
+    s = O.loss_scale("full", w, h, None)
+    assert np.all(s >= e0 - 1e-12 * s)
+    hd = np.zeros_like(h)
+    idx = np.arange(16)
+    hd[:, idx, idx] = np.abs(rng.normal(size=(50, 16)))
+    _, _, e0d = O.candidate_losses("full", w, hd, None, O.global_scale(w))
+    np.testing.assert_allclose(O.loss_scale("full", w, hd, None), e0d, rtol=1e-13)
+    imp = hd[:, idx, idx]
+    np.testing.assert_allclose(O.loss_scale("diag", w, imp, None), e0d, rtol=1e-13)
