@@ -70,6 +70,10 @@ lhcal_status launch_sweep(lhcal_mode mode, lhcal_dtype dtype, const void* w, int
                           int64_t rows, int64_t cin, const float* h, const float* p, const float* g,
                           uint8_t* codes, float* wq, float* loss, cudaStream_t stream);
 
+lhcal_status launch_sweep_tc(lhcal_mode mode, lhcal_dtype dtype, const void* w, int32_t groups,
+                             int64_t rows, int64_t cin, const float* h, const float* p, const float* g,
+                             uint8_t* codes, float* wq, float* loss, cudaStream_t stream);
+
 size_t accumulate_workspace_bytes(lhcal_mode mode, lhcal_dtype dtype, int64_t tokens, int64_t cin,
                                   int32_t groups);
 

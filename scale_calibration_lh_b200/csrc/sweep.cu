@@ -24,55 +24,20 @@
 //  * Loss: L = sum_i t_i e_i with t_i = H_ii e_i + sum_{j>i} (H_ij + H_ji) s_i s_j e_j (+ 2 c_i
 //    for the cross term), where e_i = |wq_i| - |w_i| and s_i = sign(w_i); dW_i = s_i e_i.
 #include "common.cuh"
+#include "quant_tables.cuh"
 
 namespace lhcal {
 namespace {
 
-constexpr int kCand = LHCAL_N_CANDIDATES;
-constexpr int kLev = 8;
 constexpr int kThreads = 128;
-
-__device__ __forceinline__ float pow2i(int e) {  // exact 2^e for -126 <= e <= 127
-  return __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
-}
-
-// E4M3 value of code (1..126), exact in fp32.
-__device__ __forceinline__ float e4m3_value(int code) {
-  const int e = code >> 3, m = code & 7;
-  return e == 0 ? static_cast<float>(m) * pow2i(-9) : static_cast<float>(8 + m) * pow2i(e - 10);
-}
-
-__device__ __forceinline__ float e2m1_grid(int j) {
-  // 0, 0.5, 1, 1.5, 2, 3, 4, 6
-  return j < 5 ? 0.5f * static_cast<float>(j) : (j == 5 ? 3.f : (j == 6 ? 4.f : 6.f));
-}
-
-__device__ __forceinline__ float e2m1_lower_midpoint(int j) {
-  // Midpoint between grid[j - 1] and grid[j]: 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.
-  return 0.5f * (e2m1_grid(j - 1) + e2m1_grid(j));
-}
-
-__device__ __forceinline__ float next_up(float x) {  // x >= 0, finite
-  return __uint_as_float(__float_as_uint(x) + 1u);
-}
 
 // Candidate table for one global scale g, interleaved per (candidate k, level j):
 // tab[2 * (8k + j)] = thr[k][j], tab[2 * (8k + j) + 1] = val[k][j] (see file comment).
 __device__ void build_tables(float* tab, float g) {
   for (int idx = threadIdx.x; idx < kCand * kLev; idx += blockDim.x) {
     const int k = idx >> 3, j = idx & 7;
-    const float s = __fmul_rn(e4m3_value(k + 1), g);
-    float t = 0.f;
-    if (j > 0) {
-      const float m = e2m1_lower_midpoint(j);
-      const float prod = __fmul_rn(m, s);
-      const float resid = __fmaf_rn(m, s, -prod);  // exact m*s - prod (sign is exact)
-      // Ties at the midpoint go to the even code: up for even j, down for odd j.
-      const bool tie_up = (j & 1) == 0;
-      // |w| >= t  <=>  |w| / s rounds to level >= j.
-      t = (resid < 0.f || (resid == 0.f && tie_up)) ? prod : next_up(prod);
-    }
-    tab[2 * idx] = t;
+    const float s = candidate_scale(k, g);
+    tab[2 * idx] = level_threshold(j, s);
     tab[2 * idx + 1] = __fmul_rn(e2m1_grid(j), s);
   }
 }
@@ -322,16 +287,14 @@ lhcal_status launch_sweep(lhcal_mode mode, lhcal_dtype dtype, const void* w, int
   if (rows > static_cast<int64_t>(65535) * kThreads * 1024 || cin / kBlock > 65535 || groups > 65535)
     return fail(LHCAL_ERR_INVALID_ARG, "scale sweep: grid too large (rows %lld, cin %lld, groups %d)",
                 (long long)rows, (long long)cin, groups);
+  // FULL and ACT_AWARE: quadratic form on tensor cores; DIAG: FP32 weighted sum.
+  if (mode == LHCAL_FULL || mode == LHCAL_ACT_AWARE)
+    return launch_sweep_tc(mode, dtype, w, groups, rows, cin, h, p, g, codes, wq, loss, stream);
 #define LHCAL_SWEEP_CASE(M, T)                                                                   \
   return launch_mode<M, T>(w, groups, rows, cin, h, p, g, codes, wq, loss, stream)
-  if (dtype == LHCAL_BF16) {
-    if (mode == LHCAL_FULL) LHCAL_SWEEP_CASE(LHCAL_FULL, __nv_bfloat16);
-    if (mode == LHCAL_ACT_AWARE) LHCAL_SWEEP_CASE(LHCAL_ACT_AWARE, __nv_bfloat16);
-    if (mode == LHCAL_DIAG) LHCAL_SWEEP_CASE(LHCAL_DIAG, __nv_bfloat16);
-  } else {
-    if (mode == LHCAL_FULL) LHCAL_SWEEP_CASE(LHCAL_FULL, float);
-    if (mode == LHCAL_ACT_AWARE) LHCAL_SWEEP_CASE(LHCAL_ACT_AWARE, float);
-    if (mode == LHCAL_DIAG) LHCAL_SWEEP_CASE(LHCAL_DIAG, float);
+  if (mode == LHCAL_DIAG) {
+    if (dtype == LHCAL_BF16) LHCAL_SWEEP_CASE(LHCAL_DIAG, __nv_bfloat16);
+    LHCAL_SWEEP_CASE(LHCAL_DIAG, float);
   }
 #undef LHCAL_SWEEP_CASE
   return fail(LHCAL_ERR_UNSUPPORTED, "scale sweep: unsupported mode/dtype");
