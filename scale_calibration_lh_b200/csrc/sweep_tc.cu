@@ -52,6 +52,8 @@ struct __align__(16) TcShared {
   float h[256];
   float p[256];
   float hscale;  // 2^-eH: H' = H * hscale lies below 2^15
+  float key[kUnitsPerCta];  // min |w| of each of the CTA's units (rows)
+  int perm[kUnitsPerCta];   // the CTA's rows ordered by key
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -144,7 +146,30 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
     sh.tab[idx] = make_float4(level_threshold(j, s), __uint_as_float(q16), __uint_as_float(q16 << 16),
                               __fmul_rn(e2m1_grid(j), s));
   }
+  // Order the CTA's rows by their smallest |w|, so that the units a warp evaluates together
+  // leave the all-clamped candidates at similar scales (see the clamped prefix below).
+  const int64_t rbase = static_cast<int64_t>(blockIdx.x) * kUnitsPerCta;
+  if (threadIdx.x < kUnitsPerCta) {
+    const int64_t row = rbase + threadIdx.x;
+    float m = __int_as_float(0x7f800000);
+    if (row < rows) {
+      float wt[16];
+      load_row16<WT>(w + (e * rows + row) * cin + n * kBlock, true, wt);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) m = fminf(m, fabsf(wt[i]));
+    }
+    sh.key[threadIdx.x] = m;
+  }
   __syncthreads();
+  if (threadIdx.x < kUnitsPerCta) {
+    const float my = sh.key[threadIdx.x];
+    int rank = 0;
+    for (int j = 0; j < kUnitsPerCta; ++j) {
+      const float kj = sh.key[j];
+      rank += (kj < my || (kj == my && j < static_cast<int>(threadIdx.x))) ? 1 : 0;
+    }
+    sh.perm[rank] = threadIdx.x;
+  }
   if (warp == 0) {
     uint32_t m = 0;
     for (int i = lane; i < 256; i += 32) m = max(m, __float_as_uint(sh.h[i]) & 0x7fffffffu);
@@ -182,14 +207,13 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
     }
   }
 
-  // ---- the warp's 16 units: rows r0 + gq (unit 0) and r0 + gq + 8 (unit 1)
-  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kUnitsPerCta + warp * kUnitsPerWarp;
+  // ---- the warp's 16 units: sorted positions 16 warp + gq (unit 0) and + 8 (unit 1)
   int64_t ur[2];
   bool valid[2];
   float wrow[2][16];
 #pragma unroll
   for (int u = 0; u < 2; ++u) {
-    ur[u] = r0 + gq + 8 * u;
+    ur[u] = rbase + sh.perm[warp * kUnitsPerWarp + gq + 8 * u];
     valid[u] = ur[u] < rows;
     load_row16<WT>(w + (e * rows + (valid[u] ? ur[u] : 0)) * cin + n * kBlock, valid[u], wrow[u]);
   }
