@@ -33,12 +33,15 @@
 namespace lhcal {
 namespace {
 
-// CTAs per SM the register allocation targets (launch bounds).
+// Warps per CTA (16 units each) and the CTAs per SM that the register allocation targets.
+#ifndef LHCAL_TC_WARPS
+#define LHCAL_TC_WARPS 8
+#endif
 #ifndef LHCAL_TC_MIN_BLOCKS
-#define LHCAL_TC_MIN_BLOCKS 5
+#define LHCAL_TC_MIN_BLOCKS 3
 #endif
 
-constexpr int kTcWarps = 4;
+constexpr int kTcWarps = LHCAL_TC_WARPS;
 constexpr int kTcThreads = 32 * kTcWarps;
 constexpr int kUnitsPerWarp = 16;
 constexpr int kUnitsPerCta = kUnitsPerWarp * kTcWarps;
