@@ -95,7 +95,7 @@ template <bool ACT>
 struct MmaCfg {
   static constexpr int kStages = ACT ? 3 : 4;
   static constexpr int kTensors = ACT ? 2 : 1;
-  static constexpr int kSmem = kStages * kTensors * kTileBytes;
+  static constexpr int kSmem = kStages * kTensors * kTileBytes + kStages * kTileTok * 4;  // + id ring
 };
 
 // Byte offset of 16-byte chunk c (0..15) of tile row r in the swizzled layout.
@@ -103,17 +103,14 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
   return static_cast<uint32_t>(r * kRowBytes + ((c ^ (r & 7)) << 4));
 }
 
-struct TokenSource {
-  // Dense: rows tok_begin .. tok_end-1. Grouped: rows ids[pos] for pos in [tok_begin, tok_end).
-  const int32_t* ids;
-  int64_t tok_begin, tok_end;
-  __device__ __forceinline__ int64_t row(int64_t pos) const { return ids ? static_cast<int64_t>(__ldg(ids + pos)) : pos; }
-};
 
+// Loads one 64-token x 128-column tile (both tensors for ACT). Rows pos0 + r for r < 64 with
+// pos0 + r < end; grouped tiles take the row of position pos0 + r from ids_s[r] (shared
+// memory), dense tiles use the position itself. Rows past end and columns past cin are zeros.
 template <bool ACT>
 __device__ __forceinline__ void load_tile(uint8_t* smem_stage, const __nv_bfloat16* x,
                                           const __nv_bfloat16* xq, int64_t ldx, int64_t col0,
-                                          int64_t cin, const TokenSource& src, int64_t pos0) {
+                                          int64_t cin, const int32_t* ids_s, int64_t pos0, int64_t end) {
   const int tid = threadIdx.x;
   const int c = tid & 15;
   const bool col_ok = col0 + c * 8 < cin;
@@ -121,8 +118,8 @@ __device__ __forceinline__ void load_tile(uint8_t* smem_stage, const __nv_bfloat
   for (int m = 0; m < kTileTok / 16; ++m) {
     const int r = (tid >> 4) + 16 * m;
     const int64_t pos = pos0 + r;
-    const bool ok = col_ok && pos < src.tok_end;
-    const int64_t row = ok ? src.row(pos) : 0;
+    const bool ok = col_ok && pos < end;
+    const int64_t row = ok ? (ids_s ? static_cast<int64_t>(ids_s[r]) : pos) : 0;
     const int64_t off = ok ? row * ldx + col0 + c * 8 : 0;
     const uint32_t dst = smem_u32(smem_stage) + swz(r, c);
     if (ACT) {
@@ -134,45 +131,164 @@ __device__ __forceinline__ void load_tile(uint8_t* smem_stage, const __nv_bfloat
   }
 }
 
-// out_h / out_p point at [8 blocks][256] for this CTA's slab (already offset); nblk_valid
-// is the number of blocks of the slab inside cin. accumulate_into: out += acc, else out = acc.
+// Copies the 64 token ids of the tile at positions [pos0, pos0 + 64) (zeros past end) into a
+// shared-memory slot with cp.async; 16 threads move 16 bytes each.
+__device__ __forceinline__ void load_ids(int32_t* slot, const int32_t* ids, int64_t pos0, int64_t end) {
+  const int tid = threadIdx.x;
+  if (tid < kTileTok / 4) {
+    const int64_t pos = pos0 + 4 * tid;
+    const uint32_t dst = smem_u32(slot + 4 * tid);
+    if (pos + 4 <= end && ((reinterpret_cast<uintptr_t>(ids + pos) & 15) == 0)) {
+      cp_async16(dst, ids + pos, true);
+    } else {
+      // Ragged or unaligned: element by element (4-byte copies), zeros past end.
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const bool ok = pos + j < end;
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(dst + 4 * j),
+                     "l"(ids + (ok ? pos + j : 0)), "r"(ok ? 4 : 0));
+      }
+    }
+  }
+}
+
+// One CTA owns a 128-column slab and a list of items: dense, one token range (a split, whose
+// sums go to the workspace); grouped, a run of consecutive groups (experts), each summed over
+// its routed rows and written to out at item * out_item_stride. A single cp.async pipeline runs
+// through the tiles of all items, so short items (about 5 tiles per expert) still stream; the
+// accumulators are written out after each item's last tile. accumulate_into: out += sums.
 template <bool ACT>
 __global__ void __launch_bounds__(kMmaThreads)
 accum_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ xq,
                  int64_t tokens, int64_t cin, int64_t ldx, const int32_t* __restrict__ group_offsets,
-                 const int32_t* __restrict__ token_ids, int64_t tok_per_split, float* __restrict__ out_h,
-                 float* __restrict__ out_p, int64_t out_group_stride, int64_t out_split_stride,
-                 int accumulate_into) {
+                 const int32_t* __restrict__ token_ids, int64_t tok_per_split, int64_t items_per_cta,
+                 int64_t groups, float* __restrict__ out_h, float* __restrict__ out_p,
+                 int64_t out_item_stride, int accumulate_into) {
   using Cfg = MmaCfg<ACT>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t slab = blockIdx.x;
   const int64_t col0 = slab * kSlabCols;
   const int64_t nblk = cin / kBlock;
+  const int64_t blk = slab * 8 + warp;
+  const bool blk_ok = blk < nblk;
+  const bool grouped = group_offsets != nullptr;
 
-  TokenSource src;
-  int64_t out_off;
-  if (group_offsets != nullptr) {  // grouped: blockIdx.y = group
-    src.ids = token_ids;
-    src.tok_begin = __ldg(group_offsets + blockIdx.y);
-    src.tok_end = __ldg(group_offsets + blockIdx.y + 1);
-    out_off = static_cast<int64_t>(blockIdx.y) * out_group_stride;
-  } else {  // dense: blockIdx.y = token split
-    src.ids = nullptr;
-    src.tok_begin = static_cast<int64_t>(blockIdx.y) * tok_per_split;
-    src.tok_end = imin64(tokens, src.tok_begin + tok_per_split);
-    out_off = static_cast<int64_t>(blockIdx.y) * out_split_stride;
+  int64_t it0, it1;  // this CTA's items
+  if (grouped) {
+    it0 = static_cast<int64_t>(blockIdx.y) * items_per_cta;
+    it1 = imin64(groups, it0 + items_per_cta);
+  } else {
+    it0 = blockIdx.y;
+    it1 = it0 + 1;
   }
-  const int64_t ntiles = ceil_div(imax64(src.tok_end - src.tok_begin, 0), kTileTok);
+  // Grouped: this CTA's slice of the offsets, staged in shared memory after the pipeline ring.
+  int32_t* offs_s = reinterpret_cast<int32_t*>(smem + Cfg::kSmem);
+  if (grouped) {
+    for (int64_t i = threadIdx.x; i <= it1 - it0; i += kMmaThreads) offs_s[i] = __ldg(group_offsets + it0 + i);
+    __syncthreads();
+  }
+  auto range = [&](int64_t item, int64_t& b, int64_t& e) {
+    if (grouped) {
+      b = offs_s[item - it0];
+      e = offs_s[item - it0 + 1];
+    } else {
+      b = item * tok_per_split;
+      e = imin64(tokens, b + tok_per_split);
+    }
+  };
+
+  // Accumulator layout of m16n8: c0,c1 -> (i = lane/4, j = 2*(lane%4) + {0,1}); c2,c3 -> i + 8.
+  const int i0 = lane >> 2, j0 = 2 * (lane & 3);
+  auto write_out = [&](int64_t item, const float (&ah)[2][4], const float (&ap)[2][4]) {
+    if (!blk_ok) return;
+    float* oh = out_h + item * out_item_stride + blk * 256;
+    float* op = ACT ? out_p + item * out_item_stride + blk * 256 : nullptr;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int idx = (i0 + 8 * half) * 16 + nt * 8 + j0;
+        float2 vh = make_float2(ah[nt][2 * half], ah[nt][2 * half + 1]);
+        if (accumulate_into) {
+          const float2 o = *reinterpret_cast<const float2*>(oh + idx);
+          vh.x += o.x;
+          vh.y += o.y;
+        }
+        *reinterpret_cast<float2*>(oh + idx) = vh;
+        if (ACT) {
+          float2 vp = make_float2(ap[nt][2 * half], ap[nt][2 * half + 1]);
+          if (accumulate_into) {
+            const float2 o = *reinterpret_cast<const float2*>(op + idx);
+            vp.x += o.x;
+            vp.y += o.y;
+          }
+          *reinterpret_cast<float2*>(op + idx) = vp;
+        }
+      }
+    }
+  };
 
   float acc_h[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   float acc_p[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 
+  // Tiles over all items; items without rows produce zeros (OVERWRITE) or nothing (ADD).
+  int64_t ntiles = 0;
+  for (int64_t item = it0; item < it1; ++item) {
+    int64_t b, e;
+    range(item, b, e);
+    if (e > b) ntiles += ceil_div(e - b, kTileTok);
+    else if (!accumulate_into) write_out(item, acc_h, acc_p);
+  }
+
+  // Cursors (item, position, end): ids of tiles 2S-2 ahead of consumption (grouped), data of
+  // tiles S-1 ahead, and the tile being consumed.
+  auto first_nonempty = [&](int64_t item, int64_t& pos, int64_t& end) -> int64_t {
+    for (; item < it1; ++item) {
+      int64_t b, e;
+      range(item, b, e);
+      if (e > b) {
+        pos = b;
+        end = e;
+        return item;
+      }
+    }
+    return it1;
+  };
   constexpr int S = Cfg::kStages;
   constexpr int stage_bytes = Cfg::kTensors * kTileBytes;
+  int32_t* ids_ring = reinterpret_cast<int32_t*>(smem + S * stage_bytes);  // S slots of 64 ids
+  int64_t i_pos = 0, i_end = 0, p_pos = 0, p_end = 0, c_pos = 0, c_end = 0;
+  int64_t i_item = first_nonempty(it0, i_pos, i_end);
+  int64_t i_tile = 0;
+  int64_t p_item = first_nonempty(it0, p_pos, p_end);
+  int64_t c_item = first_nonempty(it0, c_pos, c_end);
+  (void)p_item;
+  auto issue_ids = [&]() {  // ids of tile i_tile into slot i_tile % S
+    if (grouped && i_tile < ntiles) {
+      load_ids(ids_ring + (i_tile % S) * kTileTok, token_ids, i_pos, i_end);
+      i_pos += kTileTok;
+      if (i_pos >= i_end) i_item = first_nonempty(i_item + 1, i_pos, i_end);
+    }
+    ++i_tile;
+  };
+  auto produce = [&](int64_t tile) {  // data of tile into stage tile % S
+    load_tile<ACT>(smem + (tile % S) * stage_bytes, x, xq, ldx, col0, cin,
+                   grouped ? ids_ring + (tile % S) * kTileTok : nullptr, p_pos, p_end);
+    p_pos += kTileTok;
+    if (p_pos >= p_end) p_item = first_nonempty(p_item + 1, p_pos, p_end);
+  };
+
+  // Ids of the first S - 1 tiles, then the prologue: data of tiles 0..S-2 and ids S-1..2S-3.
+  for (int s2 = 0; s2 < S - 1; ++s2) issue_ids();
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
 #pragma unroll
-  for (int s = 0; s < S - 1; ++s) {
-    if (s < ntiles) load_tile<ACT>(smem + s * stage_bytes, x, xq, ldx, col0, cin, src, src.tok_begin + s * kTileTok);
+  for (int s2 = 0; s2 < S - 1; ++s2) {
+    __syncthreads();  // the id slot refilled below was read by every thread for tile s2 - 1
+    issue_ids();
+    if (s2 < ntiles) produce(s2);
     cp_async_commit();
   }
 
@@ -185,12 +301,9 @@ accum_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __res
   for (int64_t it = 0; it < ntiles; ++it) {
     cp_async_wait<S - 2>();
     __syncthreads();
-    {
-      const int64_t nt = it + S - 1;
-      if (nt < ntiles)
-        load_tile<ACT>(smem + (nt % S) * stage_bytes, x, xq, ldx, col0, cin, src, src.tok_begin + nt * kTileTok);
-      cp_async_commit();
-    }
+    issue_ids();  // tile it + 2S - 2
+    if (it + S - 1 < ntiles) produce(it + S - 1);
+    cp_async_commit();
     const uint32_t base = smem_u32(smem + (it % S) * stage_bytes);
 #pragma unroll
     for (int ts = 0; ts < kTileTok / 16; ++ts) {
@@ -213,38 +326,17 @@ accum_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __res
         mma_bf16(acc_p[1], q0, q1, q2, q3, l1, l3);
       }
     }
-  }
-  cp_async_wait<0>();
-
-  const int64_t blk = slab * 8 + warp;
-  if (blk >= nblk) return;
-  // Accumulator layout of m16n8: c0,c1 -> (i = lane/4, j = 2*(lane%4) + {0,1}); c2,c3 -> i + 8.
-  const int i0 = lane >> 2, j0 = 2 * (lane & 3);
-  float* oh = out_h + out_off + blk * 256;
-  float* op = ACT ? out_p + out_off + blk * 256 : nullptr;
+    c_pos += kTileTok;
+    if (c_pos >= c_end) {  // last tile of the consumer's item: write its sums
+      write_out(c_item, acc_h, acc_p);
 #pragma unroll
-  for (int nt = 0; nt < 2; ++nt) {
+      for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int idx = (i0 + 8 * half) * 16 + nt * 8 + j0;
-      float2 vh = make_float2(acc_h[nt][2 * half], acc_h[nt][2 * half + 1]);
-      if (accumulate_into) {
-        const float2 o = *reinterpret_cast<const float2*>(oh + idx);
-        vh.x += o.x;
-        vh.y += o.y;
-      }
-      *reinterpret_cast<float2*>(oh + idx) = vh;
-      if (ACT) {
-        float2 vp = make_float2(acc_p[nt][2 * half], acc_p[nt][2 * half + 1]);
-        if (accumulate_into) {
-          const float2 o = *reinterpret_cast<const float2*>(op + idx);
-          vp.x += o.x;
-          vp.y += o.y;
-        }
-        *reinterpret_cast<float2*>(op + idx) = vp;
-      }
+        for (int v = 0; v < 4; ++v) acc_h[nt][v] = acc_p[nt][v] = 0.f;
+      c_item = first_nonempty(c_item + 1, c_pos, c_end);
     }
   }
+  cp_async_wait<0>();
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -412,20 +504,22 @@ struct Split {
   int64_t per;      // tokens per split
 };
 
+// Token ranges so that splits * ctas_per_split does not exceed target_ctas (one wave of the
+// resident CTAs; a second, nearly empty wave would double the time).
 Split token_split(int64_t tokens, int64_t ctas_per_split, int64_t target_ctas, int64_t granule) {
   Split s;
   if (tokens <= 0) return {1, granule};
-  int64_t want = imax64(1, ceil_div(target_ctas, imax64(ctas_per_split, 1)));
+  int64_t want = imax64(1, target_ctas / imax64(ctas_per_split, 1));
   want = min(want, ceil_div(tokens, granule));
   s.per = ceil_div(ceil_div(tokens, want), granule) * granule;
   s.splits = ceil_div(tokens, s.per);
   return s;
 }
 
-Split split_for(Path path, int64_t tokens, int64_t cin) {
+Split split_for(Path path, lhcal_mode mode, int64_t tokens, int64_t cin) {
   switch (path) {
-    case Path::kMma:
-      return token_split(tokens, ceil_div(cin, kSlabCols), 3 * kNumSms, kTileTok);
+    case Path::kMma:  // resident CTAs per SM: 3 (FULL, 65 KB shared) or 2 (ACT, 97 KB)
+      return token_split(tokens, ceil_div(cin, kSlabCols), (mode == LHCAL_ACT_AWARE ? 2 : 3) * kNumSms, kTileTok);
     case Path::kDiagBf16:
       return token_split(tokens, ceil_div(cin, kDiagCols), 8 * kNumSms, kDiagUnroll);
     default:
@@ -459,27 +553,34 @@ lhcal_status launch_mma(const void* x, const void* xq, int64_t tokens, int64_t c
                         int32_t groups, const int32_t* offs, const int32_t* ids, int accumulate_into,
                         float* h, float* p, float* ws, cudaStream_t stream) {
   using Cfg = MmaCfg<ACT>;
-  // Set on every call: cheap, thread-safe, and correct whichever device is current.
+  // Allow up to the per-CTA maximum (the launch size decides occupancy). Set on every call with
+  // the same value: cheap, thread-safe, and correct whichever device is current.
+  constexpr int kMaxDynSmem = 227 * 1024;
   const cudaError_t attr = cudaFuncSetAttribute(accum_mma_kernel<ACT>,
-                                                cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
   if (attr != cudaSuccess) return fail(LHCAL_ERR_CUDA, "accumulate: %s", cudaGetErrorString(attr));
   const int64_t slabs = ceil_div(cin, kSlabCols);
   const int64_t nblk = cin / kBlock;
   const auto* xb = static_cast<const __nv_bfloat16*>(x);
   const auto* xqb = static_cast<const __nv_bfloat16*>(ACT ? xq : x);
   if (offs != nullptr) {
-    const dim3 grid(static_cast<unsigned>(slabs), static_cast<unsigned>(groups));
-    accum_mma_kernel<ACT><<<grid, kMmaThreads, Cfg::kSmem, stream>>>(
-        xb, xqb, tokens, cin, ldx, offs, ids, 0, h, p, nblk * 256, 0, accumulate_into);
+    // Runs of experts per CTA so that about one wave of CTAs covers all (slab, expert) items.
+    const int64_t ctas_per_sm = ACT ? 2 : 3;
+    const int64_t per = imax64(1, ceil_div(static_cast<int64_t>(groups) * slabs, ctas_per_sm * kNumSms));
+    const dim3 grid(static_cast<unsigned>(slabs), static_cast<unsigned>(ceil_div(groups, per)));
+    const size_t smem = Cfg::kSmem + static_cast<size_t>(ceil_div((per + 1) * 4, 16) * 16);
+    if (smem > static_cast<size_t>(kMaxDynSmem)) return fail(LHCAL_ERR_UNSUPPORTED, "accumulate: too many groups per CTA");
+    accum_mma_kernel<ACT><<<grid, kMmaThreads, smem, stream>>>(
+        xb, xqb, tokens, cin, ldx, offs, ids, 0, per, groups, h, p, nblk * 256, accumulate_into);
     return check_launch("accumulate (grouped, tensor cores)");
   }
-  const Split sp = split_for(Path::kMma, tokens, cin);
+  const Split sp = split_for(Path::kMma, ACT ? LHCAL_ACT_AWARE : LHCAL_FULL, tokens, cin);
   const int64_t per_split = nblk * 256;
   float* ws_h = ws;
   float* ws_p = ws + sp.splits * per_split;
   const dim3 grid(static_cast<unsigned>(slabs), static_cast<unsigned>(sp.splits));
   accum_mma_kernel<ACT><<<grid, kMmaThreads, Cfg::kSmem, stream>>>(
-      xb, xqb, tokens, cin, ldx, nullptr, nullptr, sp.per, ws_h, ws_p, 0, per_split, 0);
+      xb, xqb, tokens, cin, ldx, nullptr, nullptr, sp.per, 1, 0, ws_h, ws_p, per_split, 0);
   lhcal_status st = check_launch("accumulate (tensor cores)");
   if (st != LHCAL_OK) return st;
   st = launch_reduce(ws_h, sp.splits, per_split, per_split, h, accumulate_into, stream);
@@ -501,7 +602,7 @@ lhcal_status launch_generic(const void* x, const void* xq, int64_t tokens, int64
                                                             per_group, accumulate_into);
     return check_launch("accumulate (grouped)");
   }
-  const Split sp = split_for(Path::kGeneric, tokens, cin);
+  const Split sp = split_for(Path::kGeneric, MODE == LHCAL_ACT_AWARE ? LHCAL_ACT_AWARE : LHCAL_FULL, tokens, cin);
   float* ws_h = ws;
   float* ws_p = ws + sp.splits * per_group;
   const dim3 grid(static_cast<unsigned>(nblk), static_cast<unsigned>(sp.splits));
@@ -520,7 +621,7 @@ size_t accumulate_workspace_bytes(lhcal_mode mode, lhcal_dtype dtype, int64_t to
                                   int32_t groups) {
   if (groups != 1 || tokens <= 0) return 0;
   const Path path = choose_path(mode, dtype, groups);
-  const Split sp = split_for(path, tokens, cin);
+  const Split sp = split_for(path, mode, tokens, cin);
   return static_cast<size_t>(sp.splits) * floats_per_split(mode, cin) * sizeof(float);
 }
 
@@ -545,7 +646,7 @@ lhcal_status launch_accumulate(lhcal_mode mode, lhcal_dtype dtype, const void* x
     return launch_mma<false>(x, xq, tokens, cin, ldx, groups, group_offsets, token_ids, acc_into, h, p, ws, stream);
   }
   if (path == Path::kDiagBf16) {
-    const Split sp = split_for(path, tokens, cin);
+    const Split sp = split_for(path, mode, tokens, cin);
     const dim3 grid(static_cast<unsigned>(ceil_div(cin, kDiagCols)), static_cast<unsigned>(sp.splits));
     accum_diag_kernel<<<grid, kDiagThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), tokens, cin, ldx,
                                                          sp.per, ws);

@@ -46,7 +46,7 @@ def test_workspace_query_is_host_only(lib):
     dense = L.lhcal_accumulate_workspace("full", L.BF16, 16384, 4096, 1)
     assert dense > 0 and dense % (256 * 4 * 256) == 0  # whole [splits, N, 16, 16] partials
     act = L.lhcal_accumulate_workspace("act", L.BF16, 16384, 4096, 1)
-    assert act == 2 * dense
+    assert act > 0 and act % (2 * 256 * 4 * 256) == 0  # H and P partials per split
     diag = L.lhcal_accumulate_workspace("diag", L.BF16, 65536, 12288, 1)
     assert diag % (12288 * 4) == 0
     assert L.lhcal_accumulate_workspace("full", L.BF16, 16384, 2560, 512) == 0
