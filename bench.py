@@ -269,7 +269,7 @@ def run_lhcal(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     dist = world > 1
-    layer = synth.make_layer(args.workload, rank)
+    layer = synth.make_layer(args.workload, rank, rows=args.rows)
     d = P.layer_to_device(layer, dev)
     mode = L.MODE_IDS[layer.mode]
     G, R, C, T = layer.groups, layer.rows, layer.cin, layer.tokens
@@ -403,6 +403,8 @@ def main():
     ap.add_argument("--impl", choices=["lhcal", "reference"], default="lhcal")
     ap.add_argument("--workload", choices=list(WORKLOAD_TEXT), default="dense")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rows", type=int, default=None,
+                    help="weight rows per group instead of the workload's (smaller captures for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -163,7 +163,7 @@ lhcal_status lhcal_scale_sweep(lhcal_mode mode, lhcal_dtype dtype, const void* w
  *     needed. Calls that can overlap on the GPU (on different streams, or from different
  *     threads without ordering) race on the scratch and give wrong results: order them.
  */
-#define LHCAL_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+#define LHCAL_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
 lhcal_status lhcal_accumulate_noalloc(lhcal_mode mode, lhcal_dtype dtype, const void* x, const void* xq,
                                       int64_t tokens, int64_t cin, int64_t ldx, int32_t groups,
                                       const int32_t* group_offsets, const int32_t* token_ids, int32_t flags,

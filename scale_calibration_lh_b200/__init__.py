@@ -128,7 +128,7 @@ def lhcal_accumulate(mode, x, h, xq=None, p=None, group_offsets=None, token_ids=
         _stream(stream)))
 
 
-NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
+NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024
 
 
 def lhcal_accumulate_noalloc(mode, x, h, xq=None, p=None, group_offsets=None, token_ids=None,

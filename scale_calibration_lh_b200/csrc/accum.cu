@@ -20,6 +20,8 @@
 //  * accum_diag_kernel: bf16 DIAG column sums of squares; each thread streams 8 columns
 //    (16-byte loads) over a token range; partials to the workspace, then reduce.
 //  * accum_generic_kernel: CUDA-core fp32 path for fp32 inputs (and grouped bf16 DIAG).
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 
 namespace lhcal {
@@ -157,7 +159,7 @@ __device__ __forceinline__ void load_ids(int32_t* slot, const int32_t* ids, int6
 // its routed rows and written to out at item * out_item_stride. A single cp.async pipeline runs
 // through the tiles of all items, so short items (about 5 tiles per expert) still stream; the
 // accumulators are written out after each item's last tile. accumulate_into: out += sums.
-template <bool ACT>
+template <bool ACT, bool CLUSTER>
 __global__ void __launch_bounds__(kMmaThreads)
 accum_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ xq,
                  int64_t tokens, int64_t cin, int64_t ldx, const int32_t* __restrict__ group_offsets,
@@ -238,7 +240,7 @@ accum_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __res
     int64_t b, e;
     range(item, b, e);
     if (e > b) ntiles += ceil_div(e - b, kTileTok);
-    else if (!accumulate_into) write_out(item, acc_h, acc_p);
+    else if (!accumulate_into && !CLUSTER) write_out(item, acc_h, acc_p);
   }
 
   // Cursors (item, position, end): ids of tiles 2S-2 ahead of consumption (grouped), data of
@@ -328,6 +330,7 @@ accum_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __res
     }
     c_pos += kTileTok;
     if (c_pos >= c_end) {  // last tile of the consumer's item: write its sums
+      if (CLUSTER) break;  // a dense item is the CTA's only one; the cluster reduces below
       write_out(c_item, acc_h, acc_p);
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
@@ -337,6 +340,51 @@ accum_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __res
     }
   }
   cp_async_wait<0>();
+
+  if (CLUSTER) {
+    // The CTAs of a cluster summed disjoint token ranges of the same slab (dense). Each stages
+    // its sums in its own shared memory; CTA rank q then adds block q of every CTA of the
+    // cluster in rank order (distributed shared memory) and writes it.
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    float* stage = reinterpret_cast<float*>(smem);  // [H: 8 blocks x 256][P: 8 blocks x 256]
+    __syncthreads();
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int idx = (i0 + 8 * half) * 16 + nt * 8 + j0;
+        stage[warp * 256 + idx] = acc_h[nt][2 * half];
+        stage[warp * 256 + idx + 1] = acc_h[nt][2 * half + 1];
+        if (ACT) {
+          stage[2048 + warp * 256 + idx] = acc_p[nt][2 * half];
+          stage[2048 + warp * 256 + idx + 1] = acc_p[nt][2 * half + 1];
+        }
+      }
+    }
+    cluster.sync();
+    const int csize = static_cast<int>(cluster.num_blocks());
+    const int rank = static_cast<int>(cluster.block_rank());
+    for (int b = rank; b < 8; b += csize) {  // blocks of the slab this CTA finishes
+      const int64_t ob = slab * 8 + b;
+      if (ob < nblk) {
+        const int t = threadIdx.x;  // 256 threads: one entry of the 16 x 16 block each
+        float vh = 0.f, vp = 0.f;
+        for (int q = 0; q < csize; ++q) {
+          const float* rs = cluster.map_shared_rank(stage, q);
+          vh += rs[b * 256 + t];
+          if (ACT) vp += rs[2048 + b * 256 + t];
+        }
+        float* oh = out_h + ob * 256 + t;
+        *oh = accumulate_into ? *oh + vh : vh;
+        if (ACT) {
+          float* op = out_p + ob * 256 + t;
+          *op = accumulate_into ? *op + vp : vp;
+        }
+      }
+    }
+    cluster.sync();  // keep this CTA's staged sums alive until every rank has read them
+  }
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -527,6 +575,29 @@ Split split_for(Path path, lhcal_mode mode, int64_t tokens, int64_t cin) {
   }
 }
 
+// Dense bf16 FULL / ACT: when the slabs alone nearly fill a wave, clusters of cs CTAs (cs <= 8)
+// split each slab's tokens and reduce in distributed shared memory (no workspace, one launch);
+// otherwise token splits write partials that reduce_partials_kernel sums.
+struct DensePlan {
+  bool cluster;
+  int cs;
+  int64_t splits;
+  int64_t per;
+};
+
+DensePlan dense_plan(lhcal_mode mode, int64_t tokens, int64_t cin) {
+  const int64_t slabs = ceil_div(cin, kSlabCols);
+  const int64_t slots = (mode == LHCAL_ACT_AWARE ? 2 : 3) * kNumSms;
+  if (tokens > 0 && 2 * slabs * 8 >= slots) {
+    int cs = 8;
+    while (cs > 1 && slabs * cs > slots) cs /= 2;
+    const int64_t per = ceil_div(ceil_div(tokens, cs), kTileTok) * kTileTok;
+    return {true, cs, cs, per};
+  }
+  const Split sp = split_for(Path::kMma, mode, tokens, cin);
+  return {false, 0, sp.splits, sp.per};
+}
+
 size_t floats_per_split(lhcal_mode mode, int64_t cin) {
   const int64_t nblk = cin / kBlock;
   if (mode == LHCAL_DIAG) return static_cast<size_t>(cin);
@@ -556,9 +627,11 @@ lhcal_status launch_mma(const void* x, const void* xq, int64_t tokens, int64_t c
   // Allow up to the per-CTA maximum (the launch size decides occupancy). Set on every call with
   // the same value: cheap, thread-safe, and correct whichever device is current.
   constexpr int kMaxDynSmem = 227 * 1024;
-  const cudaError_t attr = cudaFuncSetAttribute(accum_mma_kernel<ACT>,
-                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-  if (attr != cudaSuccess) return fail(LHCAL_ERR_CUDA, "accumulate: %s", cudaGetErrorString(attr));
+  for (const void* fn : {reinterpret_cast<const void*>(accum_mma_kernel<ACT, false>),
+                         reinterpret_cast<const void*>(accum_mma_kernel<ACT, true>)}) {
+    const cudaError_t attr = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+    if (attr != cudaSuccess) return fail(LHCAL_ERR_CUDA, "accumulate: %s", cudaGetErrorString(attr));
+  }
   const int64_t slabs = ceil_div(cin, kSlabCols);
   const int64_t nblk = cin / kBlock;
   const auto* xb = static_cast<const __nv_bfloat16*>(x);
@@ -570,22 +643,45 @@ lhcal_status launch_mma(const void* x, const void* xq, int64_t tokens, int64_t c
     const dim3 grid(static_cast<unsigned>(slabs), static_cast<unsigned>(ceil_div(groups, per)));
     const size_t smem = Cfg::kSmem + static_cast<size_t>(ceil_div((per + 1) * 4, 16) * 16);
     if (smem > static_cast<size_t>(kMaxDynSmem)) return fail(LHCAL_ERR_UNSUPPORTED, "accumulate: too many groups per CTA");
-    accum_mma_kernel<ACT><<<grid, kMmaThreads, smem, stream>>>(
+    accum_mma_kernel<ACT, false><<<grid, kMmaThreads, smem, stream>>>(
         xb, xqb, tokens, cin, ldx, offs, ids, 0, per, groups, h, p, nblk * 256, accumulate_into);
     return check_launch("accumulate (grouped, tensor cores)");
   }
-  const Split sp = split_for(Path::kMma, ACT ? LHCAL_ACT_AWARE : LHCAL_FULL, tokens, cin);
+  const DensePlan pl = dense_plan(ACT ? LHCAL_ACT_AWARE : LHCAL_FULL, tokens, cin);
+  if (pl.cluster) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(slabs), static_cast<unsigned>(pl.cs));
+    cfg.blockDim = dim3(kMmaThreads);
+    cfg.dynamicSmemBytes = Cfg::kSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 1;
+    at[0].val.clusterDim.y = static_cast<unsigned>(pl.cs);
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, accum_mma_kernel<ACT, true>, xb, xqb, tokens, cin, ldx,
+                                             static_cast<const int32_t*>(nullptr), static_cast<const int32_t*>(nullptr),
+                                             pl.per, static_cast<int64_t>(1), static_cast<int64_t>(0), h, ACT ? p : h,
+                                             static_cast<int64_t>(0), accumulate_into);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return fail(LHCAL_ERR_CUDA, "accumulate (tensor cores, clusters): %s", cudaGetErrorString(e));
+    }
+    return check_launch("accumulate (tensor cores, clusters)");
+  }
   const int64_t per_split = nblk * 256;
   float* ws_h = ws;
-  float* ws_p = ws + sp.splits * per_split;
-  const dim3 grid(static_cast<unsigned>(slabs), static_cast<unsigned>(sp.splits));
-  accum_mma_kernel<ACT><<<grid, kMmaThreads, Cfg::kSmem, stream>>>(
-      xb, xqb, tokens, cin, ldx, nullptr, nullptr, sp.per, 1, 0, ws_h, ws_p, per_split, 0);
+  float* ws_p = ws + pl.splits * per_split;
+  const dim3 grid(static_cast<unsigned>(slabs), static_cast<unsigned>(pl.splits));
+  accum_mma_kernel<ACT, false><<<grid, kMmaThreads, Cfg::kSmem, stream>>>(
+      xb, xqb, tokens, cin, ldx, nullptr, nullptr, pl.per, 1, 0, ws_h, ws_p, per_split, 0);
   lhcal_status st = check_launch("accumulate (tensor cores)");
   if (st != LHCAL_OK) return st;
-  st = launch_reduce(ws_h, sp.splits, per_split, per_split, h, accumulate_into, stream);
+  st = launch_reduce(ws_h, pl.splits, per_split, per_split, h, accumulate_into, stream);
   if (st != LHCAL_OK || !ACT) return st;
-  return launch_reduce(ws_p, sp.splits, per_split, per_split, p, accumulate_into, stream);
+  return launch_reduce(ws_p, pl.splits, per_split, per_split, p, accumulate_into, stream);
 }
 
 template <typename T, int MODE>
@@ -621,6 +717,10 @@ size_t accumulate_workspace_bytes(lhcal_mode mode, lhcal_dtype dtype, int64_t to
                                   int32_t groups) {
   if (groups != 1 || tokens <= 0) return 0;
   const Path path = choose_path(mode, dtype, groups);
+  if (path == Path::kMma) {
+    const DensePlan pl = dense_plan(mode, tokens, cin);
+    return pl.cluster ? 0 : static_cast<size_t>(pl.splits) * floats_per_split(mode, cin) * sizeof(float);
+  }
   const Split sp = split_for(path, mode, tokens, cin);
   return static_cast<size_t>(sp.splits) * floats_per_split(mode, cin) * sizeof(float);
 }

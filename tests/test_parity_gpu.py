@@ -241,6 +241,29 @@ def test_accumulate_add_equals_one_pass_and_is_deterministic():
     assert torch.equal(p2.view(torch.int32), p3.view(torch.int32))
 
 
+@pytest.mark.parametrize("name", ["dense", "act"])
+def test_accumulate_cluster_path_overwrite_and_add(name):
+    """Wide layers (32 column slabs) reduce token splits inside CTA clusters, with no workspace."""
+    layer = synth.make_layer(name, 14, tokens=3001, cin=4096, rows=2)
+    mode = layer.mode
+    assert L.lhcal_accumulate_workspace(mode, L.BF16, layer.tokens, layer.cin, 1) == 0
+    d = P.layer_to_device(layer)
+    shape = (1, 256, 16, 16)
+    h = torch.full(shape, 3.0, dtype=torch.float32, device="cuda")
+    p = torch.full(shape, 3.0, dtype=torch.float32, device="cuda") if mode == "act" else None
+    L.lhcal_accumulate(mode, d["x"], h, xq=d["xq"], p=p, flags=L.ACCUM_OVERWRITE)
+    h2 = h.clone()
+    p2 = None if p is None else p.clone()
+    L.lhcal_accumulate(mode, d["x"], h2, xq=d["xq"], p=p2, flags=L.ACCUM_ADD)
+    _sync()
+    hs, ps, _ = _oracle_hessians(layer)
+    P.check_hessians(h.cpu().numpy(), hs, f"{name} cluster H")
+    P.check_hessians(h2.cpu().numpy(), 2 * hs, f"{name} cluster H added twice")
+    if p is not None:
+        P.check_hessians(p.cpu().numpy(), ps, f"{name} cluster P")
+        P.check_hessians(p2.cpu().numpy(), 2 * ps, f"{name} cluster P added twice")
+
+
 def test_accumulate_strided_rows_and_zero_tokens():
     layer = synth.make_layer("dense", 12, tokens=333, cin=64, rows=4)
     d = P.layer_to_device(layer)

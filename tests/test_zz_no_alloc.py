@@ -52,7 +52,7 @@ def _without_workspace(mode, d, nblk):
 def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
     # Call 1 (large: many token splits) then call 2 (smaller, different mode and fewer splits):
     # the second must not see the first call's leftovers in the shared scratch.
-    cases = [("dense", "full", dict(tokens=16384, cin=4096, rows=4)),
+    cases = [("dense", "full", dict(tokens=16384, cin=2048, rows=4)),
              ("act", "act", dict(tokens=3000, cin=1024, rows=4)),
              ("wmse", "diag", dict(tokens=5000, cin=4096, rows=4))]
     for name, mode, kw in cases:
@@ -70,10 +70,11 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     lib = L.load_library()
-    cin = 20000 * 16  # one token split of 20000 block partials: 20 MB of scratch > 16 MiB
-    need = L.lhcal_accumulate_workspace("full", L.BF16, 64, cin, 1)
+    # WMSE over X [65536, 12288]: 196 token splits x 12288 partial sums = 9.6 MB of scratch.
+    tokens, cin = 65536, 12288
+    need = L.lhcal_accumulate_workspace("diag", L.BF16, tokens, cin, 1)
     assert need > L.NOALLOC_SCRATCH_BYTES
-    st = lib.lhcal_accumulate_noalloc(L.FULL, L.BF16, None, None, 64, cin, cin, 1, None, None,
+    st = lib.lhcal_accumulate_noalloc(L.DIAG, L.BF16, None, None, tokens, cin, cin, 1, None, None,
                                       L.ACCUM_OVERWRITE, None, None, ctypes.c_void_p(0))
     assert st == L.ERR_INVALID_ARG
     assert b"scratch" in lib.lhcal_last_error_string()
