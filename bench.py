@@ -44,9 +44,17 @@ WORKLOAD_TEXT = {
     "moe": "fused-MoE gate_up: 512 experts, X bf16 [16384,2560] top-10 routed, W bf16 [512,1280,2560], "
            "grouped full H, per-expert global scale",
 }
-# dram__bytes_read.sum + dram__bytes_write.sum per launch of the sweep kernel, from one ncu
-# capture of this kernel on this workload; None until captured for the current kernel.
-SWEEP_TRAFFIC_BYTES = {}
+# dram__bytes_read.sum + dram__bytes_write.sum per launch, from one ncu capture of the current
+# kernel on this workload (summaries in profiles/); workloads without a capture report null.
+SWEEP_TRAFFIC_BYTES = {
+    "dense": 34_328_064 + 137_245_952,   # sweep_tc_kernel, profiles/sweep_tc_kernel_dense.md
+    "wmse": 101_576_704 + 166_720_000,   # sweep_diag_kernel, profiles/sweep_diag_kernel_wmse.md
+}
+ACCUM_TRAFFIC_BYTES = {
+    "dense": 134_263_808 + 3_650_816,    # accum_mma_kernel (clusters), profiles/accum_mma_kernel_dense.md
+    "act": 536_914_688 + 5_005_312,      # accum_mma_kernel (clusters), profiles/accum_mma_kernel_act.md
+    "wmse": 1_610_820_000 + 8_041_472,   # accum_diag_kernel (+ the partial reduction, not captured)
+}
 
 
 def load_peaks():
@@ -370,7 +378,7 @@ def run_lhcal(args, rank, world, local_rank):
                    "rows": R, "groups": G, "mode": layer.mode, "input_dtype": layer.dtype,
                    "l2": "no flush: inputs larger than L2 (126 MB)",
                    "parallelism": f"{world} independent layers, one per GPU (no collective)"},
-        "roofline": {"kernel": "sweep_kernel", "bound": "alu", "achieved": achieved_ops / 1e12,
+        "roofline": {"kernel": "sweep_diag_kernel" if layer.mode == "diag" else "sweep_tc_kernel", "bound": "alu", "achieved": achieved_ops / 1e12,
                      "peak": peak_ops / 1e12, "unit": "Tops/s", "frac": achieved_ops / peak_ops,
                      "traffic": traffic,
                      "note": f"FP32 lane-ops of the direct method ({ops // 126}/candidate) over the measured sweep "
@@ -378,7 +386,7 @@ def run_lhcal(args, rank, world, local_rank):
                              f"(max clock, {peak_src})"},
         "roofline_accum": {"kernel": "accumulate (incl. partial reduction)", "bound": "hbm",
                            "achieved": achieved_gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": achieved_gbs / hbm_gbs,
-                           "traffic": None, "bytes_per_step": acc_bytes,
+                           "traffic": ACCUM_TRAFFIC_BYTES.get(args.workload), "bytes_per_step": acc_bytes,
                            "note": f"algorithmic bytes over the measured accumulation time; peak {peak_src}"},
         "stages_ms": {"accumulate": t_acc, "count_finalize": t_fin, "global_scale": t_g, "sweep": t_sweep},
         "e2e": {"value": weak_scaling_value(units, world, ms_e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
