@@ -265,3 +265,34 @@ def calibrate_host(mode, x, w, buffers: Buffers, staging: dict, hxq=None, group_
     if out.loss is not None:
         out.loss.copy_(buffers.loss, non_blocking=True)
     return out
+
+
+class CalibrationGraph:
+    """The whole hot path on fixed device buffers, captured once as a CUDA graph.
+
+    Construction runs the path once eagerly (so that any first-call set-up happens outside the
+    capture), then captures accumulate, count, finalize, global scale and sweep on a side
+    stream. ``replay()`` re-runs the captured launches on the current contents of the tensors
+    given at construction: copy new activations / weights into them between replays. The
+    results land in ``self.buffers``.
+    """
+
+    def __init__(self, mode, x, w, xq=None, group_offsets=None, token_ids=None, buffers: Buffers | None = None):
+        import torch
+
+        m = _mode_id(mode)
+        groups, rows, cin = (int(v) for v in w.shape)
+        self.buffers = buffers or Buffers(m, int(x.shape[0]), cin, rows, groups, _dtype_id(x), x.device)
+        args = dict(xq=xq, group_offsets=group_offsets, token_ids=token_ids, buffers=self.buffers)
+        calibrate(m, x, w, **args)
+        torch.cuda.synchronize(x.device)
+        self.graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(device=x.device)
+        side.wait_stream(torch.cuda.current_stream(x.device))
+        with torch.cuda.graph(self.graph, stream=side, capture_error_mode="thread_local"):
+            calibrate(m, x, w, **args)
+        torch.cuda.current_stream(x.device).wait_stream(side)
+
+    def replay(self):
+        self.graph.replay()
+        return self.buffers

@@ -328,3 +328,80 @@ def _run_and_check_wmse_full(layer, units):
     ref = O.sweep("diag", w32, h, None, g, units)
     gc, gw, gl = P.gather_gpu_units(b.codes, b.wq, b.loss, units)
     P.check_sweep(gc, gw, gl, ref, "wmse full")
+
+
+# ----------------------------------------------------------------------------- more edge cases
+
+def test_grouped_add_mode_over_two_batches():
+    """Two routed batches added into the same per-expert sums equal one pass over both."""
+    layer = synth.make_layer("moe", 15, tokens=200, cin=96, rows=8, groups=16, top_k=3)
+    d = P.layer_to_device(layer)
+    x = d["x"]
+    off = layer.group_offsets
+    ids = layer.token_ids
+    # Batch 1: tokens < 100, batch 2: tokens >= 100 (ids renumbered into each batch's rows).
+    batches = []
+    for lo, hi in ((0, 100), (100, 200)):
+        o, t = [0], []
+        for e in range(16):
+            sel = [int(v) - lo for v in ids[off[e]:off[e + 1]] if lo <= v < hi]
+            t += sel
+            o.append(len(t))
+        batches.append((lo, hi, np.array(o, np.int32), np.array(t, np.int32)))
+    h = torch.full((16, 6, 16, 16), 9.0, dtype=torch.float32, device="cuda")
+    counts = torch.empty(16, dtype=torch.int64, device="cuda")
+    for j, (lo, hi, o, t) in enumerate(batches):
+        flags = L.ACCUM_OVERWRITE if j == 0 else L.ACCUM_ADD
+        do, dt = P.to_device(o, "i32"), P.to_device(t, "i32")
+        L.lhcal_accumulate("full", x[lo:hi], h, group_offsets=do, token_ids=dt, flags=flags)
+        L.lhcal_count_tokens(counts, group_offsets=do, flags=flags)
+    L.lhcal_finalize("full", counts, h)
+    _sync()
+    hs, _, c = _oracle_hessians(layer)
+    hf, _ = O.finalize("full", hs, None, c)
+    np.testing.assert_array_equal(counts.cpu().numpy(), c)
+    P.check_hessians(h.cpu().numpy(), hf, "two-batch grouped H")
+
+
+@pytest.mark.parametrize("mode", ["full", "act", "diag"])
+def test_sweep_optional_outputs_and_determinism(mode):
+    name = {"full": "dense", "act": "act", "diag": "wmse"}[mode]
+    layer = synth.make_layer(name, 16, tokens=300, cin=128, rows=200)
+    d = P.layer_to_device(layer)
+    b = L.calibrate(mode, d["x"], d["w"], xq=d["xq"])
+    codes1 = b.codes.clone()
+    wq1 = b.wq.clone()
+    loss1 = b.loss.clone()
+    codes2 = torch.empty_like(codes1)
+    L.lhcal_scale_sweep(mode, d["w"], b.h, b.g, codes2, wq=None, loss=None, p=b.p)
+    codes3 = torch.empty_like(codes1)
+    wq3 = torch.empty_like(wq1)
+    loss3 = torch.empty_like(loss1)
+    L.lhcal_scale_sweep(mode, d["w"], b.h, b.g, codes3, wq=wq3, loss=loss3, p=b.p)
+    _sync()
+    assert torch.equal(codes1, codes2) and torch.equal(codes1, codes3)
+    assert torch.equal(wq1.view(torch.int32), wq3.view(torch.int32))
+    assert torch.equal(loss1.view(torch.int32), loss3.view(torch.int32))
+
+
+def test_diag_sweep_multiple_groups():
+    layer = synth.make_layer("moe", 17, tokens=120, cin=64, rows=70, groups=6, top_k=2)
+    layer.mode = "diag"
+    _run_and_check(layer)
+
+
+def test_graph_replay_matches_eager_calls():
+    layer_a = synth.make_layer("dense", 18, tokens=700, cin=512, rows=96)
+    layer_b = synth.make_layer("dense", 19, tokens=700, cin=512, rows=96)
+    da, db = P.layer_to_device(layer_a), P.layer_to_device(layer_b)
+    x, w = da["x"].clone(), da["w"].clone()
+    graph = L.CalibrationGraph("full", x, w)
+    for d in (db, da):
+        x.copy_(d["x"])
+        w.copy_(d["w"])
+        out = graph.replay()
+        eager = L.calibrate("full", d["x"], d["w"])
+        _sync()
+        assert torch.equal(out.codes, eager.codes)
+        assert torch.equal(out.wq.view(torch.int32), eager.wq.view(torch.int32))
+        assert torch.equal(out.h.view(torch.int32), eager.h.view(torch.int32))
