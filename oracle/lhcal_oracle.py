@@ -111,6 +111,64 @@ def fake_quant(w: np.ndarray, s) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------------------
+# Activation fake quant (the input quantizer that produces X_q)
+# ---------------------------------------------------------------------------------------
+
+def e4m3_round(r) -> np.ndarray:
+    """E4M3 code (0..126) of the value nearest to each real r >= 0: ties to the even code.
+
+    Code 0 is zero; 1..126 are the positive finite values of ``e4m3_value``, so the even
+    code is the one with mantissa bit 0. Anything above 448 saturates to 448 (code 126).
+    The decision compares r with the exact midpoint of the two bracketing values.
+    """
+    r = np.asarray(r, dtype=np.float64)
+    vals = np.concatenate([[0.0], e4m3_value(candidate_codes())])
+    hi = np.clip(np.searchsorted(vals, r, side="left"), 1, N_CANDIDATES)  # vals[hi-1] < r <= vals[hi]
+    lo = hi - 1
+    mid = (vals[lo] + vals[hi]) / 2.0
+    up = (r > mid) | ((r == mid) & (hi % 2 == 0))
+    return np.where(r >= FP8_MAX, N_CANDIDATES, np.where(up, hi, lo)).astype(np.int64)
+
+
+def f32_to_bf16_values(v: np.ndarray) -> np.ndarray:
+    """Round fp32 values to bf16 (nearest, ties to even); returns the bf16 values as fp32."""
+    import torch
+
+    t = torch.from_numpy(np.ascontiguousarray(v, dtype=np.float32))
+    return t.to(torch.bfloat16).to(torch.float32).numpy()
+
+
+def act_fake_quant(x: np.ndarray, gx) -> np.ndarray:
+    """NVFP4 fake quant of activations X [T, C] with the per-tensor global scale gx (fp32).
+
+    The input quantizer whose output the activation-aware capture records ("Add
+    activation-aware local Hessian scale calibration", PR #1976, re-review): 16-wide
+    blocks along C, an E4M3 block scale and a per-tensor global scale (the NVFP4 layout of
+    "Add composable scale calibration to GPTQ", PR #2004). Reading, per (token, block):
+    code c = E4M3(amax_blk / (6 gx)) on the exact quotient (nearest, ties to even,
+    saturating at 448); s = fp32(v_c gx); each value becomes E2M1(|x| / s) on the exact
+    quotient, then bf16(fp32(q s)) with the sign of x. gx == 0 or c == 0 gives a zero
+    block. Returns fp32 values that are exactly bf16.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    t, c = x.shape
+    gx64 = np.float64(np.float32(gx))
+    xb = x.reshape(t, c // BLOCK, BLOCK)
+    amax = np.abs(xb).max(axis=-1)
+    if gx64 > 0:
+        code = e4m3_round(amax / (FP4_MAX * gx64))
+    else:
+        code = np.zeros(amax.shape, dtype=np.int64)
+    v = np.where(code > 0, e4m3_value(np.maximum(code, 1)), 0.0)
+    s = (v * gx64).astype(np.float32).astype(np.float64)[..., None]  # exact product, one rounding
+    with np.errstate(divide="ignore", invalid="ignore"):
+        u = np.where(s > 0, np.abs(xb) / np.where(s > 0, s, 1.0), 0.0)
+    q = e2m1_round(u)
+    mag = f32_to_bf16_values((q * s).astype(np.float32))
+    return np.copysign(mag, xb).reshape(t, c).astype(np.float32)
+
+
+# ---------------------------------------------------------------------------------------
 # Hessian accumulation (raw sums) and finalisation
 # ---------------------------------------------------------------------------------------
 
@@ -141,14 +199,19 @@ def importance_sum(x: np.ndarray) -> np.ndarray:
     return np.square(x).sum(axis=0).reshape(c // BLOCK, BLOCK)
 
 
-def accumulate(mode: str, x, xq=None, group_offsets=None, token_ids=None):
+def accumulate(mode: str, x, xq=None, group_offsets=None, token_ids=None, act_gx=None):
     """Raw per-group sums and token counts.
 
     Returns (h [G, N, 16, 16] or [G, N, 16] for diag, p or None, counts [G]).
     Grouped: group e sums over rows token_ids[offsets[e]:offsets[e+1]] of x
     (the tokens routed to expert e, PR #2864 / #2840).
+    ACT without xq: X_q = act_fake_quant(x, act_gx), the input quantizer's output.
     """
     x = np.asarray(x)
+    if mode == "act" and xq is None:
+        if act_gx is None:
+            raise ValueError("act needs xq or the activation global scale act_gx")
+        xq = act_fake_quant(x, act_gx)
     if group_offsets is None:
         sets = [np.arange(x.shape[0])]
     else:
@@ -321,9 +384,9 @@ def sweep(mode: str, w, h, p, g, units=None, chunk: int = 512):
     return {k: np.concatenate([o[k] for o in outs]) for k in outs[0]} if outs else {}
 
 
-def calibrate(mode: str, x, w, xq=None, group_offsets=None, token_ids=None, units=None):
+def calibrate(mode: str, x, w, xq=None, group_offsets=None, token_ids=None, units=None, act_gx=None):
     """The whole hot path: accumulate, finalize, global scale per group, sweep."""
-    hsum, psum, counts = accumulate(mode, x, xq, group_offsets, token_ids)
+    hsum, psum, counts = accumulate(mode, x, xq, group_offsets, token_ids, act_gx)
     h, p = finalize(mode, hsum, psum, counts)
     w = np.asarray(w, dtype=np.float32)
     g = np.array([global_scale(w[e]) for e in range(w.shape[0])], dtype=np.float32)

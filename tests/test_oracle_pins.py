@@ -94,6 +94,108 @@ def test_global_scale_is_448_normalized():
     assert O.global_scale(np.zeros((2, 3), np.float32)) == 0.0
 
 
+# --------------------------------------------------------------------------- activation fake quant
+
+E4M3_ALL = [Fraction(0)] + [Fraction(float(v)) for v in O.e4m3_value(O.candidate_codes())]
+
+
+def _round_binary(y: Fraction, bits: int, emin: int) -> Fraction:
+    """Round y >= 0 to `bits` significant bits (exponents below emin: fixed ulp), half to even."""
+    if y == 0:
+        return y
+    e = y.numerator.bit_length() - y.denominator.bit_length()
+    if Fraction(2) ** e > y:
+        e -= 1
+    ulp = Fraction(2) ** (max(e, emin) - (bits - 1))
+    return round(y / ulp) * ulp  # Fraction.__round__ rounds half to even
+
+
+def _e4m3_code_brute(r: Fraction) -> int:
+    """Nearest of all 127 non-negative finite E4M3 values, ties to the even code; > 448 -> 448."""
+    if r > 448:
+        return 126
+    return min(range(127), key=lambda k: (abs(E4M3_ALL[k] - r), k % 2))
+
+
+def _act_quant_brute(block, gx) -> list:
+    """One 16-value block by exact rationals and exhaustive nearest-value searches."""
+    g = Fraction(float(np.float32(gx)))
+    amax = max(abs(Fraction(float(v))) for v in block)
+    code = _e4m3_code_brute(amax / (6 * g)) if g > 0 else 0
+    s = _round_binary(E4M3_ALL[code] * g, 24, -126)
+    out = []
+    for v in block:
+        a = abs(Fraction(float(v)))
+        i = min(range(8), key=lambda j: (abs(E2M1[j] * s - a), j % 2))
+        mag = _round_binary(_round_binary(E2M1[i] * s, 24, -126), 8, -126)
+        out.append(float(np.copysign(float(mag), float(v))))
+    return out
+
+
+def _bf16_values(a: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.asarray(a, np.float32)).to(torch.bfloat16).float().numpy()
+
+
+def test_e4m3_round_brute_force_and_library():
+    rng = np.random.default_rng(11)
+    vals = np.array([float(v) for v in E4M3_ALL])
+    mids = (vals[:-1] + vals[1:]) / 2
+    r = np.concatenate([rng.uniform(0, 460, 3000), np.exp2(rng.uniform(-14, 9, 3000)), vals, mids,
+                        np.nextafter(mids, 0), np.nextafter(mids, 1e9), [0.0, 2.0 ** -10, 448.0, 463.9, 500.0, 1e30]])
+    got = O.e4m3_round(r)
+    want = np.array([_e4m3_code_brute(Fraction(float(v))) for v in r])
+    np.testing.assert_array_equal(got, want)
+    # ml_dtypes' float8_e4m3fn conversion (nearest, ties to even) agrees below its NaN range.
+    ok = r < 464
+    lib = r[ok].astype(np.float32).astype(ml_dtypes.float8_e4m3fn).view(np.uint8)
+    exact32 = r[ok] == r[ok].astype(np.float32)  # compare where the fp32 cast loses nothing
+    np.testing.assert_array_equal(got[ok][exact32], lib[exact32])
+
+
+@pytest.mark.parametrize("gx_factor", [1.0, 1e-3, 1e3, 0.0])
+def test_act_fake_quant_brute_force(gx_factor):
+    rng = np.random.default_rng(12)
+    sig = np.exp(rng.normal(0, 1.5, 64))
+    sig[[3, 40]] *= 20
+    x = _bf16_values(rng.normal(size=(5, 64)) * sig)
+    x[1, 16:32] = 0.0  # an all-zero block
+    x[2, 0:16] = -0.0
+    x[3, 32:48] *= 1e-30  # a tiny block: small and subnormal scale codes
+    gx = np.float32(O.global_scale(x) * gx_factor)
+    got = O.act_fake_quant(x, gx)
+    want = np.array([_act_quant_brute(x[t, 16 * n:16 * n + 16], gx) for t in range(5) for n in range(4)],
+                    np.float32).reshape(5, 4, 16).reshape(5, 64)
+    np.testing.assert_array_equal(got.view(np.int32), want.view(np.int32))
+    assert np.all(got == _bf16_values(got))  # bf16-exact values
+
+
+def test_act_fake_quant_hand_worked_ties():
+    # gx = 1: amax 6.375 -> 6.375 / 6 = 1.0625, midway between E4M3 1.0 (0x38) and 1.125 (0x39):
+    # the even code wins, s = 1.0. amax 7.125 -> 1.1875, midway between 1.125 (0x39) and
+    # 1.25 (0x3A): s = 1.25. With s = 1.25 every E2M1 midpoint m * 1.25 is bf16-exact.
+    blk_a = np.zeros(16, np.float32)
+    blk_a[0], blk_a[1], blk_a[2] = 6.375, -0.75, 0.25
+    blk_b = np.array([7.125, 0.3125, 0.9375, 1.5625, 2.1875, 3.125, 4.375, 6.25,
+                      -0.3125, -0.9375, -1.5625, -2.1875, -3.125, -4.375, -6.25, 0.0], np.float32)
+    x = np.stack([np.concatenate([blk_a, blk_b])])
+    got = O.act_fake_quant(x, np.float32(1.0))[0]
+    # s = 1.0: 6.375 -> 6 (clamped), 0.75 -> tie 0.5 | 1 -> 1, 0.25 -> tie 0 | 0.5 -> 0.
+    assert got[:3].tolist() == [6.0, -1.0, 0.0]
+    # s = 1.25: ties go to the even E2M1 code: .25->0, .75->1, 1.25->1, 1.75->2, 2.5->2, 3.5->4, 5->4.
+    want_b = [7.5, 0.0, 1.25, 1.25, 2.5, 2.5, 5.0, 5.0, -0.0, -1.25, -1.25, -2.5, -2.5, -5.0, -5.0, 0.0]
+    np.testing.assert_array_equal(got[16:].view(np.int32), np.array(want_b, np.float32).view(np.int32))
+
+
+def test_act_fake_quant_saturates_and_zero_global_scale():
+    x = np.full((1, 16), 3.0, np.float32)
+    # gx so small that amax / (6 gx) is far above 448: the code saturates at 448 and every
+    # value lands on the top of the grid at s = fp32(448 gx): 6 * s.
+    gx = np.float32(1e-6)
+    s = np.float32(448.0 * np.float64(gx))
+    np.testing.assert_array_equal(O.act_fake_quant(x, gx), _bf16_values(np.full((1, 16), np.float32(6 * np.float64(s)))))
+    assert np.all(O.act_fake_quant(x, np.float32(0.0)) == 0.0)
+
+
 # --------------------------------------------------------------------------- Hessians
 
 def _tiny_x(t=7, c=32, seed=3):
