@@ -33,6 +33,8 @@ g = 0 makes every q zero.
 """
 from __future__ import annotations
 
+import os
+
 import numpy as np
 
 BLOCK = 16
@@ -138,7 +140,7 @@ def f32_to_bf16_values(v: np.ndarray) -> np.ndarray:
     return t.to(torch.bfloat16).to(torch.float32).numpy()
 
 
-def act_fake_quant(x: np.ndarray, gx) -> np.ndarray:
+def act_fake_quant(x: np.ndarray, gx, rows_per_chunk: int = 1024) -> np.ndarray:
     """NVFP4 fake quant of activations X [T, C] with the per-tensor global scale gx (fp32).
 
     The input quantizer whose output the activation-aware capture records ("Add
@@ -148,24 +150,39 @@ def act_fake_quant(x: np.ndarray, gx) -> np.ndarray:
     code c = E4M3(amax_blk / (6 gx)) on the exact quotient (nearest, ties to even,
     saturating at 448); s = fp32(v_c gx); each value becomes E2M1(|x| / s) on the exact
     quotient, then bf16(fp32(q s)) with the sign of x. gx == 0 or c == 0 gives a zero
-    block. Returns fp32 values that are exactly bf16.
+    block. Returns fp32 values that are exactly bf16. Rows are independent; they are
+    processed rows_per_chunk at a time (on a thread pool) only to bound memory and time.
     """
-    x = np.asarray(x, dtype=np.float64)
+    x = np.asarray(x)
     t, c = x.shape
     gx64 = np.float64(np.float32(gx))
-    xb = x.reshape(t, c // BLOCK, BLOCK)
-    amax = np.abs(xb).max(axis=-1)
-    if gx64 > 0:
-        code = e4m3_round(amax / (FP4_MAX * gx64))
+    out = np.empty((t, c), dtype=np.float32)
+
+    def rows(lo):
+        xb = x[lo:lo + rows_per_chunk].astype(np.float64).reshape(-1, c // BLOCK, BLOCK)
+        amax = np.abs(xb).max(axis=-1)
+        if gx64 > 0:
+            code = e4m3_round(amax / (FP4_MAX * gx64))
+        else:
+            code = np.zeros(amax.shape, dtype=np.int64)
+        v = np.where(code > 0, e4m3_value(np.maximum(code, 1)), 0.0)
+        s = (v * gx64).astype(np.float32).astype(np.float64)[..., None]  # exact product, one rounding
+        with np.errstate(divide="ignore", invalid="ignore"):
+            u = np.where(s > 0, np.abs(xb) / np.where(s > 0, s, 1.0), 0.0)
+        q = e2m1_round(u)
+        mag = f32_to_bf16_values((q * s).astype(np.float32))
+        out[lo:lo + rows_per_chunk] = np.copysign(mag, xb).reshape(-1, c)
+
+    starts = range(0, t, rows_per_chunk)
+    if t > rows_per_chunk:
+        from concurrent.futures import ThreadPoolExecutor
+
+        with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+            list(ex.map(rows, starts))
     else:
-        code = np.zeros(amax.shape, dtype=np.int64)
-    v = np.where(code > 0, e4m3_value(np.maximum(code, 1)), 0.0)
-    s = (v * gx64).astype(np.float32).astype(np.float64)[..., None]  # exact product, one rounding
-    with np.errstate(divide="ignore", invalid="ignore"):
-        u = np.where(s > 0, np.abs(xb) / np.where(s > 0, s, 1.0), 0.0)
-    q = e2m1_round(u)
-    mag = f32_to_bf16_values((q * s).astype(np.float32))
-    return np.copysign(mag, xb).reshape(t, c).astype(np.float32)
+        for lo in starts:
+            rows(lo)
+    return out
 
 
 # ---------------------------------------------------------------------------------------
