@@ -39,7 +39,8 @@ FALLBACK_SM_MHZ = 1965.0
 WORKLOAD_TEXT = {
     "dense": "dense projection local_hessian: X bf16 [16384,4096] (lognormal column std, 1% outliers x20), "
              "W bf16 [4096,4096], full 16x16 H per block, 126-candidate FP8 sweep",
-    "act": "activation-aware gate_up: X, X_q bf16 [32768,4096], W bf16 [12288,4096], H and P, cross term",
+    "act": "activation-aware gate_up: X bf16 [32768,4096] through the fused NVFP4 input quantizer (X_q derived "
+           "in the kernel; its global scale calibrated beforehand), W bf16 [12288,4096], H and P, cross term",
     "wmse": "WMSE down_proj: X bf16 [65536,12288], W bf16 [4096,12288], diagonal Imp [768,16]",
     "moe": "fused-MoE gate_up: 512 experts, X bf16 [16384,2560] top-10 routed, W bf16 [512,1280,2560], "
            "grouped full H, per-expert global scale",
@@ -52,7 +53,6 @@ SWEEP_TRAFFIC_BYTES = {
 }
 ACCUM_TRAFFIC_BYTES = {
     "dense": 134_263_808 + 3_650_816,    # accum_mma_kernel (clusters), profiles/accum_mma_kernel_dense.md
-    "act": 536_914_688 + 5_005_312,      # accum_mma_kernel (clusters), profiles/accum_mma_kernel_act.md
     "wmse": 1_610_820_000 + 8_041_472,   # accum_diag_kernel (+ the partial reduction, not captured)
 }
 
@@ -161,8 +161,8 @@ def algorithmic(layer):
     ops = 126 * OPS_PER_CANDIDATE[layer.mode]
     hsz = G * nblk * (16 if layer.mode == "diag" else 256) * 4
     xb = T * C * 2
-    if layer.mode == "act":
-        acc_bytes = 2 * xb + 2 * hsz
+    if layer.mode == "act":  # X read once: X_q is derived from it inside the kernel
+        acc_bytes = xb + 2 * hsz
     elif layer.token_ids is not None:
         acc_bytes = xb + hsz + layer.token_ids.nbytes + layer.group_offsets.nbytes
     else:
@@ -189,6 +189,8 @@ def oracle_sample_step(layer, frac_tokens: float, n_units: int, seed: int = 0):
 
     T = layer.tokens
     ts = max(1, int(T * frac_tokens))
+    if layer.mode == "act" and "act_gx_oracle" not in layer.meta:
+        layer.meta["act_gx_oracle"] = O.global_scale(synth.bf16_bits_to_f32(layer.x))
     t0 = time.perf_counter()
     if layer.token_ids is not None:
         # Grouped: the first groups' routed rows, about ts rows in total.
@@ -200,8 +202,9 @@ def oracle_sample_step(layer, frac_tokens: float, n_units: int, seed: int = 0):
         frac = gcount / layer.groups
     else:
         xs = synth.bf16_bits_to_f32(layer.x[:ts])
-        xqs = synth.bf16_bits_to_f32(layer.xq[:ts]) if layer.xq is not None else None
-        O.accumulate(layer.mode, xs, xqs)
+        # Activation-aware: the oracle derives X_q with the input quantizer's global scale,
+        # computed once over the whole X before the timing starts.
+        O.accumulate(layer.mode, xs, None, act_gx=layer.meta.get("act_gx_oracle"))
         frac = ts / T
     t_acc = (time.perf_counter() - t0) / frac
     rng = np.random.default_rng(seed)
@@ -283,9 +286,16 @@ def run_lhcal(args, rank, world, local_rank):
     G, R, C, T = layer.groups, layer.rows, layer.cin, layer.tokens
     buf = L.Buffers(mode, T, C, R, G, L.BF16, dev)
     stream = torch.cuda.current_stream()
+    act_gx = None
+    if layer.mode == "act":
+        # The input quantizer's global scale, fp32(amax|X| / 2688): calibrated once before the
+        # capture (by max calibration in the pages' flow), so it is set up outside the timing.
+        act_gx = torch.empty(1, dtype=torch.float32, device=dev)
+        L.lhcal_global_scale(d["x"].view(1, T, C), act_gx)
 
     def step():
-        L.calibrate(mode, d["x"], d["w"], xq=d["xq"], group_offsets=d["offs"], token_ids=d["ids"], buffers=buf)
+        L.calibrate(mode, d["x"], d["w"], xq=d["xq"], group_offsets=d["offs"], token_ids=d["ids"], buffers=buf,
+                    act_gx=act_gx)
 
     def barrier():
         if dist:
@@ -308,8 +318,12 @@ def run_lhcal(args, rank, world, local_rank):
     for k in range(K):
         e = ev[k]
         e[0].record(stream)
-        L.lhcal_accumulate(mode, d["x"], buf.h, xq=d["xq"], p=buf.p, group_offsets=d["offs"], token_ids=d["ids"],
-                           flags=L.ACCUM_OVERWRITE, workspace=buf.workspace)
+        if act_gx is not None:
+            L.lhcal_accumulate_act_quant(d["x"], buf.h, buf.p, act_gx, flags=L.ACCUM_OVERWRITE,
+                                         workspace=buf.workspace)
+        else:
+            L.lhcal_accumulate(mode, d["x"], buf.h, xq=d["xq"], p=buf.p, group_offsets=d["offs"],
+                               token_ids=d["ids"], flags=L.ACCUM_OVERWRITE, workspace=buf.workspace)
         e[1].record(stream)
         L.lhcal_count_tokens(buf.counts, tokens=T, group_offsets=d["offs"], flags=L.ACCUM_OVERWRITE)
         L.lhcal_finalize(mode, buf.counts, buf.h, p=buf.p)
@@ -346,7 +360,8 @@ def run_lhcal(args, rank, world, local_rank):
     K2 = max(3, min(K, 10))
 
     def e2e_step():
-        L.calibrate_host(mode, hx, hw, buf, d, hxq=hxq, group_offsets=hoffs, token_ids=hids, out=out_host)
+        L.calibrate_host(mode, hx, hw, buf, d, hxq=hxq, group_offsets=hoffs, token_ids=hids, out=out_host,
+                         act_gx=act_gx)
 
     e2e_step()  # warm
     torch.cuda.synchronize()
@@ -384,7 +399,8 @@ def run_lhcal(args, rank, world, local_rank):
                      "note": f"FP32 lane-ops of the direct method ({ops // 126}/candidate) over the measured sweep "
                              f"time; peak = {N_SMS} SMs x {FP32_LANES_PER_SM} FP32 lanes x {sm_mhz:.0f} MHz "
                              f"(max clock, {peak_src})"},
-        "roofline_accum": {"kernel": "accumulate (incl. partial reduction)", "bound": "hbm",
+        "roofline_accum": {"kernel": "accumulate (incl. partial reduction)" + (
+                               ", input quantizer fused" if act_gx is not None else ""), "bound": "hbm",
                            "achieved": achieved_gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": achieved_gbs / hbm_gbs,
                            "traffic": ACCUM_TRAFFIC_BYTES.get(args.workload), "bytes_per_step": acc_bytes,
                            "note": f"algorithmic bytes over the measured accumulation time; peak {peak_src}"},

@@ -97,6 +97,52 @@ lhcal_status lhcal_accumulate(lhcal_mode mode, lhcal_dtype dtype, const void* x,
                               float* h, float* p, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * NVFP4 fake quant of activations, the input quantizer whose output X_q the activation-aware
+ * capture records (PR #1976, re-review: the input-quantizer hook captures X_q). Per token and
+ * 16-wide block along cin:
+ *   c = E4M3 code nearest to amax_blk / (6 * gx) (exact quotient, ties to the even code,
+ *       saturating at 448; c = 0 gives a zero block);
+ *   s = fp32(v_c * gx);
+ *   xq = bf16(fp32(q * s)) with the sign of x, q = E2M1 of the exact |x| / s (nearest, ties
+ *        to even, clamped at 6).
+ *   dtype : LHCAL_BF16 only (LHCAL_ERR_UNSUPPORTED otherwise).
+ *   x     : [tokens, cin] bf16, row stride ldx; xq: out [tokens, cin] bf16, row stride ldxq
+ *           (both strides >= cin with stride * 2 a multiple of 16 bytes, bases 16-byte aligned;
+ *           x and xq must not overlap).
+ *   act_gx: device fp32 scalar, the per-tensor global scale gx (for example lhcal_global_scale
+ *           of X viewed as [1, tokens, cin]: amax / (6 * 448)); finite and >= 0.
+ * Bit-exact: every rounding decision is taken on the exact quotient.
+ */
+lhcal_status lhcal_act_fake_quant(lhcal_dtype dtype, const void* x, int64_t tokens, int64_t cin, int64_t ldx,
+                                  const float* act_gx, void* xq, int64_t ldxq, void* stream);
+
+/*
+ * Bytes of workspace lhcal_accumulate_act_quant needs for these sizes (0 is possible).
+ * Host-only computation; needs no GPU. dtype must be LHCAL_BF16.
+ */
+lhcal_status lhcal_accumulate_act_quant_workspace(lhcal_dtype dtype, int64_t tokens, int64_t cin, int32_t groups,
+                                                  size_t* bytes);
+
+/*
+ * Activation-aware accumulation (lhcal_accumulate with LHCAL_ACT_AWARE) with the input
+ * quantizer fused: X_q is not read from memory but derived from x inside the kernel exactly as
+ * lhcal_act_fake_quant computes it, so the activations are read once. The sums are those of
+ * lhcal_act_fake_quant followed by lhcal_accumulate(LHCAL_ACT_AWARE, ...) with that X_q, up to
+ * the fp32 summation order (the two may split the tokens differently; grouped sums and equal
+ * splits give identical bits).
+ *   dtype : LHCAL_BF16 only (LHCAL_ERR_UNSUPPORTED otherwise).
+ *   act_gx: device fp32 scalar, the input quantizer's global scale (see lhcal_act_fake_quant);
+ *           it is an input because the quantizer's amax is calibrated before the capture.
+ *   other arguments as for lhcal_accumulate with mode LHCAL_ACT_AWARE; the workspace size is
+ *   lhcal_accumulate_act_quant_workspace(LHCAL_BF16, tokens, cin, groups).
+ */
+lhcal_status lhcal_accumulate_act_quant(lhcal_dtype dtype, const void* x, int64_t tokens, int64_t cin,
+                                        int64_t ldx, int32_t groups, const int32_t* group_offsets,
+                                        const int32_t* token_ids, const float* act_gx, int32_t flags,
+                                        float* h, float* p, void* workspace, size_t workspace_bytes,
+                                        void* stream);
+
+/*
  * Token counts B per group: counts[e] (+)= offsets[e+1] - offsets[e], or counts[0] (+)= tokens
  * when group_offsets is NULL (groups must then be 1). counts: device int64 [groups].
  * flags as for lhcal_accumulate.

@@ -47,6 +47,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lhcal_accumulate_workspace": [i32, i32, i64, i64, i32, ctypes.POINTER(sz)],
         "lhcal_accumulate": [i32, i32, vp, vp, i64, i64, i64, i32, vp, vp, i32, vp, vp, vp, sz, vp],
         "lhcal_accumulate_noalloc": [i32, i32, vp, vp, i64, i64, i64, i32, vp, vp, i32, vp, vp, vp],
+        "lhcal_accumulate_act_quant_workspace": [i32, i64, i64, i32, ctypes.POINTER(sz)],
+        "lhcal_accumulate_act_quant": [i32, vp, i64, i64, i64, i32, vp, vp, vp, i32, vp, vp, vp, sz, vp],
+        "lhcal_act_fake_quant": [i32, vp, i64, i64, i64, vp, vp, i64, vp],
         "lhcal_count_tokens": [i32, i64, vp, i32, vp, vp],
         "lhcal_finalize": [i32, i32, i64, vp, vp, vp, vp],
         "lhcal_global_scale": [i32, vp, i32, i64, i64, vp, vp],
@@ -84,6 +87,11 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+def _ld(t, cin: int) -> int:
+    """Row stride in elements; an empty tensor's stride carries no meaning, so cin is passed."""
+    return int(t.stride(0)) if t.shape[0] > 0 else cin
+
+
 def _dtype_id(t) -> int:
     import torch
 
@@ -118,14 +126,43 @@ def lhcal_accumulate(mode, x, h, xq=None, p=None, group_offsets=None, token_ids=
     """x, xq: [tokens, cin] (row stride x.stride(0)); h, p, workspace: fp32 device tensors."""
     m = _mode_id(mode)
     tokens, cin = int(x.shape[0]), int(x.shape[1])
-    if x.stride(1) != 1:
+    if x.numel() and x.stride(1) != 1:
         raise ValueError("x must have unit stride along cin")
     groups = 1 if group_offsets is None else int(group_offsets.numel()) - 1
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(load_library().lhcal_accumulate(
-        m, _dtype_id(x), _ptr(x), _ptr(xq), tokens, cin, int(x.stride(0)), groups,
+        m, _dtype_id(x), _ptr(x), _ptr(xq), tokens, cin, _ld(x, cin), groups,
         _ptr(group_offsets), _ptr(token_ids), flags, _ptr(h), _ptr(p), _ptr(workspace), ws_bytes,
         _stream(stream)))
+
+
+def lhcal_accumulate_act_quant_workspace(dtype: int, tokens: int, cin: int, groups: int = 1) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load_library().lhcal_accumulate_act_quant_workspace(dtype, tokens, cin, groups, ctypes.byref(n)))
+    return int(n.value)
+
+
+def lhcal_accumulate_act_quant(x, h, p, act_gx, group_offsets=None, token_ids=None, flags: int = ACCUM_ADD,
+                               workspace=None, stream=None):
+    """Activation-aware accumulation with the input quantizer fused: X_q is derived from x (bf16)
+    in the kernel with the global scale act_gx (fp32 device scalar); h, p as for ``act``."""
+    tokens, cin = int(x.shape[0]), int(x.shape[1])
+    if x.numel() and x.stride(1) != 1:
+        raise ValueError("x must have unit stride along cin")
+    groups = 1 if group_offsets is None else int(group_offsets.numel()) - 1
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load_library().lhcal_accumulate_act_quant(
+        _dtype_id(x), _ptr(x), tokens, cin, _ld(x, cin), groups, _ptr(group_offsets), _ptr(token_ids),
+        _ptr(act_gx), flags, _ptr(h), _ptr(p), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def lhcal_act_fake_quant(x, act_gx, xq, stream=None):
+    """X_q = NVFP4 fake quant of bf16 x [tokens, cin] with global scale act_gx, into bf16 xq."""
+    tokens, cin = int(x.shape[0]), int(x.shape[1])
+    if x.numel() and (x.stride(1) != 1 or xq.stride(1) != 1):
+        raise ValueError("x and xq must have unit stride along cin")
+    _check(load_library().lhcal_act_fake_quant(_dtype_id(x), _ptr(x), tokens, cin, _ld(x, cin), _ptr(act_gx),
+                                               _ptr(xq), _ld(xq, cin), _stream(stream)))
 
 
 NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024
@@ -142,11 +179,11 @@ def lhcal_accumulate_noalloc(mode, x, h, xq=None, p=None, group_offsets=None, to
     """
     m = _mode_id(mode)
     tokens, cin = int(x.shape[0]), int(x.shape[1])
-    if x.stride(1) != 1:
+    if x.numel() and x.stride(1) != 1:
         raise ValueError("x must have unit stride along cin")
     groups = 1 if group_offsets is None else int(group_offsets.numel()) - 1
     _check(load_library().lhcal_accumulate_noalloc(
-        m, _dtype_id(x), _ptr(x), _ptr(xq), tokens, cin, int(x.stride(0)), groups,
+        m, _dtype_id(x), _ptr(x), _ptr(xq), tokens, cin, _ld(x, cin), groups,
         _ptr(group_offsets), _ptr(token_ids), flags, _ptr(h), _ptr(p), _stream(stream)))
 
 
@@ -199,14 +236,17 @@ class Buffers:
         self.wq = torch.empty((groups, rows, cin), dtype=torch.float32, device=device) if want_wq else None
         self.loss = torch.empty((groups, rows, nblk), dtype=torch.float32, device=device) if want_loss else None
         ws = lhcal_accumulate_workspace(self.mode, x_dtype, tokens, cin, groups)
+        if self.mode == ACT_AWARE and x_dtype == BF16:  # either activation-aware entry point
+            ws = max(ws, lhcal_accumulate_act_quant_workspace(x_dtype, tokens, cin, groups))
         self.workspace = torch.empty(max(ws // 4, 1), dtype=torch.float32, device=device) if ws else None
 
 
 def calibrate(mode, x, w, xq=None, group_offsets=None, token_ids=None, buffers: Buffers | None = None,
-              stream=None) -> Buffers:
+              stream=None, act_gx=None) -> Buffers:
     """The whole hot path on one layer: accumulate, count, finalize, global scale, sweep.
 
-    x [T, C], w [G, R, C] (and xq for ``act``, CSR routing for grouped layers) are device
+    x [T, C], w [G, R, C] (and for ``act`` either xq or act_gx, the input quantizer's global
+    scale from which the kernel derives X_q; CSR routing for grouped layers) are device
     tensors. Returns the buffers holding h, p, g, codes, wq and loss.
     """
     m = _mode_id(mode)
@@ -214,8 +254,12 @@ def calibrate(mode, x, w, xq=None, group_offsets=None, token_ids=None, buffers: 
     if buffers is None:
         buffers = Buffers(m, int(x.shape[0]), cin, rows, groups, _dtype_id(x), x.device)
     b = buffers
-    lhcal_accumulate(m, x, b.h, xq=xq, p=b.p, group_offsets=group_offsets, token_ids=token_ids,
-                     flags=ACCUM_OVERWRITE, workspace=b.workspace, stream=stream)
+    if m == ACT_AWARE and xq is None and act_gx is not None:
+        lhcal_accumulate_act_quant(x, b.h, b.p, act_gx, group_offsets=group_offsets, token_ids=token_ids,
+                                   flags=ACCUM_OVERWRITE, workspace=b.workspace, stream=stream)
+    else:
+        lhcal_accumulate(m, x, b.h, xq=xq, p=b.p, group_offsets=group_offsets, token_ids=token_ids,
+                         flags=ACCUM_OVERWRITE, workspace=b.workspace, stream=stream)
     lhcal_count_tokens(b.counts, tokens=int(x.shape[0]), group_offsets=group_offsets, flags=ACCUM_OVERWRITE,
                        stream=stream)
     lhcal_finalize(m, b.counts, b.h, p=b.p, stream=stream)
@@ -240,7 +284,7 @@ class HostOutputs:
 
 
 def calibrate_host(mode, x, w, buffers: Buffers, staging: dict, hxq=None, group_offsets=None, token_ids=None,
-                   out: HostOutputs | None = None, stream=None) -> HostOutputs:
+                   out: HostOutputs | None = None, stream=None, act_gx=None) -> HostOutputs:
     """The whole hot path from host tensors (pinned for asynchronous copies) to host results.
 
     ``staging`` holds device tensors shaped like the inputs under keys "x", "w" and, when
@@ -258,7 +302,7 @@ def calibrate_host(mode, x, w, buffers: Buffers, staging: dict, hxq=None, group_
         staging["offs"].copy_(group_offsets, non_blocking=True)
         staging["ids"].copy_(token_ids, non_blocking=True)
     calibrate(mode, staging["x"], staging["w"], xq=staging.get("xq"), group_offsets=staging.get("offs"),
-              token_ids=staging.get("ids"), buffers=buffers, stream=stream)
+              token_ids=staging.get("ids"), buffers=buffers, stream=stream, act_gx=act_gx)
     out.codes.copy_(buffers.codes, non_blocking=True)
     if out.wq is not None:
         out.wq.copy_(buffers.wq, non_blocking=True)
@@ -277,13 +321,14 @@ class CalibrationGraph:
     results land in ``self.buffers``.
     """
 
-    def __init__(self, mode, x, w, xq=None, group_offsets=None, token_ids=None, buffers: Buffers | None = None):
+    def __init__(self, mode, x, w, xq=None, group_offsets=None, token_ids=None, buffers: Buffers | None = None,
+                 act_gx=None):
         import torch
 
         m = _mode_id(mode)
         groups, rows, cin = (int(v) for v in w.shape)
         self.buffers = buffers or Buffers(m, int(x.shape[0]), cin, rows, groups, _dtype_id(x), x.device)
-        args = dict(xq=xq, group_offsets=group_offsets, token_ids=token_ids, buffers=self.buffers)
+        args = dict(xq=xq, group_offsets=group_offsets, token_ids=token_ids, buffers=self.buffers, act_gx=act_gx)
         calibrate(m, x, w, **args)
         torch.cuda.synchronize(x.device)
         self.graph = torch.cuda.CUDAGraph()

@@ -14,14 +14,19 @@
 //    (X_b^T) and both B fragments (X_b) of two m16n8k16 MMAs: the 16x16 block Hessian with no
 //    wasted MACs. bf16 x bf16 products are exact in the fp32 accumulator. For P the
 //    difference D = X_q - X (exact in fp32) is split into bf16 hi + lo parts, two more MMAs
-//    each. Dense: token ranges are split across CTAs and partials go to the workspace,
+//    each. (Forming P as H - X_q^T X instead would cost two MMAs fewer, but the cancellation
+//    multiplies the accumulation error by |H| / |P|, which exceeds 100 on real blocks.) Dense: token ranges are split across CTAs and partials go to the workspace,
 //    reduced in a fixed order by reduce_partials_kernel. Grouped: one CTA per (group, slab)
 //    gathers its routed rows through the CSR and writes the group's blocks directly.
+//    Activation-aware with the input quantizer fused (QUANT): only X streams in; each warp
+//    turns its block's 64 x 16 slice of the tile into X_q in shared memory (act_quant.cuh)
+//    and synchronises only with itself before the MMAs, so X is read from HBM once.
 //  * accum_diag_kernel: bf16 DIAG column sums of squares; each thread streams 8 columns
 //    (16-byte loads) over a token range; partials to the workspace, then reduce.
 //  * accum_generic_kernel: CUDA-core fp32 path for fp32 inputs (and grouped bf16 DIAG).
 #include <cooperative_groups.h>
 
+#include "act_quant.cuh"
 #include "common.cuh"
 
 namespace lhcal {
@@ -41,6 +46,17 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool v
 }
 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+
+__device__ __forceinline__ void lds128(uint32_t addr, uint32_t* v) {
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, const uint32_t* v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3])
+               : "memory");
+}
 
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
@@ -74,13 +90,14 @@ __device__ __forceinline__ uint32_t f2_to_bf2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&b);
 }
 
-// D = Xq - X for a bf16x2 pair, split into bf16 hi + lo (hi + lo = D to ~2^-17 relative).
+// D = Xq - X for a bf16x2 pair, split into bf16 hi + lo (hi + lo = D to ~2^-17 relative). Both
+// differences are exact in fp32; packed fp32 FMAs (x * -1 + y) do the pair at once.
 __device__ __forceinline__ void diff_split(uint32_t xq, uint32_t x, uint32_t& hi, uint32_t& lo) {
-  const float2 q = bf2_to_f2(xq), v = bf2_to_f2(x);
-  const float d0 = q.x - v.x, d1 = q.y - v.y;
-  hi = f2_to_bf2(d0, d1);
-  const float2 hf = bf2_to_f2(hi);
-  lo = f2_to_bf2(d0 - hf.x, d1 - hf.y);
+  const float2 m1 = make_float2(-1.f, -1.f);
+  const float2 d = __ffma2_rn(bf2_to_f2(x), m1, bf2_to_f2(xq));
+  hi = f2_to_bf2(d.x, d.y);
+  const float2 r = __ffma2_rn(bf2_to_f2(hi), m1, d);
+  lo = f2_to_bf2(r.x, r.y);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -93,11 +110,24 @@ constexpr int kTileTok = 64;
 constexpr int kRowBytes = kSlabCols * 2;              // 256 B per token row of the slab
 constexpr int kTileBytes = kTileTok * kRowBytes;      // 16 KB per tensor per stage
 
-template <bool ACT>
+// Shared memory: the cp.async ring (X_q and X per stage for ACT, X for FULL and QUANT), the
+// token-id ring, and for QUANT the X_q tile the warps write plus the quantizer tables.
+template <bool ACT, bool QUANT>
 struct MmaCfg {
+  static constexpr bool kTwo = ACT && !QUANT;  // two tensors stream in
   static constexpr int kStages = ACT ? 3 : 4;
-  static constexpr int kTensors = ACT ? 2 : 1;
-  static constexpr int kSmem = kStages * kTensors * kTileBytes + kStages * kTileTok * 4;  // + id ring
+  // Resident CTAs per SM the launch plans for: FULL 65 KB and QUANT 74 KB of shared memory
+  // fit three, ACT's 97 KB two.
+  static constexpr int kResident = kTwo ? 2 : 3;
+  // Clusters (cs <= 8 CTAs per slab) are used when they fill at least this fraction of a wave
+  // of resident CTAs; otherwise token splits and a reduction. The fused quantizer is bound by
+  // its integer pipe and wants every resident warp; the streaming variants are bound by HBM.
+  static constexpr double kClusterFill = QUANT ? 0.9 : 0.5;
+  static constexpr int kRing = kStages * (kTwo ? 2 : 1) * kTileBytes;
+  static constexpr int kIds = kStages * kTileTok * 4;
+  static constexpr int kXq = QUANT ? kTileBytes : 0;
+  static constexpr int kTab = QUANT ? static_cast<int>(sizeof(ActQuantTables)) : 0;
+  static constexpr int kSmem = kRing + kIds + kXq + kTab;
 };
 
 // Byte offset of 16-byte chunk c (0..15) of tile row r in the swizzled layout.
@@ -109,7 +139,7 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
 // Loads one 64-token x 128-column tile (both tensors for ACT). Rows pos0 + r for r < 64 with
 // pos0 + r < end; grouped tiles take the row of position pos0 + r from ids_s[r] (shared
 // memory), dense tiles use the position itself. Rows past end and columns past cin are zeros.
-template <bool ACT>
+template <bool TWO>
 __device__ __forceinline__ void load_tile(uint8_t* smem_stage, const __nv_bfloat16* x,
                                           const __nv_bfloat16* xq, int64_t ldx, int64_t col0,
                                           int64_t cin, const int32_t* ids_s, int64_t pos0, int64_t end) {
@@ -124,7 +154,7 @@ __device__ __forceinline__ void load_tile(uint8_t* smem_stage, const __nv_bfloat
     const int64_t row = ok ? (ids_s ? static_cast<int64_t>(ids_s[r]) : pos) : 0;
     const int64_t off = ok ? row * ldx + col0 + c * 8 : 0;
     const uint32_t dst = smem_u32(smem_stage) + swz(r, c);
-    if (ACT) {
+    if (TWO) {
       cp_async16(dst, xq + off, ok);
       cp_async16(dst + kTileBytes, x + off, ok);
     } else {
@@ -159,14 +189,17 @@ __device__ __forceinline__ void load_ids(int32_t* slot, const int32_t* ids, int6
 // its routed rows and written to out at item * out_item_stride. A single cp.async pipeline runs
 // through the tiles of all items, so short items (about 5 tiles per expert) still stream; the
 // accumulators are written out after each item's last tile. accumulate_into: out += sums.
-template <bool ACT, bool CLUSTER>
-__global__ void __launch_bounds__(kMmaThreads)
+// QUANT (with ACT): xq is unused and X_q comes from X through the input quantizer with the
+// global scale *act_gx.
+template <bool ACT, bool QUANT, bool CLUSTER>
+__global__ void __launch_bounds__(kMmaThreads, QUANT ? 3 : 1)
 accum_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ xq,
                  int64_t tokens, int64_t cin, int64_t ldx, const int32_t* __restrict__ group_offsets,
                  const int32_t* __restrict__ token_ids, int64_t tok_per_split, int64_t items_per_cta,
                  int64_t groups, float* __restrict__ out_h, float* __restrict__ out_p,
-                 int64_t out_item_stride, int accumulate_into) {
-  using Cfg = MmaCfg<ACT>;
+                 int64_t out_item_stride, int accumulate_into, const float* __restrict__ act_gx) {
+  static_assert(ACT || !QUANT, "the input quantizer belongs to the activation-aware mode");
+  using Cfg = MmaCfg<ACT, QUANT>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t slab = blockIdx.x;
@@ -258,8 +291,19 @@ accum_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __res
     return it1;
   };
   constexpr int S = Cfg::kStages;
-  constexpr int stage_bytes = Cfg::kTensors * kTileBytes;
-  int32_t* ids_ring = reinterpret_cast<int32_t*>(smem + S * stage_bytes);  // S slots of 64 ids
+  constexpr int stage_bytes = Cfg::kRing / S;
+  int32_t* ids_ring = reinterpret_cast<int32_t*>(smem + Cfg::kRing);  // S slots of 64 ids
+  uint8_t* xq_tile = smem + Cfg::kRing + Cfg::kIds;
+  ActQuantTables* tab = reinterpret_cast<ActQuantTables*>(smem + Cfg::kRing + Cfg::kIds + Cfg::kXq);
+  float inv6gx = 0.f;
+  bool steps = false;
+  if (QUANT) {
+    const float gx = __ldg(act_gx);
+    build_act_tables(*tab, gx, threadIdx.x, kMmaThreads);
+    inv6gx = 1.f / (6.f * gx);  // only a first guess of each block's scale code
+    steps = act_quant_steps(gx);
+    __syncthreads();
+  }
   int64_t i_pos = 0, i_end = 0, p_pos = 0, p_end = 0, c_pos = 0, c_end = 0;
   int64_t i_item = first_nonempty(it0, i_pos, i_end);
   int64_t i_tile = 0;
@@ -275,7 +319,7 @@ accum_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __res
     ++i_tile;
   };
   auto produce = [&](int64_t tile) {  // data of tile into stage tile % S
-    load_tile<ACT>(smem + (tile % S) * stage_bytes, x, xq, ldx, col0, cin,
+    load_tile<Cfg::kTwo>(smem + (tile % S) * stage_bytes, x, xq, ldx, col0, cin,
                    grouped ? ids_ring + (tile % S) * kTileTok : nullptr, p_pos, p_end);
     p_pos += kTileTok;
     if (p_pos >= p_end) p_item = first_nonempty(p_item + 1, p_pos, p_end);
@@ -307,16 +351,44 @@ accum_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __res
     if (it + S - 1 < ntiles) produce(it + S - 1);
     cp_async_commit();
     const uint32_t base = smem_u32(smem + (it % S) * stage_bytes);
+    uint32_t qbase = base;               // X_q (ACT) or X (FULL)
+    uint32_t xbase = base + kTileBytes;  // X (ACT)
+    if (QUANT) {
+      // This warp's block: tokens lane and lane + 32, chunks 2 warp and 2 warp + 1 of the tile.
+      qbase = smem_u32(xq_tile);
+      xbase = base;
+      // Both rows' loads, then both codes, then both table look-ups: the two dependency
+      // chains (row -> code -> thresholds) overlap.
+      uint32_t xv[2][8], av[2][8];
+      int code[2];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int r = lane + 32 * half;
+        lds128(base + swz(r, 2 * warp), xv[half]);
+        lds128(base + swz(r, 2 * warp + 1), xv[half] + 4);
+      }
+#pragma unroll
+      for (int half = 0; half < 2; ++half) code[half] = act_block_code(xv[half], av[half], inv6gx, *tab, steps);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int r = lane + 32 * half;
+        uint32_t qv[8];
+        act_block_apply(xv[half], av[half], code[half], qv, *tab, steps);
+        sts128(qbase + swz(r, 2 * warp), qv);
+        sts128(qbase + swz(r, 2 * warp + 1), qv + 4);
+      }
+      __syncwarp();  // the ldmatrix below reads rows written by the other lanes of this warp
+    }
 #pragma unroll
     for (int ts = 0; ts < kTileTok / 16; ++ts) {
-      const uint32_t addr = base + swz(ts * 16 + lrow, lchunk);
+      const uint32_t off = swz(ts * 16 + lrow, lchunk);
       uint32_t q0, q1, q2, q3;
-      ldmatrix_x4_trans(addr, q0, q1, q2, q3);  // X_q (ACT) or X (FULL)
+      ldmatrix_x4_trans(qbase + off, q0, q1, q2, q3);
       mma_bf16(acc_h[0], q0, q1, q2, q3, q0, q2);
       mma_bf16(acc_h[1], q0, q1, q2, q3, q1, q3);
       if (ACT) {
         uint32_t x0, x1, x2, x3;
-        ldmatrix_x4_trans(addr + kTileBytes, x0, x1, x2, x3);
+        ldmatrix_x4_trans(xbase + off, x0, x1, x2, x3);
         uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
         diff_split(q0, x0, h0, l0);
         diff_split(q1, x1, h1, l1);
@@ -564,10 +636,11 @@ Split token_split(int64_t tokens, int64_t ctas_per_split, int64_t target_ctas, i
   return s;
 }
 
-Split split_for(Path path, lhcal_mode mode, int64_t tokens, int64_t cin) {
+// resident: CTAs per SM of the tensor-core variant launched (MmaCfg::kResident).
+Split split_for(Path path, lhcal_mode mode, int64_t tokens, int64_t cin, int resident = 3) {
   switch (path) {
-    case Path::kMma:  // resident CTAs per SM: 3 (FULL, 65 KB shared) or 2 (ACT, 97 KB)
-      return token_split(tokens, ceil_div(cin, kSlabCols), (mode == LHCAL_ACT_AWARE ? 2 : 3) * kNumSms, kTileTok);
+    case Path::kMma:
+      return token_split(tokens, ceil_div(cin, kSlabCols), resident * kNumSms, kTileTok);
     case Path::kDiagBf16:
       return token_split(tokens, ceil_div(cin, kDiagCols), 8 * kNumSms, kDiagUnroll);
     default:
@@ -585,16 +658,16 @@ struct DensePlan {
   int64_t per;
 };
 
-DensePlan dense_plan(lhcal_mode mode, int64_t tokens, int64_t cin) {
+DensePlan dense_plan(lhcal_mode mode, int64_t tokens, int64_t cin, int resident, double cluster_fill) {
   const int64_t slabs = ceil_div(cin, kSlabCols);
-  const int64_t slots = (mode == LHCAL_ACT_AWARE ? 2 : 3) * kNumSms;
-  if (tokens > 0 && 2 * slabs * 8 >= slots) {
+  const int64_t slots = static_cast<int64_t>(resident) * kNumSms;
+  if (tokens > 0 && static_cast<double>(imin64(slabs * 8, slots)) >= cluster_fill * static_cast<double>(slots)) {
     int cs = 8;
     while (cs > 1 && slabs * cs > slots) cs /= 2;
     const int64_t per = ceil_div(ceil_div(tokens, cs), kTileTok) * kTileTok;
     return {true, cs, cs, per};
   }
-  const Split sp = split_for(Path::kMma, mode, tokens, cin);
+  const Split sp = split_for(Path::kMma, mode, tokens, cin, resident);
   return {false, 0, sp.splits, sp.per};
 }
 
@@ -619,35 +692,35 @@ lhcal_status launch_reduce(const float* ws, int64_t splits, int64_t stride, int6
   return check_launch("reduce partials");
 }
 
-template <bool ACT>
+template <bool ACT, bool QUANT>
 lhcal_status launch_mma(const void* x, const void* xq, int64_t tokens, int64_t cin, int64_t ldx,
                         int32_t groups, const int32_t* offs, const int32_t* ids, int accumulate_into,
-                        float* h, float* p, float* ws, cudaStream_t stream) {
-  using Cfg = MmaCfg<ACT>;
+                        float* h, float* p, float* ws, cudaStream_t stream, const float* act_gx) {
+  using Cfg = MmaCfg<ACT, QUANT>;
   // Allow up to the per-CTA maximum (the launch size decides occupancy). Set on every call with
   // the same value: cheap, thread-safe, and correct whichever device is current.
   constexpr int kMaxDynSmem = 227 * 1024;
-  for (const void* fn : {reinterpret_cast<const void*>(accum_mma_kernel<ACT, false>),
-                         reinterpret_cast<const void*>(accum_mma_kernel<ACT, true>)}) {
+  for (const void* fn : {reinterpret_cast<const void*>(accum_mma_kernel<ACT, QUANT, false>),
+                         reinterpret_cast<const void*>(accum_mma_kernel<ACT, QUANT, true>)}) {
     const cudaError_t attr = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
     if (attr != cudaSuccess) return fail(LHCAL_ERR_CUDA, "accumulate: %s", cudaGetErrorString(attr));
   }
   const int64_t slabs = ceil_div(cin, kSlabCols);
   const int64_t nblk = cin / kBlock;
   const auto* xb = static_cast<const __nv_bfloat16*>(x);
-  const auto* xqb = static_cast<const __nv_bfloat16*>(ACT ? xq : x);
+  const auto* xqb = static_cast<const __nv_bfloat16*>(Cfg::kTwo ? xq : x);
   if (offs != nullptr) {
     // Runs of experts per CTA so that about one wave of CTAs covers all (slab, expert) items.
-    const int64_t ctas_per_sm = ACT ? 2 : 3;
+    const int64_t ctas_per_sm = Cfg::kResident;
     const int64_t per = imax64(1, ceil_div(static_cast<int64_t>(groups) * slabs, ctas_per_sm * kNumSms));
     const dim3 grid(static_cast<unsigned>(slabs), static_cast<unsigned>(ceil_div(groups, per)));
     const size_t smem = Cfg::kSmem + static_cast<size_t>(ceil_div((per + 1) * 4, 16) * 16);
     if (smem > static_cast<size_t>(kMaxDynSmem)) return fail(LHCAL_ERR_UNSUPPORTED, "accumulate: too many groups per CTA");
-    accum_mma_kernel<ACT, false><<<grid, kMmaThreads, smem, stream>>>(
-        xb, xqb, tokens, cin, ldx, offs, ids, 0, per, groups, h, p, nblk * 256, accumulate_into);
+    accum_mma_kernel<ACT, QUANT, false><<<grid, kMmaThreads, smem, stream>>>(
+        xb, xqb, tokens, cin, ldx, offs, ids, 0, per, groups, h, p, nblk * 256, accumulate_into, act_gx);
     return check_launch("accumulate (grouped, tensor cores)");
   }
-  const DensePlan pl = dense_plan(ACT ? LHCAL_ACT_AWARE : LHCAL_FULL, tokens, cin);
+  const DensePlan pl = dense_plan(ACT ? LHCAL_ACT_AWARE : LHCAL_FULL, tokens, cin, Cfg::kResident, Cfg::kClusterFill);
   if (pl.cluster) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(slabs), static_cast<unsigned>(pl.cs));
@@ -661,10 +734,10 @@ lhcal_status launch_mma(const void* x, const void* xq, int64_t tokens, int64_t c
     at[0].val.clusterDim.z = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, accum_mma_kernel<ACT, true>, xb, xqb, tokens, cin, ldx,
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, accum_mma_kernel<ACT, QUANT, true>, xb, xqb, tokens, cin, ldx,
                                              static_cast<const int32_t*>(nullptr), static_cast<const int32_t*>(nullptr),
                                              pl.per, static_cast<int64_t>(1), static_cast<int64_t>(0), h, ACT ? p : h,
-                                             static_cast<int64_t>(0), accumulate_into);
+                                             static_cast<int64_t>(0), accumulate_into, act_gx);
     if (e != cudaSuccess) {
       cudaGetLastError();
       return fail(LHCAL_ERR_CUDA, "accumulate (tensor cores, clusters): %s", cudaGetErrorString(e));
@@ -675,8 +748,8 @@ lhcal_status launch_mma(const void* x, const void* xq, int64_t tokens, int64_t c
   float* ws_h = ws;
   float* ws_p = ws + pl.splits * per_split;
   const dim3 grid(static_cast<unsigned>(slabs), static_cast<unsigned>(pl.splits));
-  accum_mma_kernel<ACT, false><<<grid, kMmaThreads, Cfg::kSmem, stream>>>(
-      xb, xqb, tokens, cin, ldx, nullptr, nullptr, pl.per, 1, 0, ws_h, ws_p, per_split, 0);
+  accum_mma_kernel<ACT, QUANT, false><<<grid, kMmaThreads, Cfg::kSmem, stream>>>(
+      xb, xqb, tokens, cin, ldx, nullptr, nullptr, pl.per, 1, 0, ws_h, ws_p, per_split, 0, act_gx);
   lhcal_status st = check_launch("accumulate (tensor cores)");
   if (st != LHCAL_OK) return st;
   st = launch_reduce(ws_h, pl.splits, per_split, per_split, h, accumulate_into, stream);
@@ -714,11 +787,17 @@ lhcal_status launch_generic(const void* x, const void* xq, int64_t tokens, int64
 }  // namespace
 
 size_t accumulate_workspace_bytes(lhcal_mode mode, lhcal_dtype dtype, int64_t tokens, int64_t cin,
-                                  int32_t groups) {
+                                  int32_t groups, bool quant) {
   if (groups != 1 || tokens <= 0) return 0;
   const Path path = choose_path(mode, dtype, groups);
   if (path == Path::kMma) {
-    const DensePlan pl = dense_plan(mode, tokens, cin);
+    DensePlan pl;
+    if (mode == LHCAL_ACT_AWARE && quant)
+      pl = dense_plan(mode, tokens, cin, MmaCfg<true, true>::kResident, MmaCfg<true, true>::kClusterFill);
+    else if (mode == LHCAL_ACT_AWARE)
+      pl = dense_plan(mode, tokens, cin, MmaCfg<true, false>::kResident, MmaCfg<true, false>::kClusterFill);
+    else
+      pl = dense_plan(mode, tokens, cin, MmaCfg<false, false>::kResident, MmaCfg<false, false>::kClusterFill);
     return pl.cluster ? 0 : static_cast<size_t>(pl.splits) * floats_per_split(mode, cin) * sizeof(float);
   }
   const Split sp = split_for(path, mode, tokens, cin);
@@ -728,7 +807,7 @@ size_t accumulate_workspace_bytes(lhcal_mode mode, lhcal_dtype dtype, int64_t to
 lhcal_status launch_accumulate(lhcal_mode mode, lhcal_dtype dtype, const void* x, const void* xq,
                                int64_t tokens, int64_t cin, int64_t ldx, int32_t groups,
                                const int32_t* group_offsets, const int32_t* token_ids, int32_t flags,
-                               float* h, float* p, void* workspace, cudaStream_t stream) {
+                               float* h, float* p, void* workspace, cudaStream_t stream, const float* act_gx) {
   const int acc_into = (flags & LHCAL_ACCUM_OVERWRITE) ? 0 : 1;
   const int64_t nblk = cin / kBlock;
   const int64_t out_count = static_cast<int64_t>(groups) * (mode == LHCAL_DIAG ? cin : nblk * 256);
@@ -740,10 +819,17 @@ lhcal_status launch_accumulate(lhcal_mode mode, lhcal_dtype dtype, const void* x
   }
   float* ws = static_cast<float*>(workspace);
   const Path path = choose_path(mode, dtype, groups);
+  if (act_gx != nullptr && path != Path::kMma)
+    return fail(LHCAL_ERR_UNSUPPORTED, "the fused input quantizer needs bf16 activations");
   if (path == Path::kMma) {
+    if (mode == LHCAL_ACT_AWARE && act_gx != nullptr)
+      return launch_mma<true, true>(x, nullptr, tokens, cin, ldx, groups, group_offsets, token_ids, acc_into, h, p,
+                                    ws, stream, act_gx);
     if (mode == LHCAL_ACT_AWARE)
-      return launch_mma<true>(x, xq, tokens, cin, ldx, groups, group_offsets, token_ids, acc_into, h, p, ws, stream);
-    return launch_mma<false>(x, xq, tokens, cin, ldx, groups, group_offsets, token_ids, acc_into, h, p, ws, stream);
+      return launch_mma<true, false>(x, xq, tokens, cin, ldx, groups, group_offsets, token_ids, acc_into, h, p, ws,
+                                     stream, nullptr);
+    return launch_mma<false, false>(x, xq, tokens, cin, ldx, groups, group_offsets, token_ids, acc_into, h, p, ws,
+                                    stream, nullptr);
   }
   if (path == Path::kDiagBf16) {
     const Split sp = split_for(path, mode, tokens, cin);

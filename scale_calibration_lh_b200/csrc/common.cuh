@@ -74,13 +74,20 @@ lhcal_status launch_sweep_tc(lhcal_mode mode, lhcal_dtype dtype, const void* w, 
                              int64_t rows, int64_t cin, const float* h, const float* p, const float* g,
                              uint8_t* codes, float* wq, float* loss, cudaStream_t stream);
 
+// quant: the activation-aware variant with the input quantizer fused (X_q derived from x).
 size_t accumulate_workspace_bytes(lhcal_mode mode, lhcal_dtype dtype, int64_t tokens, int64_t cin,
-                                  int32_t groups);
+                                  int32_t groups, bool quant = false);
 
+// act_gx != NULL (ACT_AWARE, bf16 only): X_q is not read but derived from x in the kernel by the
+// NVFP4 activation fake quant with global scale *act_gx (xq must then be NULL).
 lhcal_status launch_accumulate(lhcal_mode mode, lhcal_dtype dtype, const void* x, const void* xq,
                                int64_t tokens, int64_t cin, int64_t ldx, int32_t groups,
                                const int32_t* group_offsets, const int32_t* token_ids, int32_t flags,
-                               float* h, float* p, void* workspace, cudaStream_t stream);
+                               float* h, float* p, void* workspace, cudaStream_t stream,
+                               const float* act_gx = nullptr);
+
+lhcal_status launch_act_fake_quant(const void* x, int64_t tokens, int64_t cin, int64_t ldx, const float* gx,
+                                   void* xq, int64_t ldq, cudaStream_t stream);
 
 lhcal_status launch_count_tokens(int32_t groups, int64_t tokens, const int32_t* group_offsets,
                                  int32_t flags, int64_t* counts, cudaStream_t stream);

@@ -87,6 +87,50 @@ lhcal_status check_groups(int32_t groups) {
     if (st_ != LHCAL_OK) return st_;            \
   } while (0)
 
+// Validation shared by lhcal_accumulate and lhcal_accumulate_act_quant (act_gx != NULL: X_q is
+// derived from x in the kernel, xq must be NULL).
+lhcal_status accumulate_checked(lhcal_mode mode, lhcal_dtype dtype, const void* x, const void* xq, int64_t tokens,
+                                int64_t cin, int64_t ldx, int32_t groups, const int32_t* group_offsets,
+                                const int32_t* token_ids, int32_t flags, float* h, float* p, void* workspace,
+                                size_t workspace_bytes, void* stream, const float* act_gx) {
+  if (!valid_mode(mode) || !valid_dtype(dtype)) return fail(LHCAL_ERR_UNSUPPORTED, "unknown mode or dtype");
+  LHCAL_TRY(check_cin(cin));
+  LHCAL_TRY(check_groups(groups));
+  if (tokens < 0) return fail(LHCAL_ERR_INVALID_ARG, "tokens (%lld) is negative", (long long)tokens);
+  if (tokens > (int64_t)INT32_MAX)
+    return fail(LHCAL_ERR_INVALID_ARG, "tokens (%lld) must fit in int32", (long long)tokens);
+  if (ldx < cin) return fail(LHCAL_ERR_INVALID_ARG, "ldx (%lld) < cin (%lld)", (long long)ldx, (long long)cin);
+  if ((ldx * (int64_t)elt_size(dtype)) % 16 != 0)
+    return fail(LHCAL_ERR_INVALID_ARG, "ldx * element size must be a multiple of 16 bytes");
+  if (flags != LHCAL_ACCUM_ADD && flags != LHCAL_ACCUM_OVERWRITE)
+    return fail(LHCAL_ERR_INVALID_ARG, "unknown flags %d", flags);
+  const bool grouped = group_offsets != nullptr || token_ids != nullptr;
+  if (grouped && (group_offsets == nullptr || token_ids == nullptr))
+    return fail(LHCAL_ERR_INVALID_ARG, "group_offsets and token_ids must both be set or both be NULL");
+  if (!grouped && groups != 1) return fail(LHCAL_ERR_INVALID_ARG, "groups > 1 needs group_offsets and token_ids");
+  if (mode == LHCAL_ACT_AWARE && xq == nullptr && act_gx == nullptr)
+    return fail(LHCAL_ERR_INVALID_ARG, "ACT_AWARE needs xq");
+  if (mode != LHCAL_ACT_AWARE && (xq != nullptr || p != nullptr))
+    return fail(LHCAL_ERR_INVALID_ARG, "xq and p are only for ACT_AWARE");
+  const size_t need = accumulate_workspace_bytes(mode, dtype, tokens, cin, groups, act_gx != nullptr);
+  if (workspace_bytes < need)
+    return fail(LHCAL_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
+  if (tokens > 0 || grouped) {
+    LHCAL_TRY(check_device_ptr(x, 16, "x"));
+    if (mode == LHCAL_ACT_AWARE && act_gx == nullptr) LHCAL_TRY(check_device_ptr(xq, 16, "xq"));
+  }
+  if (act_gx != nullptr) LHCAL_TRY(check_device_ptr(act_gx, 4, "act_gx"));
+  if (grouped) {
+    LHCAL_TRY(check_device_ptr(group_offsets, 4, "group_offsets"));
+    LHCAL_TRY(check_device_ptr(token_ids, 4, "token_ids"));
+  }
+  LHCAL_TRY(check_device_ptr(h, 16, "h"));
+  if (mode == LHCAL_ACT_AWARE) LHCAL_TRY(check_device_ptr(p, 16, "p"));
+  if (need > 0) LHCAL_TRY(check_device_ptr(workspace, 256, "workspace"));
+  return launch_accumulate(mode, dtype, x, xq, tokens, cin, ldx, groups, group_offsets, token_ids, flags, h, p,
+                           workspace, static_cast<cudaStream_t>(stream), act_gx);
+}
+
 }  // namespace
 }  // namespace lhcal
 
@@ -121,40 +165,50 @@ lhcal_status lhcal_accumulate(lhcal_mode mode, lhcal_dtype dtype, const void* x,
                               const int32_t* group_offsets, const int32_t* token_ids, int32_t flags,
                               float* h, float* p, void* workspace, size_t workspace_bytes, void* stream) {
   clear_error();
-  if (!valid_mode(mode) || !valid_dtype(dtype)) return fail(LHCAL_ERR_UNSUPPORTED, "unknown mode or dtype");
+  return accumulate_checked(mode, dtype, x, xq, tokens, cin, ldx, groups, group_offsets, token_ids, flags, h, p,
+                            workspace, workspace_bytes, stream, nullptr);
+}
+
+lhcal_status lhcal_accumulate_act_quant_workspace(lhcal_dtype dtype, int64_t tokens, int64_t cin, int32_t groups,
+                                                  size_t* bytes) {
+  clear_error();
+  if (bytes == nullptr) return fail(LHCAL_ERR_INVALID_ARG, "bytes is NULL");
+  if (dtype != LHCAL_BF16) return fail(LHCAL_ERR_UNSUPPORTED, "the fused input quantizer takes bf16 activations");
   LHCAL_TRY(check_cin(cin));
   LHCAL_TRY(check_groups(groups));
   if (tokens < 0) return fail(LHCAL_ERR_INVALID_ARG, "tokens (%lld) is negative", (long long)tokens);
-  if (tokens > (int64_t)INT32_MAX)
-    return fail(LHCAL_ERR_INVALID_ARG, "tokens (%lld) must fit in int32", (long long)tokens);
-  if (ldx < cin) return fail(LHCAL_ERR_INVALID_ARG, "ldx (%lld) < cin (%lld)", (long long)ldx, (long long)cin);
-  if ((ldx * (int64_t)elt_size(dtype)) % 16 != 0)
-    return fail(LHCAL_ERR_INVALID_ARG, "ldx * element size must be a multiple of 16 bytes");
-  if (flags != LHCAL_ACCUM_ADD && flags != LHCAL_ACCUM_OVERWRITE)
-    return fail(LHCAL_ERR_INVALID_ARG, "unknown flags %d", flags);
-  const bool grouped = group_offsets != nullptr || token_ids != nullptr;
-  if (grouped && (group_offsets == nullptr || token_ids == nullptr))
-    return fail(LHCAL_ERR_INVALID_ARG, "group_offsets and token_ids must both be set or both be NULL");
-  if (!grouped && groups != 1) return fail(LHCAL_ERR_INVALID_ARG, "groups > 1 needs group_offsets and token_ids");
-  if (mode == LHCAL_ACT_AWARE && xq == nullptr) return fail(LHCAL_ERR_INVALID_ARG, "ACT_AWARE needs xq");
-  if (mode != LHCAL_ACT_AWARE && (xq != nullptr || p != nullptr))
-    return fail(LHCAL_ERR_INVALID_ARG, "xq and p are only for ACT_AWARE");
-  const size_t need = accumulate_workspace_bytes(mode, dtype, tokens, cin, groups);
-  if (workspace_bytes < need)
-    return fail(LHCAL_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
-  if (tokens > 0 || grouped) {
-    LHCAL_TRY(check_device_ptr(x, 16, "x"));
-    if (mode == LHCAL_ACT_AWARE) LHCAL_TRY(check_device_ptr(xq, 16, "xq"));
-  }
-  if (grouped) {
-    LHCAL_TRY(check_device_ptr(group_offsets, 4, "group_offsets"));
-    LHCAL_TRY(check_device_ptr(token_ids, 4, "token_ids"));
-  }
-  LHCAL_TRY(check_device_ptr(h, 16, "h"));
-  if (mode == LHCAL_ACT_AWARE) LHCAL_TRY(check_device_ptr(p, 16, "p"));
-  if (need > 0) LHCAL_TRY(check_device_ptr(workspace, 256, "workspace"));
-  return launch_accumulate(mode, dtype, x, xq, tokens, cin, ldx, groups, group_offsets, token_ids, flags, h, p,
-                           workspace, static_cast<cudaStream_t>(stream));
+  *bytes = accumulate_workspace_bytes(LHCAL_ACT_AWARE, dtype, tokens, cin, groups, true);
+  return LHCAL_OK;
+}
+
+lhcal_status lhcal_accumulate_act_quant(lhcal_dtype dtype, const void* x, int64_t tokens, int64_t cin,
+                                        int64_t ldx, int32_t groups, const int32_t* group_offsets,
+                                        const int32_t* token_ids, const float* act_gx, int32_t flags,
+                                        float* h, float* p, void* workspace, size_t workspace_bytes,
+                                        void* stream) {
+  clear_error();
+  if (dtype != LHCAL_BF16) return fail(LHCAL_ERR_UNSUPPORTED, "the fused input quantizer takes bf16 activations");
+  if (act_gx == nullptr) return fail(LHCAL_ERR_INVALID_ARG, "act_gx is NULL");
+  return accumulate_checked(LHCAL_ACT_AWARE, dtype, x, nullptr, tokens, cin, ldx, groups, group_offsets, token_ids,
+                            flags, h, p, workspace, workspace_bytes, stream, act_gx);
+}
+
+lhcal_status lhcal_act_fake_quant(lhcal_dtype dtype, const void* x, int64_t tokens, int64_t cin, int64_t ldx,
+                                  const float* act_gx, void* xq, int64_t ldxq, void* stream) {
+  clear_error();
+  if (dtype != LHCAL_BF16) return fail(LHCAL_ERR_UNSUPPORTED, "the activation quantizer takes bf16");
+  LHCAL_TRY(check_cin(cin));
+  if (tokens < 0) return fail(LHCAL_ERR_INVALID_ARG, "tokens (%lld) is negative", (long long)tokens);
+  if (ldx < cin || ldxq < cin)
+    return fail(LHCAL_ERR_INVALID_ARG, "row strides (%lld, %lld) must be >= cin (%lld)", (long long)ldx,
+                (long long)ldxq, (long long)cin);
+  if ((ldx * 2) % 16 != 0 || (ldxq * 2) % 16 != 0)
+    return fail(LHCAL_ERR_INVALID_ARG, "row strides * 2 must be multiples of 16 bytes");
+  LHCAL_TRY(check_device_ptr(act_gx, 4, "act_gx"));
+  if (tokens == 0) return LHCAL_OK;
+  LHCAL_TRY(check_device_ptr(x, 16, "x"));
+  LHCAL_TRY(check_device_ptr(xq, 16, "xq"));
+  return launch_act_fake_quant(x, tokens, cin, ldx, act_gx, xq, ldxq, static_cast<cudaStream_t>(stream));
 }
 
 lhcal_status lhcal_count_tokens(int32_t groups, int64_t tokens, const int32_t* group_offsets, int32_t flags,

@@ -11,8 +11,9 @@ Workloads (token-major activations X[T, C], weights W[G, R, C]):
 * ``dense`` : X bf16 [16384, 4096], per-column std sigma_i = exp(N(0, 1)) with
   round(1% of C) distinct columns (chosen uniformly) multiplied by 20;
   W bf16 [4096, 4096] ~ N(0, (1/sqrt(4096))^2); full H.
-* ``act``   : X as ``dense`` at [32768, 4096]; X_q = NVFP4 max fake-quant of X
-  (see ``nvfp4_act_fake_quant``); W bf16 [12288, 4096]; activation-aware H and P.
+* ``act``   : X as ``dense`` at [32768, 4096]; W bf16 [12288, 4096]; activation-aware H
+  and P, where X_q is the NVFP4 input quantizer's output of X (derived from X by the
+  calibration path itself; this module draws X only).
 * ``wmse``  : X bf16 [65536, 12288], sigma_i = exp(N(0, 1.5^2)), no outliers;
   W bf16 [4096, 12288] ~ N(0, 1/12288); diagonal importance.
 * ``moe``   : X bf16 [16384, 2560] drawn as ``dense``; each token routed to 10
@@ -133,75 +134,6 @@ def _column_sigma(cin: int, seed: int, log_std: float, outlier_frac: float) -> n
     return sigma
 
 
-# --- activation quantizer for the ``act`` workload (input data, not the method) ---------
-
-_E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
-
-
-def _e4m3_round_positive(x: np.ndarray) -> np.ndarray:
-    """Nearest E4M3 value (ties to even), saturating at 448, for x >= 0 (fp64)."""
-    x = np.minimum(np.asarray(x, dtype=np.float64), 448.0)
-    out = np.zeros_like(x)
-    nz = x > 0
-    xe = x[nz]
-    # E4M3: 3 mantissa bits, min normal 2^-6, subnormal step 2^-9.
-    _, ex = np.frexp(xe)  # xe = m * 2^ex with m in [0.5, 1): floor(log2 xe) = ex - 1
-    e = np.maximum(ex.astype(np.float64) - 1.0, -6.0)
-    step = np.exp2(e - 3.0)
-    q = xe / step
-    fl = np.floor(q)
-    frac = q - fl
-    up = (frac > 0.5) | ((frac == 0.5) & (np.mod(fl, 2.0) == 1.0))
-    out[nz] = np.minimum((fl + up) * step, 448.0)
-    return out
-
-
-def _e2m1_round(u: np.ndarray) -> np.ndarray:
-    u = np.minimum(u, 6.0)
-    d = np.abs(u[..., None] - _E2M1_GRID)
-    best = d.min(axis=-1, keepdims=True)
-    tie_ok = d == best
-    # Among equally near grid points take the one with an even code (index).
-    even_ok = tie_ok & (np.arange(8) % 2 == 0)
-    idx = np.where(even_ok.any(-1), np.argmax(even_ok, -1), np.argmax(tie_ok, -1))
-    return _E2M1_GRID[idx]
-
-
-def nvfp4_act_fake_quant(x_bits: np.ndarray) -> np.ndarray:
-    """NVFP4 max fake-quant of bf16 activations X[T, C]; returns bf16 bits of X_q.
-
-    Per-tensor global scale gx = fp32(amax|X| / 2688); per (token, 16-wide block)
-    scale = E4M3(amax_blk / (6 gx)) * gx in fp32; each value rounds to E2M1
-    (nearest, ties to even, clamped at 6) and is rescaled, keeping its sign.
-    This only produces input data for the activation-aware workload.
-    """
-    x = bf16_bits_to_f32(x_bits).astype(np.float64)
-    t, c = x.shape
-    gx = np.float32(np.abs(x).max() / 2688.0)
-    out = np.empty((t, c), dtype=np.uint16)
-    rows_per = max(1, (1 << 18) // c)
-
-    def one(span):
-        lo, hi = span
-        xb = x[lo:hi].reshape(hi - lo, c // 16, 16)
-        amax_blk = np.abs(xb).max(-1)
-        if gx > 0:
-            code = _e4m3_round_positive(amax_blk / (6.0 * np.float64(gx)))
-        else:
-            code = np.zeros_like(amax_blk)
-        s = (code * np.float64(gx)).astype(np.float32).astype(np.float64)[..., None]
-        with np.errstate(divide="ignore", invalid="ignore"):
-            u = np.where(s > 0, np.abs(xb) / np.where(s > 0, s, 1.0), 0.0)
-        q = _e2m1_round(u)
-        xq = np.copysign((q * s).astype(np.float32), xb.astype(np.float32))
-        out[lo:hi] = f32_to_bf16_bits(xq.reshape(hi - lo, c))
-
-    spans = [(r, min(t, r + rows_per)) for r in range(0, t, rows_per)]
-    with _pool() as ex:
-        list(ex.map(one, spans))
-    return out
-
-
 # --- workloads ------------------------------------------------------------------------------
 
 
@@ -291,8 +223,6 @@ def make_layer(name: str, seed: int = 0, tokens: int | None = None, cin: int | N
     w = f32_to_bf16_bits(wf)
     del wf
     layer = Layer(name, mode, "bf16", x, w, meta={"sigma": sigma})
-    if name == "act":
-        layer.xq = nvfp4_act_fake_quant(x)
     if name == "moe":
         layer.group_offsets, layer.token_ids = moe_routing(T, G, top_k, seed)
     return layer

@@ -33,14 +33,41 @@ def to_device(a: np.ndarray | None, kind: str, device="cuda"):
     raise ValueError(kind)
 
 
+def act_inputs(layer):
+    """The input quantizer's side of an activation-aware layer, from the oracle: its global
+    scale gx = fp32(amax|X| / 2688) (meta["act_gx"]) and X_q = act_fake_quant(X, gx) (layer.xq).
+    The unfused entry point reads this X_q; the fused one derives it from X and gx itself."""
+    from oracle import lhcal_oracle as O
+    from scale_calibration_lh_b200 import synth
+
+    x = layer.x_f32()
+    gx = O.global_scale(x)
+    layer.meta["act_gx"] = gx
+    xq = O.act_fake_quant(x, gx)
+    layer.xq = synth.f32_to_bf16_bits(xq) if layer.dtype == "bf16" else xq
+    return layer
+
+
+def make_layer(name: str, seed: int = 0, **kw):
+    """synth.make_layer plus, for the activation-aware workload, the input quantizer's data."""
+    from scale_calibration_lh_b200 import synth
+
+    layer = synth.make_layer(name, seed, **kw)
+    return act_inputs(layer) if layer.mode == "act" else layer
+
+
 def layer_to_device(layer, device="cuda"):
+    import torch
+
     kind = "bf16" if layer.dtype == "bf16" else "f32"
+    gx = layer.meta.get("act_gx")
     return {
         "x": to_device(layer.x, kind, device),
         "xq": to_device(layer.xq, kind, device),
         "w": to_device(layer.w, kind, device),
         "offs": to_device(layer.group_offsets, "i32", device),
         "ids": to_device(layer.token_ids, "i32", device),
+        "act_gx": None if gx is None else torch.tensor([float(gx)], dtype=torch.float32, device=device),
     }
 
 

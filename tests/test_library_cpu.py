@@ -99,3 +99,17 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(L, "_lib", None)
     with pytest.raises(RuntimeError, match="not found"):
         L.load_library(str(tmp_path / "nope.so"))
+
+
+def test_input_quantizer_entry_points_validate_without_gpu(lib):
+    q = lib.lhcal_act_fake_quant
+    assert q(L.F32, None, 4, 32, 32, None, None, 32, None) == L.ERR_UNSUPPORTED
+    assert q(L.BF16, None, 4, 33, 33, None, None, 33, None) == L.ERR_INVALID_ARG  # cin not a multiple of 16
+    assert q(L.BF16, None, 4, 32, 36, None, None, 32, None) == L.ERR_INVALID_ARG  # 72-byte row stride
+    assert q(L.BF16, None, 4, 32, 32, None, None, 16, None) == L.ERR_INVALID_ARG  # ldxq < cin
+    assert q(L.BF16, None, -1, 32, 32, None, None, 32, None) == L.ERR_INVALID_ARG
+    assert q(L.BF16, None, 4, 32, 32, None, None, 32, None) == L.ERR_INVALID_ARG  # act_gx NULL
+    a = lib.lhcal_accumulate_act_quant
+    assert a(L.F32, None, 4, 32, 32, 1, None, None, None, 0, None, None, None, 0, None) == L.ERR_UNSUPPORTED
+    assert a(L.BF16, None, 4, 32, 32, 1, None, None, None, 0, None, None, None, 0, None) == L.ERR_INVALID_ARG
+    assert b"act_gx" in lib.lhcal_last_error_string()

@@ -33,29 +33,38 @@ def _sync():
     torch.cuda.synchronize()
 
 
-def _oracle_hessians(layer):
+def _oracle_hessians(layer, fused=False):
+    if fused:  # the oracle derives X_q from X with the input quantizer's global scale
+        return O.accumulate("act", layer.x_f32(), None, layer.group_offsets, layer.token_ids,
+                            act_gx=layer.meta["act_gx"])
     xq = layer.xq_f32() if layer.xq is not None else None
     hs, ps, counts = O.accumulate(layer.mode, layer.x_f32(), xq, layer.group_offsets, layer.token_ids)
     return hs, ps, counts
 
 
-def _run_and_check(layer, units=None, check_raw=True):
+def _run_and_check(layer, units=None, check_raw=True, fused=False):
+    """fused: activation-aware layer through the fused input quantizer (X and gx, no X_q)."""
     d = P.layer_to_device(layer)
     mode = L.MODE_IDS[layer.mode]
     G, R, C = layer.groups, layer.rows, layer.cin
     nblk = C // 16
     # Raw sums first (OVERWRITE into fresh buffers), compared before finalisation.
     b = L.Buffers(mode, layer.tokens, C, R, G, L.BF16 if layer.dtype == "bf16" else L.F32, "cuda")
-    L.lhcal_accumulate(mode, d["x"], b.h, xq=d["xq"], p=b.p, group_offsets=d["offs"], token_ids=d["ids"],
-                       flags=L.ACCUM_OVERWRITE, workspace=b.workspace)
+    if fused:
+        L.lhcal_accumulate_act_quant(d["x"], b.h, b.p, d["act_gx"], group_offsets=d["offs"], token_ids=d["ids"],
+                                     flags=L.ACCUM_OVERWRITE, workspace=b.workspace)
+    else:
+        L.lhcal_accumulate(mode, d["x"], b.h, xq=d["xq"], p=b.p, group_offsets=d["offs"], token_ids=d["ids"],
+                           flags=L.ACCUM_OVERWRITE, workspace=b.workspace)
     _sync()
-    hs, ps, counts = _oracle_hessians(layer)
+    hs, ps, counts = _oracle_hessians(layer, fused)
     report = {}
     if check_raw:
         report["h_raw"] = P.check_hessians(b.h.cpu().numpy(), hs, f"{layer.name} raw H")
         if ps is not None:
             report["p_raw"] = P.check_hessians(b.p.cpu().numpy(), ps, f"{layer.name} raw P")
-    b2 = L.calibrate(mode, d["x"], d["w"], xq=d["xq"], group_offsets=d["offs"], token_ids=d["ids"], buffers=b)
+    b2 = L.calibrate(mode, d["x"], d["w"], xq=None if fused else d["xq"], group_offsets=d["offs"],
+                     token_ids=d["ids"], buffers=b, act_gx=d["act_gx"] if fused else None)
     _sync()
     h, p = O.finalize(layer.mode, hs, ps, counts)
     report["h"] = P.check_hessians(b2.h.cpu().numpy(), h, f"{layer.name} H")
@@ -76,41 +85,41 @@ def _run_and_check(layer, units=None, check_raw=True):
 # ----------------------------------------------------------------------------- small cases
 
 def test_tiny_full_size_end_to_end():
-    r = _run_and_check(synth.make_layer("tiny", 0))
+    r = _run_and_check(P.make_layer("tiny", 0))
     assert r["sweep"]["units"] == 128
 
 
 @pytest.mark.parametrize("tokens,cin,rows", [(1000, 272, 300), (64, 128, 128), (1, 16, 1), (130, 400, 257)])
 def test_dense_full_bf16(tokens, cin, rows):
-    _run_and_check(synth.make_layer("dense", 1, tokens=tokens, cin=cin, rows=rows))
+    _run_and_check(P.make_layer("dense", 1, tokens=tokens, cin=cin, rows=rows))
 
 
 @pytest.mark.parametrize("tokens,cin,rows", [(777, 160, 200), (65, 48, 129)])
 def test_act_aware_bf16(tokens, cin, rows):
-    _run_and_check(synth.make_layer("act", 2, tokens=tokens, cin=cin, rows=rows))
+    _run_and_check(P.make_layer("act", 2, tokens=tokens, cin=cin, rows=rows))
 
 
 @pytest.mark.parametrize("tokens,cin,rows", [(1500, 2064, 130), (9, 32, 3)])
 def test_wmse_diag_bf16(tokens, cin, rows):
-    _run_and_check(synth.make_layer("wmse", 3, tokens=tokens, cin=cin, rows=rows))
+    _run_and_check(P.make_layer("wmse", 3, tokens=tokens, cin=cin, rows=rows))
 
 
 def test_moe_grouped_with_empty_experts():
-    layer = synth.make_layer("moe", 4, tokens=40, cin=160, rows=40, groups=64, top_k=3)
+    layer = P.make_layer("moe", 4, tokens=40, cin=160, rows=40, groups=64, top_k=3)
     counts = np.diff(layer.group_offsets)
     assert (counts == 0).any() and (counts > 1).any()
     _run_and_check(layer)
 
 
 def test_moe_grouped_full_rank_experts():
-    layer = synth.make_layer("moe", 13, tokens=600, cin=272, rows=150, groups=24, top_k=4)
+    layer = P.make_layer("moe", 13, tokens=600, cin=272, rows=150, groups=24, top_k=4)
     assert np.diff(layer.group_offsets).min() >= 32
     r = _run_and_check(layer)
     assert r["sweep"]["exempt"] < 0.05 * r["sweep"]["units"]
 
 
 def test_moe_grouped_diag_bf16_generic_path():
-    layer = synth.make_layer("moe", 5, tokens=50, cin=48, rows=20, groups=8, top_k=2)
+    layer = P.make_layer("moe", 5, tokens=50, cin=48, rows=20, groups=8, top_k=2)
     layer.mode = "diag"
     _run_and_check(layer)
 
@@ -217,7 +226,7 @@ def test_sweep_identity_hessian_is_plain_mse():
 # ----------------------------------------------------------------------------- accumulate semantics
 
 def test_accumulate_add_equals_one_pass_and_is_deterministic():
-    layer = synth.make_layer("act", 11, tokens=700, cin=96, rows=8)
+    layer = P.make_layer("act", 11, tokens=700, cin=96, rows=8)
     d = P.layer_to_device(layer)
     x, xq = d["x"], d["xq"]
     nb = 96 // 16
@@ -244,7 +253,7 @@ def test_accumulate_add_equals_one_pass_and_is_deterministic():
 @pytest.mark.parametrize("name", ["dense", "act"])
 def test_accumulate_cluster_path_overwrite_and_add(name):
     """Wide layers (32 column slabs) reduce token splits inside CTA clusters, with no workspace."""
-    layer = synth.make_layer(name, 14, tokens=3001, cin=4096, rows=2)
+    layer = P.make_layer(name, 14, tokens=3001, cin=4096, rows=2)
     mode = layer.mode
     assert L.lhcal_accumulate_workspace(mode, L.BF16, layer.tokens, layer.cin, 1) == 0
     d = P.layer_to_device(layer)
@@ -265,7 +274,7 @@ def test_accumulate_cluster_path_overwrite_and_add(name):
 
 
 def test_accumulate_strided_rows_and_zero_tokens():
-    layer = synth.make_layer("dense", 12, tokens=333, cin=64, rows=4)
+    layer = P.make_layer("dense", 12, tokens=333, cin=64, rows=4)
     d = P.layer_to_device(layer)
     wide = torch.zeros((333, 96), dtype=torch.bfloat16, device="cuda")
     wide[:, :64] = d["x"]
@@ -303,13 +312,13 @@ def test_device_and_host_pointer_errors():
 
 @pytest.mark.parametrize("name", ["dense", "act", "wmse", "moe"])
 def test_full_size_workload(name):
-    layer = synth.make_layer(name, 0)
+    layer = P.make_layer(name, 0)
     G, R, C = layer.groups, layer.rows, layer.cin
     units = P.sample_units(G, R, C // 16, 3000, seed=1)
     if name == "wmse":
         _run_and_check_wmse_full(layer, units)
-    else:
-        _run_and_check(layer, units=units, check_raw=False)
+    else:  # the activation-aware workload runs with the input quantizer fused, as benchmarked
+        _run_and_check(layer, units=units, check_raw=False, fused=name == "act")
 
 
 def _run_and_check_wmse_full(layer, units):
@@ -334,7 +343,7 @@ def _run_and_check_wmse_full(layer, units):
 
 def test_grouped_add_mode_over_two_batches():
     """Two routed batches added into the same per-expert sums equal one pass over both."""
-    layer = synth.make_layer("moe", 15, tokens=200, cin=96, rows=8, groups=16, top_k=3)
+    layer = P.make_layer("moe", 15, tokens=200, cin=96, rows=8, groups=16, top_k=3)
     d = P.layer_to_device(layer)
     x = d["x"]
     off = layer.group_offsets
@@ -366,7 +375,7 @@ def test_grouped_add_mode_over_two_batches():
 @pytest.mark.parametrize("mode", ["full", "act", "diag"])
 def test_sweep_optional_outputs_and_determinism(mode):
     name = {"full": "dense", "act": "act", "diag": "wmse"}[mode]
-    layer = synth.make_layer(name, 16, tokens=300, cin=128, rows=200)
+    layer = P.make_layer(name, 16, tokens=300, cin=128, rows=200)
     d = P.layer_to_device(layer)
     b = L.calibrate(mode, d["x"], d["w"], xq=d["xq"])
     codes1 = b.codes.clone()
@@ -385,14 +394,14 @@ def test_sweep_optional_outputs_and_determinism(mode):
 
 
 def test_diag_sweep_multiple_groups():
-    layer = synth.make_layer("moe", 17, tokens=120, cin=64, rows=70, groups=6, top_k=2)
+    layer = P.make_layer("moe", 17, tokens=120, cin=64, rows=70, groups=6, top_k=2)
     layer.mode = "diag"
     _run_and_check(layer)
 
 
 def test_graph_replay_matches_eager_calls():
-    layer_a = synth.make_layer("dense", 18, tokens=700, cin=512, rows=96)
-    layer_b = synth.make_layer("dense", 19, tokens=700, cin=512, rows=96)
+    layer_a = P.make_layer("dense", 18, tokens=700, cin=512, rows=96)
+    layer_b = P.make_layer("dense", 19, tokens=700, cin=512, rows=96)
     da, db = P.layer_to_device(layer_a), P.layer_to_device(layer_b)
     x, w = da["x"].clone(), da["w"].clone()
     graph = L.CalibrationGraph("full", x, w)
@@ -405,3 +414,104 @@ def test_graph_replay_matches_eager_calls():
         assert torch.equal(out.codes, eager.codes)
         assert torch.equal(out.wq.view(torch.int32), eager.wq.view(torch.int32))
         assert torch.equal(out.h.view(torch.int32), eager.h.view(torch.int32))
+
+
+# ----------------------------------------------------------------------------- input quantizer
+
+def _act_x(tokens, cin, seed):
+    """bf16 activations drawn like the dense workload, plus blocks that stress the quantizer:
+    all-zero, negative-zero, tiny (small and subnormal scale codes) and huge outlier blocks."""
+    rng = np.random.default_rng(seed)
+    sig = np.exp(rng.normal(0, 1, cin))
+    sig[rng.choice(cin, max(1, cin // 100), replace=False)] *= 20
+    x = rng.normal(size=(tokens, cin)) * sig
+    if tokens >= 4 and cin >= 32:
+        x[0, :16] = 0.0
+        x[1, 16:32] = -0.0
+        x[2, :16] *= 1e-30
+        x[3, 16:32] *= 1e4
+    return synth.f32_to_bf16_bits(x.astype(np.float32))
+
+
+@pytest.mark.parametrize("tokens,cin,pad,gx_factor", [(1, 16, 0, 1.0), (37, 48, 8, 1.0), (300, 4096, 0, 1.0),
+                                                       (129, 256, 24, 1e-3), (129, 256, 0, 1e3),
+                                                       (64, 64, 0, 0.0), (0, 32, 0, 1.0)])
+def test_act_fake_quant_kernel_bit_exact(tokens, cin, pad, gx_factor):
+    xb = _act_x(tokens, cin, 40 + tokens)
+    x32 = synth.bf16_bits_to_f32(xb)
+    gx = np.float32(O.global_scale(x32) * gx_factor) if tokens else np.float32(1.0)
+    want = synth.f32_to_bf16_bits(O.act_fake_quant(x32, gx)) if tokens else np.zeros((0, cin), np.uint16)
+    ld = cin + pad
+    xfull = np.zeros((tokens, ld), np.uint16)
+    xfull[:, :cin] = xb
+    dx = P.to_device(xfull, "bf16")[:, :cin]
+    dq_full = torch.full((tokens, ld), 7.0, dtype=torch.bfloat16, device="cuda")
+    dq = dq_full[:, :cin]
+    L.lhcal_act_fake_quant(dx, torch.tensor([float(gx)], device="cuda"), dq)
+    _sync()
+    got = dq_full.cpu().view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(got[:, :cin], want)
+    assert np.all(got[:, cin:] == np.uint16(0x40E0))  # the padding columns (7.0) are untouched
+
+
+@pytest.mark.parametrize("tokens,cin,rows", [(1000, 256, 40), (70, 48, 24), (2500, 4096, 16), (1, 16, 8)])
+def test_fused_act_quant_accumulation(tokens, cin, rows):
+    """X and gx in, no X_q: split (few slabs), cluster (4096 wide) and ragged cases."""
+    _run_and_check(P.make_layer("act", 31, tokens=tokens, cin=cin, rows=rows), fused=True)
+
+
+def test_fused_act_quant_grouped():
+    layer = synth.make_layer("moe", 32, tokens=300, cin=96, rows=24, groups=12, top_k=3)
+    layer.mode = "act"
+    P.act_inputs(layer)
+    _run_and_check(layer, fused=True)
+
+
+@pytest.mark.parametrize("tokens,cin,grouped,same_order", [(3000, 512, False, True), (2048, 4096, False, False),
+                                                            (400, 160, True, True)])
+def test_fused_equals_quantizer_then_unfused(tokens, cin, grouped, same_order):
+    """The fused kernel's sums equal the standalone quantizer's X_q fed to the two-tensor
+    accumulation: bit for bit where both split the tokens alike (the 512-wide layer, grouped
+    sums), else up to the fp32 summation order (the 4096-wide layer: clusters vs splits)."""
+    if grouped:
+        layer = synth.make_layer("moe", 33, tokens=tokens, cin=cin, rows=4, groups=10, top_k=3)
+        layer.mode = "act"
+        P.act_inputs(layer)
+    else:
+        layer = P.make_layer("act", 33, tokens=tokens, cin=cin, rows=4)
+    d = P.layer_to_device(layer)
+    G = layer.groups
+    shape = (G, cin // 16, 16, 16)
+    ws_bytes = max(L.lhcal_accumulate_workspace("act", L.BF16, tokens, cin, G),
+                   L.lhcal_accumulate_act_quant_workspace(L.BF16, tokens, cin, G))
+    ws = torch.empty(max(ws_bytes // 4, 1), dtype=torch.float32, device="cuda")
+    hf, pf = (torch.full(shape, 1.0, device="cuda") for _ in range(2))
+    L.lhcal_accumulate_act_quant(d["x"], hf, pf, d["act_gx"], group_offsets=d["offs"], token_ids=d["ids"],
+                                 flags=L.ACCUM_OVERWRITE, workspace=ws)
+    xq = torch.empty_like(d["x"])
+    L.lhcal_act_fake_quant(d["x"], d["act_gx"], xq)
+    hu, pu = (torch.full(shape, 2.0, device="cuda") for _ in range(2))
+    L.lhcal_accumulate("act", d["x"], hu, xq=xq, p=pu, group_offsets=d["offs"], token_ids=d["ids"],
+                       flags=L.ACCUM_OVERWRITE, workspace=ws)
+    _sync()
+    if same_order:
+        assert torch.equal(hf.view(torch.int32), hu.view(torch.int32))
+        assert torch.equal(pf.view(torch.int32), pu.view(torch.int32))
+    else:
+        P.check_hessians(hf.cpu().numpy(), hu.cpu().numpy().astype(np.float64), "fused vs unfused H", tol=1e-5)
+        P.check_hessians(pf.cpu().numpy(), pu.cpu().numpy().astype(np.float64), "fused vs unfused P", tol=1e-5)
+    # and the GPU quantizer's X_q is the oracle's
+    np.testing.assert_array_equal(xq.cpu().view(torch.int16).numpy().view(np.uint16), layer.xq)
+
+
+def test_fused_act_quant_rejects_fp32_and_missing_scale():
+    x = torch.zeros((8, 32), dtype=torch.float32, device="cuda")
+    h = torch.zeros((1, 2, 16, 16), device="cuda")
+    p = torch.zeros_like(h)
+    gx = torch.ones(1, device="cuda")
+    with pytest.raises(L.LhcalError) as e:
+        L.lhcal_accumulate_act_quant(x, h, p, gx, flags=L.ACCUM_OVERWRITE)
+    assert e.value.status == L.ERR_UNSUPPORTED
+    with pytest.raises(L.LhcalError) as e:
+        L.lhcal_accumulate_act_quant(x.bfloat16(), h, p, None, flags=L.ACCUM_OVERWRITE)
+    assert e.value.status == L.ERR_INVALID_ARG

@@ -56,7 +56,7 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
              ("act", "act", dict(tokens=3000, cin=1024, rows=4)),
              ("wmse", "diag", dict(tokens=5000, cin=4096, rows=4))]
     for name, mode, kw in cases:
-        layer = synth.make_layer(name, 21, **kw)
+        layer = P.make_layer(name, 21, **kw)
         d = P.layer_to_device(layer)
         nblk = layer.cin // 16
         assert L.lhcal_accumulate_workspace(mode, L.BF16, layer.tokens, layer.cin, 1) > 0
