@@ -85,10 +85,11 @@ def e2m1_round(u: np.ndarray) -> np.ndarray:
 # Global scale and candidate scales
 # ---------------------------------------------------------------------------------------
 
-def global_scale(w: np.ndarray) -> np.float32:
-    """g = fp32(amax|W| / (6 * 448)) (PR #2004: 448-normalized NVFP4 scaling)."""
+def global_scale(w: np.ndarray, fp8_max: float = FP8_MAX) -> np.float32:
+    """g = fp32(amax|W| / (6 * fp8_max)) (PR #2004: 448-normalized NVFP4 scaling; the NVFP4
+    "4/6" variant of the same page normalizes by 256 instead)."""
     amax = float(np.abs(np.asarray(w, dtype=np.float64)).max()) if np.size(w) else 0.0
-    return np.float32(amax / (FP4_MAX * FP8_MAX))
+    return np.float32(amax / (FP4_MAX * float(fp8_max)))
 
 
 def candidate_scales(g) -> np.ndarray:
@@ -284,7 +285,8 @@ def candidate_losses(mode: str, w_blk: np.ndarray, h_blk: np.ndarray, p_blk, g) 
 
     w_blk: [U, 16] fp32 weights; h_blk: [U, 16, 16] (full/act) or [U, 16] (diag);
     p_blk: [U, 16, 16] (act) or None. Returns (L [U, 126], wq [U, 126, 16] fp32, E0 [U]).
-    FULL: L = dW^T H dW; ACT: + 2 dW^T (P w); DIAG: sum Imp dW^2, with dW = wq - w (PR #1976).
+    FULL: L = dW^T H dW; ACT: + 2 dW^T (P w); DIAG: sum Imp dW^2, with dW = wq - w (PR #1976);
+    MSE: sum dW^2, the plain block MSE (h_blk unused), i.e. H = I.
     E0 is the q = 0 loss without the cross term, the scale for relative comparisons.
     """
     w = np.asarray(w_blk, dtype=np.float32)
@@ -292,6 +294,8 @@ def candidate_losses(mode: str, w_blk: np.ndarray, h_blk: np.ndarray, p_blk, g) 
     wq = fake_quant(w[:, None, :], s[None, :, None])  # [U, 126, 16]
     dw = wq.astype(np.float64) - w.astype(np.float64)[:, None, :]
     w64 = w.astype(np.float64)
+    if mode == "mse":
+        return np.einsum("uki,uki->uk", dw, dw), wq, np.einsum("ui,ui->u", w64, w64)
     h = np.asarray(h_blk, dtype=np.float64)
     if mode == "diag":
         loss = np.einsum("uki,ui->uk", dw * dw, h)
@@ -346,6 +350,8 @@ def loss_scale(mode: str, w_blk, h_blk, p_blk) -> np.ndarray:
     and loss errors are measured relative to max(|L*|, this scale).
     """
     a = np.abs(np.asarray(w_blk, dtype=np.float64))
+    if mode == "mse":
+        return np.einsum("ui,ui->u", a, a)
     h = np.abs(np.asarray(h_blk, dtype=np.float64))
     if mode == "diag":
         return np.einsum("ui,ui->u", a * a, h)
@@ -365,7 +371,7 @@ def gather_units(mode: str, w, h, p, g, units):
     ge, r, n = units[:, 0], units[:, 1], units[:, 2]
     cols = n[:, None] * BLOCK + np.arange(BLOCK)[None, :]
     w_blk = np.asarray(w)[ge[:, None], r[:, None], cols]
-    h_blk = np.asarray(h)[ge, n]
+    h_blk = None if h is None else np.asarray(h)[ge, n]
     p_blk = None if p is None else np.asarray(p)[ge, n]
     return w_blk, h_blk, p_blk, np.asarray(g)[ge]
 
@@ -390,7 +396,7 @@ def sweep(mode: str, w, h, p, g, units=None, chunk: int = 512):
         order = []
         for gv in np.unique(gu):
             sel = np.nonzero(gu == gv)[0]
-            o = sweep_units(mode, wb[sel], hb[sel], None if pb is None else pb[sel], gv)
+            o = sweep_units(mode, wb[sel], None if hb is None else hb[sel], None if pb is None else pb[sel], gv)
             for k in res:
                 res[k].append(o[k])
             order.append(sel)
@@ -401,8 +407,36 @@ def sweep(mode: str, w, h, p, g, units=None, chunk: int = 512):
     return {k: np.concatenate([o[k] for o in outs]) for k in outs[0]} if outs else {}
 
 
+def apply_scales(w, g, codes):
+    """Fake-quantized weights and per-block amax for chosen block-scale codes.
+
+    w [G, R, C] fp32 values; g [G]; codes [G, R, C/16] (E4M3 bytes, 0 = zero scale, values
+    above 126 taken as 126). Returns (wq fp32 [G, R, C], wq rounded to bf16 [G, R, C] as fp32
+    values, amax [G, R, C/16] fp32). The block's amax is the value whose NVFP4 scale is the
+    chosen one, fp32(6 v g) ("Add WMSE weight scale search calibration", PR #2283, the
+    quantizer state it fingerprints: amax and the per-block _amax); the exact product has at
+    most 29 significant bits, so it is rounded once.
+    """
+    w = np.asarray(w, dtype=np.float32)
+    gcount, rows, cin = w.shape
+    c = np.minimum(np.asarray(codes, dtype=np.int64), N_CANDIDATES)
+    v = np.where(c > 0, e4m3_value(np.maximum(c, 1)), 0.0)  # [G, R, N]
+    g64 = np.asarray(g, dtype=np.float32).astype(np.float64)[:, None, None]
+    s = (v * g64).astype(np.float32)
+    wq = fake_quant(w.reshape(gcount, rows, cin // BLOCK, BLOCK), s[..., None]).reshape(gcount, rows, cin)
+    amax = (FP4_MAX * v * g64).astype(np.float32)
+    return wq, f32_to_bf16_values(wq), amax
+
+
 def calibrate(mode: str, x, w, xq=None, group_offsets=None, token_ids=None, units=None, act_gx=None):
-    """The whole hot path: accumulate, finalize, global scale per group, sweep."""
+    """The whole hot path: accumulate, finalize, global scale per group, sweep. MSE has no
+    statistics: x is ignored and the sweep uses H = I."""
+    if mode == "mse":
+        w = np.asarray(w, dtype=np.float32)
+        g = np.array([global_scale(w[e]) for e in range(w.shape[0])], dtype=np.float32)
+        out = sweep(mode, w, None, None, g, units)
+        out.update({"h": None, "p": None, "g": g, "counts": None})
+        return out
     hsum, psum, counts = accumulate(mode, x, xq, group_offsets, token_ids, act_gx)
     h, p = finalize(mode, hsum, psum, counts)
     w = np.asarray(w, dtype=np.float32)

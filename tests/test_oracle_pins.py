@@ -320,6 +320,53 @@ def test_identity_hessian_is_plain_block_mse_by_exact_rationals():
             assert abs(loss[r, k] - float(ref)) <= 1e-12 * float(ref)
 
 
+def test_mse_mode_is_plain_block_mse_by_exact_rationals_and_equals_identity_hessian():
+    _, w = _layer(12, rows=4, cin=32)
+    g = O.global_scale(w[0])
+    s = O.candidate_scales(g)
+    wb = w[0].reshape(8, 16)
+    loss, _, e0 = O.candidate_losses("mse", wb, None, None, g)
+    for u in range(0, 8, 3):
+        for k in range(0, 126, 7):
+            ref = sum((Fraction(_fq_exact(float(wi), float(s[k]))) - Fraction(float(wi))) ** 2 for wi in wb[u])
+            assert abs(loss[u, k] - float(ref)) <= 1e-12 * float(ref)
+        assert e0[u] == pytest.approx(float(sum(Fraction(float(v)) ** 2 for v in wb[u])), rel=1e-14)
+    a = O.sweep("mse", w, None, None, np.array([g], np.float32))
+    b = O.sweep("full", w, np.eye(16)[None, None].repeat(2, 1), None, np.array([g], np.float32))
+    np.testing.assert_array_equal(a["codes"], b["codes"])
+    np.testing.assert_array_equal(a["wq"].view(np.int32), b["wq"].view(np.int32))
+
+
+def test_global_scale_four_over_six_is_256_normalized():
+    w = np.array([[0.5, -1.75, 0.25]], np.float32)
+    assert O.global_scale(w, 256.0) == np.float32(1.75 / 1536.0)
+    assert O.global_scale(w) == O.global_scale(w, 448.0) == np.float32(1.75 / 2688.0)
+
+
+def test_apply_scales_matches_the_sweep_and_exact_amax():
+    _, w = _layer(13, rows=6, cin=48)
+    g = np.array([O.global_scale(w[0])], np.float32)
+    out = O.sweep("mse", w, None, None, g)
+    codes = out["codes"].reshape(1, 6, 3).astype(np.int64)
+    codes[0, 0, 0] = 0    # zero scale: every weight becomes +-0
+    codes[0, 1, 1] = 200  # above 126: taken as 126
+    wq, wq16, amax = O.apply_scales(w, g, codes)
+    ref = out["wq"].reshape(1, 6, 3, 16).copy()
+    ref[0, 0, 0] = np.copysign(np.float32(0.0), w[0, 0, :16])
+    ref[0, 1, 1] = O.fake_quant(w[0, 1, 16:32], O.candidate_scales(g[0])[125])
+    np.testing.assert_array_equal(wq.view(np.int32), ref.reshape(1, 6, 48).view(np.int32))
+    gq = Fraction(float(g[0]))
+    for r in range(6):
+        for n in range(3):
+            c = min(int(codes[0, r, n]), 126)
+            exact = 6 * E4M3_ALL[c] * gq
+            assert amax[0, r, n] == np.float32(float(_round_binary(exact, 24, -126)))
+            for i in range(0, 16, 5):
+                v = Fraction(float(wq[0, r, 16 * n + i]))
+                mag = float(_round_binary(abs(v), 8, -126))
+                assert wq16[0, r, 16 * n + i] == np.copysign(mag, float(wq[0, r, 16 * n + i]))
+
+
 def test_sweep_is_exhaustive_lowest_code_on_ties():
     x, w = _layer(12, rows=8, cin=32)
     hs, _, c = O.accumulate("full", x)
