@@ -54,7 +54,9 @@ typedef enum { LHCAL_F32 = 0, LHCAL_BF16 = 1 } lhcal_dtype;
 typedef enum {
   LHCAL_FULL = 0,      /* H_n = X_b^T X_b / B                      (PR #788)  */
   LHCAL_ACT_AWARE = 1, /* H = X_q^T X_q / B, P = X_q^T (X_q - X) / B (PR #1976) */
-  LHCAL_DIAG = 2       /* Imp_i = ||X[:, i]||^2                      (PR #2283) */
+  LHCAL_DIAG = 2,      /* Imp_i = ||X[:, i]||^2                      (PR #2283) */
+  LHCAL_MSE = 3        /* plain block MSE, H = I: the "mse" method (PR #2283 fingerprint
+                          control); lhcal_scale_sweep only, with h = p = NULL */
 } lhcal_mode;
 
 /* lhcal_accumulate flags. */
@@ -169,11 +171,22 @@ lhcal_status lhcal_global_scale(lhcal_dtype dtype, const void* w, int32_t groups
                                 int64_t cin, float* g, void* stream);
 
 /*
+ * lhcal_global_scale with the FP8 normalization as a parameter: g[e] = fp32(max |W_e| /
+ * (6 * fp8_max)). fp8_max = 448 is lhcal_global_scale; 256 is the NVFP4 "4/6" variant, which
+ * "Add composable scale calibration to GPTQ" (PR #2004) names as 256-normalized. fp8_max must
+ * be finite and in (0, 448] with 6 * fp8_max exact in fp32 (any value with at most 21
+ * significant bits); LHCAL_ERR_INVALID_ARG otherwise.
+ */
+lhcal_status lhcal_global_scale_ex(lhcal_dtype dtype, const void* w, int32_t groups, int64_t rows,
+                                   int64_t cin, float fp8_max, float* g, void* stream);
+
+/*
  * Exhaustive FP8 scale sweep (PR #2283 "How", PR #1976 reviews). For each unit (e, r, n):
  *   for code k = 1..126: s_k = fp32(v_k * g[e]) with v_k the E4M3 value of k;
  *     q_i = E2M1 round-to-nearest-even of the exact |w_i| / s_k, clamped at 6;
  *     wq_i = copysign(fp32(q_i * s_k), w_i); dW = wq - w;
  *     L_k = dW^T H_n dW (FULL), + 2 dW^T (P_n w) (ACT), or sum_i Imp_{n,i} dW_i^2 (DIAG);
+ *     MSE: sum_i dW_i^2 (h = p = NULL);
  *   k* = the lowest k with the smallest L_k (losses may be negative).
  * Decisions on the quotient are exact for g >= 2^-90 or g == 0 (g == 0 gives wq = +-0 and
  * code 1). Losses are evaluated in fp32.
@@ -188,6 +201,23 @@ lhcal_status lhcal_global_scale(lhcal_dtype dtype, const void* w, int32_t groups
 lhcal_status lhcal_scale_sweep(lhcal_mode mode, lhcal_dtype dtype, const void* w, int32_t groups,
                                int64_t rows, int64_t cin, const float* h, const float* p,
                                const float* g, uint8_t* codes, float* wq, float* loss, void* stream);
+
+/*
+ * Outputs for chosen block-scale codes (for example the codes lhcal_scale_sweep wrote): for each
+ * unit (e, r, n) with s = fp32(v_c * g[e]), v_c the E4M3 value of code c:
+ *   wq   : out [groups, rows, cin] fp32, copysign(fp32(q_i * s), w_i), q_i the E2M1 rounding
+ *          of the exact |w_i| / s as in lhcal_scale_sweep (bit-identical to its wq), or NULL;
+ *   wq16 : out [groups, rows, cin] bf16, that fp32 value rounded to nearest even, or NULL;
+ *   amax : out [groups, rows, cin/16] fp32, the block's amax fp32(6 * v_c * g[e]) (the value
+ *          that maps to the chosen scale), or NULL.
+ * Code 0 is a zero scale (wq = +-0, amax = 0); codes above 126 are taken as 126. w: fp32 or
+ * bf16 [groups, rows, cin], 16-byte aligned; codes: device uint8 [groups, rows, cin/16].
+ * The fake-quantized weights are what the quantizer state of "Add WMSE weight scale search
+ * calibration" (PR #2283, refactor check) records next to amax and the per-block _amax.
+ */
+lhcal_status lhcal_apply_scales(lhcal_dtype dtype, const void* w, int32_t groups, int64_t rows, int64_t cin,
+                                const float* g, const uint8_t* codes, float* wq, void* wq16, float* amax,
+                                void* stream);
 
 /*
  * lhcal_accumulate for callers that cannot allocate device memory. The pages have no

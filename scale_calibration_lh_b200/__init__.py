@@ -18,11 +18,11 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_DEVICE_MISMATCH, ERR_CUDA, ERR_TIMEOUT
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "DEVICE_MISMATCH", 4: "CUDA", 5: "TIMEOUT"}
 # lhcal_dtype / lhcal_mode / flags
 F32, BF16 = 0, 1
-FULL, ACT_AWARE, DIAG = 0, 1, 2
+FULL, ACT_AWARE, DIAG, MSE = 0, 1, 2, 3
 ACCUM_ADD, ACCUM_OVERWRITE = 0, 1
 N_CANDIDATES = 126
 BLOCK = 16
-MODE_IDS = {"full": FULL, "act": ACT_AWARE, "diag": DIAG}
+MODE_IDS = {"full": FULL, "act": ACT_AWARE, "diag": DIAG, "mse": MSE}
 
 _lib = None
 
@@ -53,6 +53,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lhcal_count_tokens": [i32, i64, vp, i32, vp, vp],
         "lhcal_finalize": [i32, i32, i64, vp, vp, vp, vp],
         "lhcal_global_scale": [i32, vp, i32, i64, i64, vp, vp],
+        "lhcal_global_scale_ex": [i32, vp, i32, i64, i64, ctypes.c_float, vp, vp],
+        "lhcal_apply_scales": [i32, vp, i32, i64, i64, vp, vp, vp, vp, vp, vp],
         "lhcal_scale_sweep": [i32, i32, vp, i32, i64, i64, vp, vp, vp, vp, vp, vp, vp],
     }
     for name, args in sigs.items():
@@ -200,10 +202,21 @@ def lhcal_finalize(mode, counts, h, p=None, stream=None):
     _check(load_library().lhcal_finalize(m, groups, cin, _ptr(counts), _ptr(h), _ptr(p), _stream(stream)))
 
 
-def lhcal_global_scale(w, g, stream=None):
-    """w: [groups, rows, cin] fp32/bf16; g: fp32 [groups]."""
+def lhcal_global_scale(w, g, stream=None, fp8_max: float | None = None):
+    """w: [groups, rows, cin] fp32/bf16; g: fp32 [groups]. fp8_max: 448 (default) or 256 (4/6)."""
     groups, rows, cin = (int(v) for v in w.shape)
-    _check(load_library().lhcal_global_scale(_dtype_id(w), _ptr(w), groups, rows, cin, _ptr(g), _stream(stream)))
+    if fp8_max is None:
+        _check(load_library().lhcal_global_scale(_dtype_id(w), _ptr(w), groups, rows, cin, _ptr(g), _stream(stream)))
+    else:
+        _check(load_library().lhcal_global_scale_ex(_dtype_id(w), _ptr(w), groups, rows, cin, float(fp8_max),
+                                                    _ptr(g), _stream(stream)))
+
+
+def lhcal_apply_scales(w, g, codes, wq=None, wq16=None, amax=None, stream=None):
+    """Fake-quantized weights (fp32 wq, bf16 wq16) and per-block amax for chosen codes."""
+    groups, rows, cin = (int(v) for v in w.shape)
+    _check(load_library().lhcal_apply_scales(_dtype_id(w), _ptr(w), groups, rows, cin, _ptr(g), _ptr(codes),
+                                             _ptr(wq), _ptr(wq16), _ptr(amax), _stream(stream)))
 
 
 def lhcal_scale_sweep(mode, w, h, g, codes, wq=None, loss=None, p=None, stream=None):
@@ -228,14 +241,15 @@ class Buffers:
         self.mode = _mode_id(mode)
         nblk = cin // BLOCK
         hshape = (groups, nblk, BLOCK) if self.mode == DIAG else (groups, nblk, BLOCK, BLOCK)
-        self.h = torch.empty(hshape, dtype=torch.float32, device=device)
+        # MSE (H = I) needs no statistics.
+        self.h = None if self.mode == MSE else torch.empty(hshape, dtype=torch.float32, device=device)
         self.p = torch.empty(hshape, dtype=torch.float32, device=device) if self.mode == ACT_AWARE else None
         self.counts = torch.empty(groups, dtype=torch.int64, device=device)
         self.g = torch.empty(groups, dtype=torch.float32, device=device)
         self.codes = torch.empty((groups, rows, nblk), dtype=torch.uint8, device=device)
         self.wq = torch.empty((groups, rows, cin), dtype=torch.float32, device=device) if want_wq else None
         self.loss = torch.empty((groups, rows, nblk), dtype=torch.float32, device=device) if want_loss else None
-        ws = lhcal_accumulate_workspace(self.mode, x_dtype, tokens, cin, groups)
+        ws = 0 if self.mode == MSE else lhcal_accumulate_workspace(self.mode, x_dtype, tokens, cin, groups)
         if self.mode == ACT_AWARE and x_dtype == BF16:  # either activation-aware entry point
             ws = max(ws, lhcal_accumulate_act_quant_workspace(x_dtype, tokens, cin, groups))
         self.workspace = torch.empty(max(ws // 4, 1), dtype=torch.float32, device=device) if ws else None
@@ -251,6 +265,11 @@ def calibrate(mode, x, w, xq=None, group_offsets=None, token_ids=None, buffers: 
     """
     m = _mode_id(mode)
     groups, rows, cin = (int(v) for v in w.shape)
+    if m == MSE:  # plain block MSE: no statistics, x is not read
+        b = buffers or Buffers(m, 0, cin, rows, groups, _dtype_id(w), w.device)
+        lhcal_global_scale(w, b.g, stream=stream)
+        lhcal_scale_sweep(m, w, None, b.g, b.codes, wq=b.wq, loss=b.loss, stream=stream)
+        return b
     if buffers is None:
         buffers = Buffers(m, int(x.shape[0]), cin, rows, groups, _dtype_id(x), x.device)
     b = buffers

@@ -96,6 +96,10 @@ lhcal_status launch_finalize(lhcal_mode mode, int32_t groups, int64_t cin, const
                              float* h, float* p, cudaStream_t stream);
 
 lhcal_status launch_global_scale(lhcal_dtype dtype, const void* w, int32_t groups, int64_t rows,
-                                 int64_t cin, float* g, cudaStream_t stream);
+                                 int64_t cin, float* g, cudaStream_t stream, float fp8_max = 448.f);
+
+lhcal_status launch_apply_scales(lhcal_dtype dtype, const void* w, int32_t groups, int64_t rows, int64_t cin,
+                                 const float* g, const uint8_t* codes, float* wq, void* wq16, float* amax,
+                                 cudaStream_t stream);
 
 }  // namespace lhcal

@@ -63,7 +63,9 @@ lhcal_status check_launch(const char* what) {
 
 namespace {
 
+// Modes with activation statistics (accumulate / finalize); the sweep also takes LHCAL_MSE.
 bool valid_mode(lhcal_mode m) { return m == LHCAL_FULL || m == LHCAL_ACT_AWARE || m == LHCAL_DIAG; }
+bool valid_sweep_mode(lhcal_mode m) { return valid_mode(m) || m == LHCAL_MSE; }
 bool valid_dtype(lhcal_dtype d) { return d == LHCAL_F32 || d == LHCAL_BF16; }
 size_t elt_size(lhcal_dtype d) { return d == LHCAL_F32 ? 4 : 2; }
 
@@ -250,11 +252,45 @@ lhcal_status lhcal_global_scale(lhcal_dtype dtype, const void* w, int32_t groups
   return launch_global_scale(dtype, w, groups, rows, cin, g, static_cast<cudaStream_t>(stream));
 }
 
+lhcal_status lhcal_global_scale_ex(lhcal_dtype dtype, const void* w, int32_t groups, int64_t rows, int64_t cin,
+                                   float fp8_max, float* g, void* stream) {
+  clear_error();
+  if (!valid_dtype(dtype)) return fail(LHCAL_ERR_UNSUPPORTED, "unknown dtype");
+  if (!(fp8_max > 0.f && fp8_max <= 448.f) || static_cast<double>(6.f * fp8_max) != 6.0 * fp8_max)
+    return fail(LHCAL_ERR_INVALID_ARG, "fp8_max (%g) must be in (0, 448] with 6 * fp8_max exact in fp32",
+                static_cast<double>(fp8_max));
+  LHCAL_TRY(check_cin(cin));
+  LHCAL_TRY(check_groups(groups));
+  if (rows <= 0) return fail(LHCAL_ERR_INVALID_ARG, "rows (%lld) must be positive", (long long)rows);
+  LHCAL_TRY(check_device_ptr(w, 16, "w"));
+  LHCAL_TRY(check_device_ptr(g, 4, "g"));
+  return launch_global_scale(dtype, w, groups, rows, cin, g, static_cast<cudaStream_t>(stream), fp8_max);
+}
+
+lhcal_status lhcal_apply_scales(lhcal_dtype dtype, const void* w, int32_t groups, int64_t rows, int64_t cin,
+                                const float* g, const uint8_t* codes, float* wq, void* wq16, float* amax,
+                                void* stream) {
+  clear_error();
+  if (!valid_dtype(dtype)) return fail(LHCAL_ERR_UNSUPPORTED, "unknown dtype");
+  LHCAL_TRY(check_cin(cin));
+  LHCAL_TRY(check_groups(groups));
+  if (rows <= 0) return fail(LHCAL_ERR_INVALID_ARG, "rows (%lld) must be positive", (long long)rows);
+  LHCAL_TRY(check_device_ptr(w, 16, "w"));
+  LHCAL_TRY(check_device_ptr(g, 4, "g"));
+  LHCAL_TRY(check_device_ptr(codes, 1, "codes"));
+  if (wq != nullptr) LHCAL_TRY(check_device_ptr(wq, 16, "wq"));
+  if (wq16 != nullptr) LHCAL_TRY(check_device_ptr(wq16, 16, "wq16"));
+  if (amax != nullptr) LHCAL_TRY(check_device_ptr(amax, 4, "amax"));
+  return launch_apply_scales(dtype, w, groups, rows, cin, g, codes, wq, wq16, amax, static_cast<cudaStream_t>(stream));
+}
+
 lhcal_status lhcal_scale_sweep(lhcal_mode mode, lhcal_dtype dtype, const void* w, int32_t groups, int64_t rows,
                                int64_t cin, const float* h, const float* p, const float* g, uint8_t* codes,
                                float* wq, float* loss, void* stream) {
   clear_error();
-  if (!valid_mode(mode) || !valid_dtype(dtype)) return fail(LHCAL_ERR_UNSUPPORTED, "unknown mode or dtype");
+  if (!valid_sweep_mode(mode) || !valid_dtype(dtype)) return fail(LHCAL_ERR_UNSUPPORTED, "unknown mode or dtype");
+  if (mode == LHCAL_MSE && (h != nullptr || p != nullptr))
+    return fail(LHCAL_ERR_INVALID_ARG, "MSE takes no h or p");
   LHCAL_TRY(check_cin(cin));
   LHCAL_TRY(check_groups(groups));
   if (rows <= 0) return fail(LHCAL_ERR_INVALID_ARG, "rows (%lld) must be positive", (long long)rows);
@@ -262,7 +298,7 @@ lhcal_status lhcal_scale_sweep(lhcal_mode mode, lhcal_dtype dtype, const void* w
   if (mode == LHCAL_ACT_AWARE && p == nullptr) return fail(LHCAL_ERR_INVALID_ARG, "ACT_AWARE needs p");
   if (mode != LHCAL_ACT_AWARE && p != nullptr) return fail(LHCAL_ERR_INVALID_ARG, "p is only for ACT_AWARE");
   LHCAL_TRY(check_device_ptr(w, 16, "w"));
-  LHCAL_TRY(check_device_ptr(h, 16, "h"));
+  if (mode != LHCAL_MSE) LHCAL_TRY(check_device_ptr(h, 16, "h"));
   if (mode == LHCAL_ACT_AWARE) LHCAL_TRY(check_device_ptr(p, 16, "p"));
   LHCAL_TRY(check_device_ptr(g, 4, "g"));
   LHCAL_TRY(check_device_ptr(codes, 1, "codes"));

@@ -4,8 +4,12 @@
 // H and P are divided by the number of accumulated rows B. "[2/3] Speed up layerwise GPTQ on
 // MoE models" (PR #2864), embedded #2840: an expert that no token reaches gets the plain
 // search (here H = I, P = 0, Imp = 1). "Add composable scale calibration to GPTQ" (PR #2004):
-// 448-normalized NVFP4 global scale g = amax / (6 * 448).
+// 448-normalized NVFP4 global scale g = amax / (6 * 448), and 256-normalized for the page's
+// NVFP4 "4/6" variant. The output epilogue (apply_scales) writes the fake-quantized weights in
+// fp32 and bf16 and the per-block amax, the quantizer state "Add WMSE weight scale search
+// calibration" (PR #2283) fingerprints (amax, _amax, the fake-quantized weights).
 #include "common.cuh"
+#include "quant_tables.cuh"
 
 namespace lhcal {
 namespace {
@@ -89,11 +93,67 @@ amax_kernel(const T* __restrict__ w, int64_t per_group, uint32_t* __restrict__ a
   }
 }
 
-__global__ void scale_from_amax_kernel(int32_t groups, float* __restrict__ g) {
+// g = RN(amax / divisor), divisor = 6 * fp8_max exactly (2688 for 448, 1536 for 256).
+__global__ void scale_from_amax_kernel(int32_t groups, float divisor, float* __restrict__ g) {
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= groups) return;
   const float amax = __uint_as_float(reinterpret_cast<const uint32_t*>(g)[e]);
-  g[e] = __fdiv_rn(amax, 2688.f);  // 6 * 448
+  g[e] = __fdiv_rn(amax, divisor);
+}
+
+// Outputs for chosen codes: one thread per unit (group, row, block). s = fp32(v_c g) with the
+// exact E2M1 thresholds of quant_tables.cuh; wq = copysign(fp32(q s), w); the bf16 copy rounds
+// that fp32 value to nearest even; amax = fp32(6 v_c g). Code 0 is a zero scale; codes above
+// 126 are taken as 126.
+template <typename T>
+__global__ void __launch_bounds__(256)
+apply_scales_kernel(const T* __restrict__ w, int64_t units, int64_t nblk, int64_t rows_x_nblk,
+                    const float* __restrict__ g, const uint8_t* __restrict__ codes, float* __restrict__ wq,
+                    __nv_bfloat16* __restrict__ wq16, float* __restrict__ amax) {
+  for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < units;
+       u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t e = u / rows_x_nblk;
+    const int c = min(static_cast<int>(codes[u]), kCand);
+    const float gv = __ldg(g + e);
+    const float v = c == 0 ? 0.f : e4m3_value(c);
+    const float s = __fmul_rn(v, gv);
+    if (amax) amax[u] = __fmul_rn(6.f * v, gv);  // 6 v is exact
+    if (!wq && !wq16) continue;
+    float thr[kLev], val[kLev];
+#pragma unroll
+    for (int j = 0; j < kLev; ++j) {
+      thr[j] = level_threshold(j, s);
+      val[j] = __fmul_rn(e2m1_grid(j), s);
+    }
+    float x[kBlock];
+    load8<T>(w + u * kBlock, x);
+    load8<T>(w + u * kBlock + 8, x + 8);
+    float out[kBlock];
+#pragma unroll
+    for (int i = 0; i < kBlock; ++i) {
+      const float a = fabsf(x[i]);
+      float m = 0.f;  // s == 0: every threshold is 0 and every value 0
+#pragma unroll
+      for (int j = 1; j < kLev; ++j) m = a >= thr[j] ? val[j] : m;
+      out[i] = copysignf(m, x[i]);
+    }
+    if (wq) {
+      float4* dst = reinterpret_cast<float4*>(wq + u * kBlock);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) dst[q] = make_float4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
+    }
+    if (wq16) {
+      uint32_t pk[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const __nv_bfloat162 b = __floats2bfloat162_rn(out[2 * q], out[2 * q + 1]);
+        pk[q] = *reinterpret_cast<const uint32_t*>(&b);
+      }
+      uint4* dst = reinterpret_cast<uint4*>(wq16 + u * kBlock);
+      dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    }
+  }
 }
 
 }  // namespace
@@ -122,7 +182,7 @@ lhcal_status launch_finalize(lhcal_mode mode, int32_t groups, int64_t cin, const
 }
 
 lhcal_status launch_global_scale(lhcal_dtype dtype, const void* w, int32_t groups, int64_t rows,
-                                 int64_t cin, float* g, cudaStream_t stream) {
+                                 int64_t cin, float* g, cudaStream_t stream, float fp8_max) {
   // g doubles as the amax accumulator (bit patterns), then is converted in place.
   cudaError_t e = cudaMemsetAsync(g, 0, sizeof(float) * static_cast<size_t>(groups), stream);
   if (e != cudaSuccess) return fail(LHCAL_ERR_CUDA, "global scale: %s", cudaGetErrorString(e));
@@ -138,8 +198,25 @@ lhcal_status launch_global_scale(lhcal_dtype dtype, const void* w, int32_t group
     amax_kernel<float><<<grid, kAmaxThreads, 0, stream>>>(static_cast<const float*>(w), per_group, bits);
   lhcal_status st = check_launch("global scale (amax)");
   if (st != LHCAL_OK) return st;
-  scale_from_amax_kernel<<<static_cast<unsigned>(ceil_div(groups, 256)), 256, 0, stream>>>(groups, g);
+  scale_from_amax_kernel<<<static_cast<unsigned>(ceil_div(groups, 256)), 256, 0, stream>>>(groups, 6.f * fp8_max,
+                                                                                              g);
   return check_launch("global scale");
+}
+
+lhcal_status launch_apply_scales(lhcal_dtype dtype, const void* w, int32_t groups, int64_t rows, int64_t cin,
+                                 const float* g, const uint8_t* codes, float* wq, void* wq16, float* amax,
+                                 cudaStream_t stream) {
+  const int64_t nblk = cin / kBlock;
+  const int64_t units = static_cast<int64_t>(groups) * rows * nblk;
+  const unsigned blocks = static_cast<unsigned>(imin64(ceil_div(units, 256), 8 * kNumSms));
+  auto* w16 = static_cast<__nv_bfloat16*>(wq16);
+  if (dtype == LHCAL_BF16)
+    apply_scales_kernel<__nv_bfloat16><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(w), units, nblk,
+                                                                    rows * nblk, g, codes, wq, w16, amax);
+  else
+    apply_scales_kernel<float><<<blocks, 256, 0, stream>>>(static_cast<const float*>(w), units, nblk, rows * nblk,
+                                                           g, codes, wq, w16, amax);
+  return check_launch("apply scales");
 }
 
 }  // namespace lhcal

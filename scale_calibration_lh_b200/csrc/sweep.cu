@@ -5,7 +5,9 @@
 // Imp_i = ||X[:, i]||^2 replaces the block Hessian, the loss is sum_i Imp_i dW_i^2, and the
 // kernel's DIAGONAL specialization uses a weighted sum instead of a matrix product.
 // "Add activation-aware local Hessian scale calibration" (PR #1976) reviews: dW = quant(w) - w,
-// best loss starts at +inf. FULL and activation-aware losses run in sweep_tc.cu.
+// best loss starts at +inf. FULL and activation-aware losses run in sweep_tc.cu. The plain
+// block MSE (LHCAL_MSE, H = I: the "mse" method next to which "Add WMSE weight scale search
+// calibration" fingerprints local_hessian) is this kernel with every importance 1.
 //
 // Design (sm_100a, FP32 pipe):
 //  * One thread owns one unit (group e, row r, block n); a CTA covers 128 rows of one block.
@@ -59,7 +61,7 @@ __device__ __forceinline__ void load_w16(const WT* src, float* w) {
 
 template <typename WT>
 __global__ void __launch_bounds__(kThreads)
-sweep_diag_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float* __restrict__ imp,
+sweep_diag_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float* __restrict__ imp,  // NULL: all 1
                   const float* __restrict__ g, uint8_t* __restrict__ codes, float* __restrict__ wq,
                   float* __restrict__ loss) {
   __shared__ DiagShared sh;
@@ -74,7 +76,7 @@ sweep_diag_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const flo
     const float s = candidate_scale(k, gs);
     sh.tab[idx] = make_float2(level_threshold(j, s), __fmul_rn(e2m1_grid(j), s));
   }
-  if (threadIdx.x < kBlock) sh.imp[threadIdx.x] = __ldg(imp + (e * nblk + n) * kBlock + threadIdx.x);
+  if (threadIdx.x < kBlock) sh.imp[threadIdx.x] = imp ? __ldg(imp + (e * nblk + n) * kBlock + threadIdx.x) : 1.f;
   {
     const int64_t row = rbase + threadIdx.x;
     float m = __int_as_float(0x7f800000);
@@ -251,7 +253,8 @@ lhcal_status launch_sweep(lhcal_mode mode, lhcal_dtype dtype, const void* w, int
   // FULL and ACT_AWARE: quadratic form on tensor cores; DIAG: FP32 weighted sum.
   if (mode == LHCAL_FULL || mode == LHCAL_ACT_AWARE)
     return launch_sweep_tc(mode, dtype, w, groups, rows, cin, h, p, g, codes, wq, loss, stream);
-  if (mode != LHCAL_DIAG) return fail(LHCAL_ERR_UNSUPPORTED, "scale sweep: unsupported mode");
+  if (mode != LHCAL_DIAG && mode != LHCAL_MSE) return fail(LHCAL_ERR_UNSUPPORTED, "scale sweep: unsupported mode");
+  if (mode == LHCAL_MSE) h = nullptr;
   const dim3 grid(static_cast<unsigned>(ceil_div(rows, kThreads)), static_cast<unsigned>(cin / kBlock),
                   static_cast<unsigned>(groups));
   if (dtype == LHCAL_BF16)

@@ -113,3 +113,21 @@ def test_input_quantizer_entry_points_validate_without_gpu(lib):
     assert a(L.F32, None, 4, 32, 32, 1, None, None, None, 0, None, None, None, 0, None) == L.ERR_UNSUPPORTED
     assert a(L.BF16, None, 4, 32, 32, 1, None, None, None, 0, None, None, None, 0, None) == L.ERR_INVALID_ARG
     assert b"act_gx" in lib.lhcal_last_error_string()
+
+
+def test_mse_scale_and_output_entry_points_validate_without_gpu(lib):
+    # MSE takes no statistics.
+    assert lib.lhcal_scale_sweep(3, 1, None, 1, 4, 32, ctypes.c_void_p(256), None, None, None, None, None,
+                                 None) == L.ERR_INVALID_ARG
+    assert b"MSE" in lib.lhcal_last_error_string()
+    # MSE is a sweep mode only.
+    assert lib.lhcal_finalize(3, 1, 32, None, None, None, None) == L.ERR_UNSUPPORTED
+    gs = lib.lhcal_global_scale_ex
+    for bad in (0.0, -1.0, 449.0, 1.0 / 3.0, float("nan")):
+        assert gs(1, None, 1, 4, 32, bad, None, None) == L.ERR_INVALID_ARG, bad
+    assert b"fp8_max" in lib.lhcal_last_error_string()
+    assert gs(7, None, 1, 4, 32, 256.0, None, None) == L.ERR_UNSUPPORTED
+    ap = lib.lhcal_apply_scales
+    assert ap(1, None, 1, 4, 33, None, None, None, None, None, None) == L.ERR_INVALID_ARG
+    assert ap(1, None, 1, 0, 32, None, None, None, None, None, None) == L.ERR_INVALID_ARG
+    assert ap(5, None, 1, 4, 32, None, None, None, None, None, None) == L.ERR_UNSUPPORTED

@@ -515,3 +515,87 @@ def test_fused_act_quant_rejects_fp32_and_missing_scale():
     with pytest.raises(L.LhcalError) as e:
         L.lhcal_accumulate_act_quant(x.bfloat16(), h, p, None, flags=L.ACCUM_OVERWRITE)
     assert e.value.status == L.ERR_INVALID_ARG
+
+
+# ----------------------------------------------------------------------------- mse, 4/6 scale, outputs
+
+@pytest.mark.parametrize("name,kw", [("dense", dict(tokens=16, cin=272, rows=300)), ("tiny", dict()),
+                                     ("moe", dict(tokens=16, cin=64, rows=40, groups=5, top_k=2))])
+def test_mse_sweep(name, kw):
+    """Plain block MSE (H = I): no statistics, the diagonal kernel with unit weights."""
+    layer = synth.make_layer(name, 41, **kw)
+    d = P.layer_to_device(layer)
+    b = L.calibrate("mse", None, d["w"])
+    _sync()
+    assert b.h is None
+    w32 = layer.w_f32()
+    G, R, C = layer.groups, layer.rows, layer.cin
+    g = np.array([O.global_scale(w32[e]) for e in range(G)], np.float32)
+    np.testing.assert_array_equal(b.g.cpu().numpy().view(np.int32), g.view(np.int32))
+    units = P.all_units(G, R, C // 16)
+    ref = O.sweep("mse", w32, None, None, g, units)
+    gc, gw, gl = P.gather_gpu_units(b.codes, b.wq, b.loss, units)
+    P.check_sweep(gc, gw, gl, ref, f"{name} mse")
+
+
+def test_mse_sweep_full_size_weights():
+    layer = synth.make_layer("dense", 0, tokens=16)
+    d = P.layer_to_device(layer)
+    b = L.calibrate("mse", None, d["w"])
+    _sync()
+    w32 = layer.w_f32()
+    g = np.array([O.global_scale(w32[0])], np.float32)
+    units = P.sample_units(1, layer.rows, layer.cin // 16, 3000, seed=2)
+    ref = O.sweep("mse", w32, None, None, g, units)
+    gc, gw, gl = P.gather_gpu_units(b.codes, b.wq, b.loss, units)
+    P.check_sweep(gc, gw, gl, ref, "dense mse full size")
+
+
+@pytest.mark.parametrize("name", ["dense", "tiny", "moe"])
+def test_global_scale_fp8_max(name):
+    layer = synth.make_layer(name, 42, tokens=16, rows=64, cin=64, **({"groups": 7, "top_k": 2} if name == "moe" else {}))
+    d = P.layer_to_device(layer)
+    w32 = layer.w_f32()
+    for fp8_max in (448.0, 256.0):
+        g = torch.empty(layer.groups, dtype=torch.float32, device="cuda")
+        L.lhcal_global_scale(d["w"], g, fp8_max=fp8_max)
+        _sync()
+        want = np.array([O.global_scale(w32[e], fp8_max) for e in range(layer.groups)], np.float32)
+        np.testing.assert_array_equal(g.cpu().numpy().view(np.int32), want.view(np.int32))
+    g = torch.empty(layer.groups, dtype=torch.float32, device="cuda")
+    for bad in (0.0, 500.0, 1.0 / 3.0):
+        with pytest.raises(L.LhcalError) as e:
+            L.lhcal_global_scale(d["w"], g, fp8_max=bad)
+        assert e.value.status == L.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("name,kw", [("dense", dict(tokens=400, cin=256, rows=96)), ("tiny", dict()),
+                                     ("moe", dict(tokens=80, cin=96, rows=24, groups=6, top_k=2))])
+def test_apply_scales_bit_exact(name, kw):
+    """Fake-quantized weights (fp32, bf16) and per-block amax for the sweep's codes and for
+    arbitrary codes (zero, every candidate, out of range), against the oracle."""
+    layer = synth.make_layer(name, 43, **kw)
+    d = P.layer_to_device(layer)
+    mode = layer.mode
+    b = L.calibrate(mode, d["x"], d["w"], group_offsets=d["offs"], token_ids=d["ids"])
+    G, R, C = layer.groups, layer.rows, layer.cin
+    rng = np.random.default_rng(7)
+    crafted = rng.integers(0, 256, (G, R, C // 16)).astype(np.uint8)
+    crafted.flat[:128] = np.arange(128, dtype=np.uint8)
+    w32 = layer.w_f32()
+    g_host = b.g.cpu().numpy()
+    for codes in (b.codes, P.to_device(crafted, "i32").to(torch.uint8)):
+        wq = torch.empty((G, R, C), dtype=torch.float32, device="cuda")
+        wq16 = torch.empty((G, R, C), dtype=torch.bfloat16, device="cuda")
+        amax = torch.empty((G, R, C // 16), dtype=torch.float32, device="cuda")
+        L.lhcal_apply_scales(d["w"], b.g, codes, wq=wq, wq16=wq16, amax=amax)
+        _sync()
+        rw, rw16, ra = O.apply_scales(w32, g_host, codes.cpu().numpy())
+        np.testing.assert_array_equal(wq.cpu().numpy().view(np.int32), rw.view(np.int32))
+        np.testing.assert_array_equal(wq16.float().cpu().numpy().view(np.int32), rw16.view(np.int32))
+        np.testing.assert_array_equal(amax.cpu().numpy().view(np.int32), ra.view(np.int32))
+    # The sweep's own fake-quantized weights are the apply_scales output for its codes.
+    wq = torch.empty((G, R, C), dtype=torch.float32, device="cuda")
+    L.lhcal_apply_scales(d["w"], b.g, b.codes, wq=wq)
+    _sync()
+    assert torch.equal(wq.view(torch.int32), b.wq.view(torch.int32))
