@@ -77,8 +77,8 @@ __device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
   return v;
 }
 
-// addr - step if a < t (fp32 compare), else addr. Plain C lets the compiler fold the compare into a
-// predicated subtract; it measured faster than the inline-asm select it replaces, with the same codes.
+// addr - step if a < t (fp32 compare), else addr. Plain C: measured faster than an inline-asm
+// predicated select, with the same codes.
 __device__ __forceinline__ uint32_t drop_if_below(uint32_t addr, float a, float t, uint32_t step) {
   return a < t ? addr - step : addr;
 }
