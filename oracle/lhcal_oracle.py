@@ -407,6 +407,107 @@ def sweep(mode: str, w, h, p, g, units=None, chunk: int = 512):
     return {k: np.concatenate([o[k] for o in outs]) for k in outs[0]} if outs else {}
 
 
+def losses_for_scales(mode: str, w_blk, h_blk, p_blk, s) -> tuple:
+    """Losses of given block scales: s [U, K] fp32 (0 allowed) for U units.
+
+    Same definitions as ``candidate_losses`` (which is this with the 126 candidate scales
+    for every unit). Returns (L [U, K], wq [U, K, 16] fp32).
+    """
+    w = np.asarray(w_blk, dtype=np.float32)
+    s = np.asarray(s, dtype=np.float32)
+    wq = fake_quant(w[:, None, :], s[:, :, None])
+    dw = wq.astype(np.float64) - w.astype(np.float64)[:, None, :]
+    if mode == "mse":
+        return np.einsum("uki,uki->uk", dw, dw), wq
+    h = np.asarray(h_blk, dtype=np.float64)
+    if mode == "diag":
+        return np.einsum("uki,ui->uk", dw * dw, h), wq
+    loss = np.einsum("uki,uij,ukj->uk", dw, h, dw)
+    if mode == "act":
+        pw = np.einsum("uij,uj->ui", np.asarray(p_blk, dtype=np.float64), w.astype(np.float64))
+        loss = loss + 2.0 * np.einsum("uki,ui->uk", dw, pw)
+    return loss, wq
+
+
+def multiplier_codes(w_blk, g, multipliers) -> np.ndarray:
+    """Block-scale codes of the amax-multiplier search: [U, M].
+
+    For multiplier m the block's candidate amax is fp32(m * amax_blk) (amax_blk = max |w| of
+    the block), and it becomes a block scale as in the NVFP4 quantizer: the E4M3 code nearest to
+    amax / (6 g) on the exact quotient (ties to the even code, saturating at 448; 0 is a zero
+    scale). g == 0 gives code 0.
+    """
+    w = np.asarray(w_blk, dtype=np.float32)
+    amax = np.abs(w.astype(np.float64)).max(axis=1)  # exact
+    m = np.asarray(multipliers, dtype=np.float32).astype(np.float64)
+    with np.errstate(invalid="ignore"):
+        a = (m[None, :] * amax[:, None]).astype(np.float32).astype(np.float64)  # exact product, one rounding
+    a = np.where(np.isnan(a) | (a < 0), 0.0, a)  # a negative or NaN candidate amax counts as 0
+    g64 = np.float64(np.float32(g))
+    if g64 == 0:
+        return np.zeros(a.shape, dtype=np.int64)
+    return e4m3_round(a / (FP4_MAX * g64))
+
+
+def multiplier_search_units(mode: str, w_blk, h_blk, p_blk, g, multipliers):
+    """Amax-multiplier search on U units (the non-sweep search of the MSE calibrator that
+    "add local hessian calibration", PR #788, configures by step size and multipliers).
+
+    Candidates are the multipliers in the given order; each is scored with the loss of
+    ``mode`` at the scale of its code (``multiplier_codes``); the first multiplier with the
+    smallest loss wins (strict <). Returns codes, wq, loss, index (winning multiplier),
+    second (the best loss among candidates with another code; +inf if none), e0, escale.
+    """
+    w = np.asarray(w_blk, dtype=np.float32)
+    codes = multiplier_codes(w, g, multipliers)
+    v = np.where(codes > 0, e4m3_value(np.maximum(codes, 1)), 0.0)
+    s = (v * np.float64(np.float32(g))).astype(np.float32)
+    loss, wq = losses_for_scales(mode, w, h_blk, p_blk, s)
+    idx, best, _ = argmin_lowest(loss)
+    u = np.arange(len(idx))
+    bc = codes[u, idx]
+    other = np.where(codes != bc[:, None], loss, np.inf)
+    w64 = w.astype(np.float64)  # E0: the q = 0 loss without the cross term
+    if mode == "mse":
+        e0 = np.einsum("ui,ui->u", w64, w64)
+    elif mode == "diag":
+        e0 = np.einsum("ui,ui->u", w64 * w64, np.asarray(h_blk, dtype=np.float64))
+    else:
+        e0 = np.einsum("ui,uij,uj->u", w64, np.asarray(h_blk, dtype=np.float64), w64)
+    return {
+        "codes": bc.astype(np.uint8),
+        "wq": wq[u, idx],
+        "loss": best,
+        "index": idx,
+        "second": other.min(axis=1),
+        "e0": e0,
+        "escale": loss_scale(mode, w, h_blk, p_blk),
+        "all_codes": codes,
+    }
+
+
+def multiplier_search(mode: str, w, h, p, g, multipliers, units=None):
+    """``multiplier_search_units`` over the given units (default: all) of a layer."""
+    w = np.asarray(w, dtype=np.float32)
+    gcount, rows, cin = w.shape
+    if units is None:
+        ge, r, n = np.meshgrid(np.arange(gcount), np.arange(rows), np.arange(cin // BLOCK), indexing="ij")
+        units = np.stack([ge.ravel(), r.ravel(), n.ravel()], axis=1)
+    units = np.asarray(units, dtype=np.int64)
+    wb, hb, pb, gu = gather_units(mode, w, h, p, g, units)
+    keys = ("codes", "wq", "loss", "index", "second", "e0", "escale")
+    res = {k: np.empty((len(units),) + ((BLOCK,) if k == "wq" else ()),
+                       dtype={"codes": np.uint8, "wq": np.float32, "index": np.int64}.get(k, np.float64))
+           for k in keys}
+    for gv in np.unique(gu):  # units of one group share g
+        sel = np.nonzero(gu == gv)[0]
+        o = multiplier_search_units(mode, wb[sel], None if hb is None else hb[sel],
+                                    None if pb is None else pb[sel], gv, multipliers)
+        for k in keys:
+            res[k][sel] = o[k]
+    return res
+
+
 def apply_scales(w, g, codes):
     """Fake-quantized weights and per-block amax for chosen block-scale codes.
 

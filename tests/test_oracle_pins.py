@@ -431,3 +431,67 @@ def test_loss_scale_bounds_e0_and_equals_it_for_diagonal_h():
     np.testing.assert_allclose(O.loss_scale("full", w, hd, None), e0d, rtol=1e-13)
     imp = hd[:, idx, idx]
     np.testing.assert_allclose(O.loss_scale("diag", w, imp, None), e0d, rtol=1e-13)
+
+
+# --------------------------------------------------------------------------- amax-multiplier search
+
+@pytest.mark.parametrize("mode", ["full", "act", "diag", "mse"])
+def test_losses_for_scales_is_candidate_losses_at_the_candidate_scales(mode):
+    rng = np.random.default_rng(21)
+    w = rng.normal(0, 0.05, (9, 16)).astype(np.float32)
+    a = rng.normal(size=(9, 16, 16))
+    h = a @ a.transpose(0, 2, 1) / 16 if mode in ("full", "act") else (np.abs(rng.normal(size=(9, 16))) + 0.5)
+    p = 0.05 * rng.normal(size=(9, 16, 16)) if mode == "act" else None
+    g = O.global_scale(w)
+    ref, wq_ref, _ = O.candidate_losses(mode, w, None if mode == "mse" else h, p, g)
+    s = np.broadcast_to(O.candidate_scales(g), (9, 126))
+    got, wq = O.losses_for_scales(mode, w, None if mode == "mse" else h, p, s)
+    np.testing.assert_array_equal(got, ref)
+    np.testing.assert_array_equal(wq.view(np.int32), wq_ref.view(np.int32))
+
+
+def test_multiplier_codes_by_exact_rationals():
+    rng = np.random.default_rng(22)
+    w = (rng.normal(0, 0.05, (6, 16)) * np.exp(rng.normal(0, 2, (6, 1)))).astype(np.float32)
+    w[5] = 0.0
+    g = np.float32(O.global_scale(w) * 0.7)
+    m = np.concatenate([np.linspace(0.05, 3.0, 40), [0.0, -1.0, np.nan, 1e30]]).astype(np.float32)
+    codes = O.multiplier_codes(w, g, m)
+    gq = Fraction(float(g))
+    for u in range(6):
+        amax = max(abs(Fraction(float(v))) for v in w[u])
+        for i, mi in enumerate(m):
+            if not np.isfinite(mi):
+                want = 0
+            else:
+                a = _round_binary(abs(Fraction(float(mi)) * amax), 24, -126) * (1 if mi >= 0 else -1)
+                if a > Fraction(float(np.finfo(np.float32).max)):
+                    want = 126  # the fp32 product overflows to +inf
+                else:
+                    want = 0 if a <= 0 else _e4m3_code_brute(a / (6 * gq))
+            assert codes[u, i] == want, (u, i, float(mi))
+    assert np.all(O.multiplier_codes(w, np.float32(0.0), m) == 0)
+
+
+@pytest.mark.parametrize("mode", ["full", "diag", "mse"])
+def test_dense_multipliers_reproduce_the_sweep(mode):
+    """Multipliers so dense that every code 1..126 is some multiplier's code: the search then
+    scores every sweep candidate, in ascending code order, so it finds the sweep's winner."""
+    _, w = _layer(23, rows=5, cin=32)
+    g = np.array([O.global_scale(w[0])], np.float32)
+    h = None
+    if mode == "full":
+        a = np.random.default_rng(3).normal(size=(2, 16, 16))
+        h = (a @ a.transpose(0, 2, 1))[None] / 16
+    elif mode == "diag":
+        h = np.abs(np.random.default_rng(3).normal(size=(1, 2, 16))) + 0.5
+    mult = np.exp(np.linspace(np.log(1e-7), np.log(1e4), 9000)).astype(np.float32)
+    ms = O.multiplier_search(mode, w, h, None, g, mult)
+    sw = O.sweep(mode, w, h, None, g)
+    wb = w[0].reshape(10, 16)
+    cover = np.array([set(range(1, 127)) <= set(O.multiplier_codes(wb[u:u + 1], g[0], mult)[0].tolist())
+                      for u in range(10)])
+    assert cover.all()
+    np.testing.assert_array_equal(ms["codes"], sw["codes"])
+    np.testing.assert_array_equal(ms["wq"].view(np.int32), sw["wq"].view(np.int32))
+    np.testing.assert_array_equal(ms["loss"], sw["loss"])
