@@ -66,6 +66,8 @@ typedef enum {
 /* Number of 126 candidate block scales (E4M3 codes 0x01..0x7E), PR #2283 "How". */
 #define LHCAL_N_CANDIDATES 126
 #define LHCAL_BLOCK 16
+/* Most multipliers lhcal_multiplier_search takes. */
+#define LHCAL_MAX_MULTIPLIERS 1024
 
 /*
  * Bytes of workspace lhcal_accumulate needs for these sizes (0 is possible). Host-only
@@ -201,6 +203,28 @@ lhcal_status lhcal_global_scale_ex(lhcal_dtype dtype, const void* w, int32_t gro
 lhcal_status lhcal_scale_sweep(lhcal_mode mode, lhcal_dtype dtype, const void* w, int32_t groups,
                                int64_t rows, int64_t cin, const float* h, const float* p,
                                const float* g, uint8_t* codes, float* wq, float* loss, void* stream);
+
+/*
+ * Amax-multiplier search: the block-scale search without the FP8 sweep that "add local hessian
+ * calibration" (PR #788, Changes table: configurable step size and multipliers) runs with the
+ * same Hessian-weighted losses. For each unit (e, r, n), amax_blk = max |w| of its 16 weights,
+ * and for each multiplier m_i in the given order:
+ *   a_i = fp32(m_i * amax_blk) (a negative or NaN value counts as 0);
+ *   c_i = the E4M3 code nearest to a_i / (6 * g[e]) on the exact quotient (ties to the even code,
+ *         saturating at 448; 0 is a zero scale; g[e] == 0 gives 0): the NVFP4 block scale
+ *         the quantizer derives from that amax;
+ *   L_i = the loss of lhcal_scale_sweep's mode at s = fp32(v_{c_i} * g[e]).
+ * The first multiplier with the smallest L_i wins. Outputs as for lhcal_scale_sweep: codes (the
+ * winner's c, which may be 0), wq (or NULL), loss (or NULL).
+ *   mode        : LHCAL_FULL, LHCAL_ACT_AWARE, LHCAL_DIAG or LHCAL_MSE (h = p = NULL).
+ *   multipliers : device fp32 [n_multipliers], 1 <= n_multipliers <= LHCAL_MAX_MULTIPLIERS;
+ *                 finite and >= 0 (for example start + i * step).
+ *   other arguments as for lhcal_scale_sweep.
+ */
+lhcal_status lhcal_multiplier_search(lhcal_mode mode, lhcal_dtype dtype, const void* w, int32_t groups,
+                                     int64_t rows, int64_t cin, const float* h, const float* p, const float* g,
+                                     const float* multipliers, int32_t n_multipliers, uint8_t* codes, float* wq,
+                                     float* loss, void* stream);
 
 /*
  * Outputs for chosen block-scale codes (for example the codes lhcal_scale_sweep wrote): for each

@@ -54,6 +54,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lhcal_finalize": [i32, i32, i64, vp, vp, vp, vp],
         "lhcal_global_scale": [i32, vp, i32, i64, i64, vp, vp],
         "lhcal_global_scale_ex": [i32, vp, i32, i64, i64, ctypes.c_float, vp, vp],
+        "lhcal_multiplier_search": [i32, i32, vp, i32, i64, i64, vp, vp, vp, vp, i32, vp, vp, vp, vp],
         "lhcal_apply_scales": [i32, vp, i32, i64, i64, vp, vp, vp, vp, vp, vp],
         "lhcal_scale_sweep": [i32, i32, vp, i32, i64, i64, vp, vp, vp, vp, vp, vp, vp],
     }
@@ -210,6 +211,14 @@ def lhcal_global_scale(w, g, stream=None, fp8_max: float | None = None):
     else:
         _check(load_library().lhcal_global_scale_ex(_dtype_id(w), _ptr(w), groups, rows, cin, float(fp8_max),
                                                     _ptr(g), _stream(stream)))
+
+
+def lhcal_multiplier_search(mode, w, h, g, multipliers, codes, wq=None, loss=None, p=None, stream=None):
+    """Amax-multiplier search: multipliers fp32 device [M]; other tensors as lhcal_scale_sweep."""
+    groups, rows, cin = (int(v) for v in w.shape)
+    _check(load_library().lhcal_multiplier_search(
+        _mode_id(mode), _dtype_id(w), _ptr(w), groups, rows, cin, _ptr(h), _ptr(p), _ptr(g), _ptr(multipliers),
+        int(multipliers.numel()), _ptr(codes), _ptr(wq), _ptr(loss), _stream(stream)))
 
 
 def lhcal_apply_scales(w, g, codes, wq=None, wq16=None, amax=None, stream=None):

@@ -21,7 +21,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "liblhcal.so")
-SOURCES = ["lhcal_api.cu", "sweep.cu", "sweep_tc.cu", "accum.cu", "act_quant.cu", "misc.cu", "noalloc.cu"]
+SOURCES = ["lhcal_api.cu", "sweep.cu", "sweep_tc.cu", "accum.cu", "act_quant.cu", "misc.cu", "msearch.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

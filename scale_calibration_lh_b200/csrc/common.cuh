@@ -16,6 +16,7 @@ namespace lhcal {
 // queried at run time) so that results and workspace sizes are reproducible.
 constexpr int kNumSms = 148;
 constexpr int kBlock = LHCAL_BLOCK;
+constexpr int kMaxMultipliers = LHCAL_MAX_MULTIPLIERS;
 
 // Thread-local last-error message (lhcal_last_error_string).
 void set_error(const char* fmt, ...);
@@ -97,6 +98,10 @@ lhcal_status launch_finalize(lhcal_mode mode, int32_t groups, int64_t cin, const
 
 lhcal_status launch_global_scale(lhcal_dtype dtype, const void* w, int32_t groups, int64_t rows,
                                  int64_t cin, float* g, cudaStream_t stream, float fp8_max = 448.f);
+
+lhcal_status launch_multiplier_search(lhcal_mode mode, lhcal_dtype dtype, const void* w, int32_t groups, int64_t rows,
+                                      int64_t cin, const float* h, const float* p, const float* g, const float* mult,
+                                      int32_t n_mult, uint8_t* codes, float* wq, float* loss, cudaStream_t stream);
 
 lhcal_status launch_apply_scales(lhcal_dtype dtype, const void* w, int32_t groups, int64_t rows, int64_t cin,
                                  const float* g, const uint8_t* codes, float* wq, void* wq16, float* amax,

@@ -284,6 +284,34 @@ lhcal_status lhcal_apply_scales(lhcal_dtype dtype, const void* w, int32_t groups
   return launch_apply_scales(dtype, w, groups, rows, cin, g, codes, wq, wq16, amax, static_cast<cudaStream_t>(stream));
 }
 
+lhcal_status lhcal_multiplier_search(lhcal_mode mode, lhcal_dtype dtype, const void* w, int32_t groups,
+                                     int64_t rows, int64_t cin, const float* h, const float* p, const float* g,
+                                     const float* multipliers, int32_t n_multipliers, uint8_t* codes, float* wq,
+                                     float* loss, void* stream) {
+  clear_error();
+  if (!valid_sweep_mode(mode) || !valid_dtype(dtype)) return fail(LHCAL_ERR_UNSUPPORTED, "unknown mode or dtype");
+  LHCAL_TRY(check_cin(cin));
+  LHCAL_TRY(check_groups(groups));
+  if (rows <= 0 || rows > (int64_t)INT32_MAX * 64)
+    return fail(LHCAL_ERR_INVALID_ARG, "rows (%lld) out of range", (long long)rows);
+  if (n_multipliers < 1 || n_multipliers > LHCAL_MAX_MULTIPLIERS)
+    return fail(LHCAL_ERR_INVALID_ARG, "n_multipliers (%d) must be in [1, %d]", n_multipliers, LHCAL_MAX_MULTIPLIERS);
+  if (mode == LHCAL_MSE && (h != nullptr || p != nullptr)) return fail(LHCAL_ERR_INVALID_ARG, "MSE takes no h or p");
+  if (mode == LHCAL_ACT_AWARE && p == nullptr) return fail(LHCAL_ERR_INVALID_ARG, "ACT_AWARE needs p");
+  if (mode != LHCAL_ACT_AWARE && p != nullptr) return fail(LHCAL_ERR_INVALID_ARG, "p is only for ACT_AWARE");
+  LHCAL_TRY(check_device_ptr(w, 16, "w"));
+  if (mode != LHCAL_MSE) LHCAL_TRY(check_device_ptr(h, 16, "h"));
+  if (mode == LHCAL_ACT_AWARE) LHCAL_TRY(check_device_ptr(p, 16, "p"));
+  LHCAL_TRY(check_device_ptr(g, 4, "g"));
+  LHCAL_TRY(check_device_ptr(multipliers, 4, "multipliers"));
+  LHCAL_TRY(check_device_ptr(codes, 1, "codes"));
+  if (wq != nullptr) LHCAL_TRY(check_device_ptr(wq, 16, "wq"));
+  if (loss != nullptr) LHCAL_TRY(check_device_ptr(loss, 4, "loss"));
+  if (ceil_div(rows, 128) > 0x7fffffff) return fail(LHCAL_ERR_INVALID_ARG, "rows too large");
+  return launch_multiplier_search(mode, dtype, w, groups, rows, cin, h, p, g, multipliers, n_multipliers, codes, wq,
+                                  loss, static_cast<cudaStream_t>(stream));
+}
+
 lhcal_status lhcal_scale_sweep(lhcal_mode mode, lhcal_dtype dtype, const void* w, int32_t groups, int64_t rows,
                                int64_t cin, const float* h, const float* p, const float* g, uint8_t* codes,
                                float* wq, float* loss, void* stream) {

@@ -131,3 +131,13 @@ def test_mse_scale_and_output_entry_points_validate_without_gpu(lib):
     assert ap(1, None, 1, 4, 33, None, None, None, None, None, None) == L.ERR_INVALID_ARG
     assert ap(1, None, 1, 0, 32, None, None, None, None, None, None) == L.ERR_INVALID_ARG
     assert ap(5, None, 1, 4, 32, None, None, None, None, None, None) == L.ERR_UNSUPPORTED
+
+
+def test_multiplier_search_validates_without_gpu(lib):
+    f = lib.lhcal_multiplier_search
+    assert f(9, 1, None, 1, 4, 32, None, None, None, None, 8, None, None, None, None) == L.ERR_UNSUPPORTED
+    assert f(0, 1, None, 1, 4, 33, None, None, None, None, 8, None, None, None, None) == L.ERR_INVALID_ARG
+    assert f(0, 1, None, 1, 4, 32, None, None, None, None, 0, None, None, None, None) == L.ERR_INVALID_ARG
+    assert f(0, 1, None, 1, 4, 32, None, None, None, None, 2000, None, None, None, None) == L.ERR_INVALID_ARG
+    assert b"n_multipliers" in lib.lhcal_last_error_string()
+    assert f(1, 1, None, 1, 4, 32, None, None, None, None, 8, None, None, None, None) == L.ERR_INVALID_ARG  # no p

@@ -599,3 +599,61 @@ def test_apply_scales_bit_exact(name, kw):
     L.lhcal_apply_scales(d["w"], b.g, b.codes, wq=wq)
     _sync()
     assert torch.equal(wq.view(torch.int32), b.wq.view(torch.int32))
+
+
+# ----------------------------------------------------------------------------- amax-multiplier search
+
+@pytest.mark.parametrize("mode,name,kw", [
+    ("full", "dense", dict(tokens=500, cin=96, rows=150)),
+    ("act", "act", dict(tokens=400, cin=64, rows=130)),
+    ("diag", "wmse", dict(tokens=300, cin=80, rows=140)),
+    ("mse", "dense", dict(tokens=16, cin=48, rows=200)),
+    ("full", "tiny", dict()),
+    ("full", "moe", dict(tokens=60, cin=64, rows=40, groups=5, top_k=2)),
+])
+def test_multiplier_search(mode, name, kw):
+    """Both sides get the oracle's finalized H (and P) rounded to fp32, the same global scales
+    and multipliers 0.5, 0.55, ..., 2.0 (plus 0 and one that reaches the 448 saturation)."""
+    layer = P.make_layer(name, 51, **kw)
+    G, R, C = layer.groups, layer.rows, layer.cin
+    w32 = layer.w_f32()
+    g = np.array([O.global_scale(w32[e]) for e in range(G)], np.float32)
+    h = p = None
+    if mode != "mse":
+        xq = layer.xq_f32() if mode == "act" else None
+        hs, ps, counts = O.accumulate(mode, layer.x_f32(), xq, layer.group_offsets, layer.token_ids)
+        h, p = O.finalize(mode, hs, ps, counts)
+        h = h.astype(np.float32).astype(np.float64)
+        p = None if p is None else p.astype(np.float32).astype(np.float64)
+    mult = np.concatenate([np.arange(0.5, 2.0001, 0.05), [0.0, 5000.0]]).astype(np.float32)
+    d = P.layer_to_device(layer)
+    codes = torch.empty((G, R, C // 16), dtype=torch.uint8, device="cuda")
+    wq = torch.empty((G, R, C), dtype=torch.float32, device="cuda")
+    loss = torch.empty((G, R, C // 16), dtype=torch.float32, device="cuda")
+    L.lhcal_multiplier_search(mode, d["w"], None if h is None else P.to_device(h, "f32"), P.to_device(g, "f32"),
+                              P.to_device(mult, "f32"), codes, wq=wq, loss=loss,
+                              p=None if p is None else P.to_device(p, "f32"))
+    _sync()
+    units = P.all_units(G, R, C // 16)
+    ref = O.multiplier_search(mode, w32, h, p, g, mult, units)
+    gc, gw, gl = P.gather_gpu_units(codes, wq, loss, units)
+    rep = P.check_sweep(gc, gw, gl, ref, f"{name} {mode} multiplier search")
+    assert rep["units"] == len(units)
+    # Optional outputs: codes alone give the same codes.
+    codes2 = torch.empty_like(codes)
+    L.lhcal_multiplier_search(mode, d["w"], None if h is None else P.to_device(h, "f32"), P.to_device(g, "f32"),
+                              P.to_device(mult, "f32"), codes2, p=None if p is None else P.to_device(p, "f32"))
+    _sync()
+    assert torch.equal(codes, codes2)
+
+
+def test_multiplier_search_rejects_bad_counts():
+    w = torch.zeros((1, 4, 32), dtype=torch.bfloat16, device="cuda")
+    g = torch.ones(1, device="cuda")
+    codes = torch.empty((1, 4, 2), dtype=torch.uint8, device="cuda")
+    for n in (0, 1025):
+        m = torch.ones(max(n, 1), device="cuda")
+        lib = L.load_library()
+        st = lib.lhcal_multiplier_search(3, 1, L._ptr(w), 1, 4, 32, None, None, L._ptr(g), L._ptr(m), n,
+                                         L._ptr(codes), None, None, None)
+        assert st == L.ERR_INVALID_ARG
