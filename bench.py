@@ -355,7 +355,9 @@ def run_lhcal(args, rank, world, local_rank):
         hxq.copy_(d["xq"])
     hw = torch.empty(d["w"].shape, dtype=d["w"].dtype, pin_memory=True)
     hw.copy_(d["w"])
-    out_host = L.HostOutputs(buf)
+    # The step's result read back: the codes (the chosen scales) and the winning losses; the
+    # fake-quantized weights stay on the device (lhcal_apply_scales derives them from the codes).
+    out_host = L.HostOutputs(buf, want_wq=False)
     hoffs = None if d["offs"] is None else d["offs"].cpu().pin_memory()
     hids = None if d["ids"] is None else d["ids"].cpu().pin_memory()
     K2 = max(3, min(K, 10))

@@ -272,38 +272,36 @@ def calibrate(mode, x, w, xq=None, group_offsets=None, token_ids=None, buffers: 
     scale from which the kernel derives X_q; CSR routing for grouped layers) are device
     tensors. Returns the buffers holding h, p, g, codes, wq and loss.
     """
+    if stream is not None:  # enqueue everything on the given stream
+        import torch
+
+        with torch.cuda.stream(stream):
+            return calibrate(mode, x, w, xq, group_offsets, token_ids, buffers, None, act_gx)
     m = _mode_id(mode)
     groups, rows, cin = (int(v) for v in w.shape)
     if m == MSE:  # plain block MSE: no statistics, x is not read
         b = buffers or Buffers(m, 0, cin, rows, groups, _dtype_id(w), w.device)
-        lhcal_global_scale(w, b.g, stream=stream)
-        lhcal_scale_sweep(m, w, None, b.g, b.codes, wq=b.wq, loss=b.loss, stream=stream)
+        _scales_and_sweep(m, w, b, 0, groups)
         return b
     if buffers is None:
         buffers = Buffers(m, int(x.shape[0]), cin, rows, groups, _dtype_id(x), x.device)
     b = buffers
-    if m == ACT_AWARE and xq is None and act_gx is not None:
-        lhcal_accumulate_act_quant(x, b.h, b.p, act_gx, group_offsets=group_offsets, token_ids=token_ids,
-                                   flags=ACCUM_OVERWRITE, workspace=b.workspace, stream=stream)
-    else:
-        lhcal_accumulate(m, x, b.h, xq=xq, p=b.p, group_offsets=group_offsets, token_ids=token_ids,
-                         flags=ACCUM_OVERWRITE, workspace=b.workspace, stream=stream)
-    lhcal_count_tokens(b.counts, tokens=int(x.shape[0]), group_offsets=group_offsets, flags=ACCUM_OVERWRITE,
-                       stream=stream)
-    lhcal_finalize(m, b.counts, b.h, p=b.p, stream=stream)
-    lhcal_global_scale(w, b.g, stream=stream)
-    lhcal_scale_sweep(m, w, b.h, b.g, b.codes, wq=b.wq, loss=b.loss, p=b.p, stream=stream)
+    _statistics(m, x, b, xq=xq, group_offsets=group_offsets, token_ids=token_ids, act_gx=act_gx)
+    _scales_and_sweep(m, w, b, 0, groups)
     return b
 
 
 class HostOutputs:
-    """Pinned host copies of a calibration's results: codes, fake-quantized weights, losses."""
+    """Pinned host copies of a calibration's results: the codes (the chosen block scales) and the
+    winning losses, and the fake-quantized weights when ``want_wq`` (they follow from the codes
+    through lhcal_apply_scales, so a caller may leave them on the device)."""
 
-    def __init__(self, buffers: Buffers):
+    def __init__(self, buffers: Buffers, want_wq: bool = True):
         import torch
 
         self.codes = torch.empty(buffers.codes.shape, dtype=torch.uint8, pin_memory=True)
-        self.wq = None if buffers.wq is None else torch.empty(buffers.wq.shape, dtype=torch.float32, pin_memory=True)
+        self.wq = (torch.empty(buffers.wq.shape, dtype=torch.float32, pin_memory=True)
+                   if want_wq and buffers.wq is not None else None)
         self.loss = None if buffers.loss is None else torch.empty(buffers.loss.shape, dtype=torch.float32,
                                                                    pin_memory=True)
 
@@ -311,31 +309,99 @@ class HostOutputs:
         return sum(t.numel() * t.element_size() for t in (self.codes, self.wq, self.loss) if t is not None)
 
 
+_side_streams: dict = {}
+
+
+def _side_stream(device, which: str):
+    import torch
+
+    key = (str(device), which)
+    if key not in _side_streams:
+        _side_streams[key] = torch.cuda.Stream(device=device)
+    return _side_streams[key]
+
+
+def _statistics(m, x, buffers, xq=None, group_offsets=None, token_ids=None, act_gx=None):
+    """Accumulate, count and finalize on the current stream (nothing for MSE)."""
+    b = buffers
+    if m == MSE:
+        return
+    if m == ACT_AWARE and xq is None and act_gx is not None:
+        lhcal_accumulate_act_quant(x, b.h, b.p, act_gx, group_offsets=group_offsets, token_ids=token_ids,
+                                   flags=ACCUM_OVERWRITE, workspace=b.workspace)
+    else:
+        lhcal_accumulate(m, x, b.h, xq=xq, p=b.p, group_offsets=group_offsets, token_ids=token_ids,
+                         flags=ACCUM_OVERWRITE, workspace=b.workspace)
+    lhcal_count_tokens(b.counts, tokens=int(x.shape[0]), group_offsets=group_offsets, flags=ACCUM_OVERWRITE)
+    lhcal_finalize(m, b.counts, b.h, p=b.p)
+
+
+def _scales_and_sweep(m, w, buffers, e0: int, e1: int):
+    """Global scales and sweep of groups [e0, e1) on the current stream."""
+    b = buffers
+    sl = slice(e0, e1)
+    lhcal_global_scale(w[sl], b.g[sl])
+    lhcal_scale_sweep(m, w[sl], None if b.h is None else b.h[sl], b.g[sl], b.codes[sl],
+                      wq=None if b.wq is None else b.wq[sl], loss=None if b.loss is None else b.loss[sl],
+                      p=None if b.p is None else b.p[sl])
+
+
 def calibrate_host(mode, x, w, buffers: Buffers, staging: dict, hxq=None, group_offsets=None, token_ids=None,
-                   out: HostOutputs | None = None, stream=None, act_gx=None) -> HostOutputs:
-    """The whole hot path from host tensors (pinned for asynchronous copies) to host results.
+                   out: HostOutputs | None = None, act_gx=None, group_chunks: int = 8) -> HostOutputs:
+    """The whole hot path from host tensors (pinned, for asynchronous copies) to host results.
 
     ``staging`` holds device tensors shaped like the inputs under keys "x", "w" and, when
-    used, "xq", "offs", "ids". Inputs are copied host to device on the current stream, the
-    layer is calibrated, and codes / wq / loss are copied back into ``out``. Returns ``out``
-    without synchronising.
+    used, "xq", "offs", "ids". Activations (and routing) are copied in and the statistics
+    computed on the current stream. A grouped layer (groups > 1) is then pipelined over
+    ``group_chunks`` chunks of groups: each chunk's weights are copied in on a side stream while
+    the current stream computes global scales and sweeps the chunks already resident, and each
+    chunk's results are copied out on another side stream as soon as they are ready. A layer
+    with one group copies its weights, computes the scale and sweeps. The results land in
+    ``out`` (codes, loss, and wq if requested); the function returns without synchronising,
+    and the current stream waits for every copy it issued.
     """
+    import torch
+
+    m = _mode_id(mode)
     if out is None:
         out = HostOutputs(buffers)
-    staging["x"].copy_(x, non_blocking=True)
-    staging["w"].copy_(w, non_blocking=True)
-    if hxq is not None:
-        staging["xq"].copy_(hxq, non_blocking=True)
-    if group_offsets is not None:
-        staging["offs"].copy_(group_offsets, non_blocking=True)
-        staging["ids"].copy_(token_ids, non_blocking=True)
-    calibrate(mode, staging["x"], staging["w"], xq=staging.get("xq"), group_offsets=staging.get("offs"),
-              token_ids=staging.get("ids"), buffers=buffers, stream=stream, act_gx=act_gx)
-    out.codes.copy_(buffers.codes, non_blocking=True)
-    if out.wq is not None:
-        out.wq.copy_(buffers.wq, non_blocking=True)
-    if out.loss is not None:
-        out.loss.copy_(buffers.loss, non_blocking=True)
+    cur = torch.cuda.current_stream()
+    if m != MSE:
+        staging["x"].copy_(x, non_blocking=True)
+        if hxq is not None:
+            staging["xq"].copy_(hxq, non_blocking=True)
+        if group_offsets is not None:
+            staging["offs"].copy_(group_offsets, non_blocking=True)
+            staging["ids"].copy_(token_ids, non_blocking=True)
+        # X_q is read only when the caller copies it in; otherwise (act_gx) the kernel derives it.
+        _statistics(m, staging["x"], buffers, xq=staging["xq"] if hxq is not None else None,
+                    group_offsets=staging.get("offs") if group_offsets is not None else None,
+                    token_ids=staging.get("ids") if token_ids is not None else None, act_gx=act_gx)
+    groups = int(w.shape[0])
+    n = max(1, min(group_chunks, groups))
+    bounds = [groups * j // n for j in range(n + 1)]
+    dev = staging["w"].device
+    s_in, s_out = _side_stream(dev, "in"), _side_stream(dev, "out")
+    s_in.wait_stream(cur)
+    s_out.wait_stream(cur)
+    for e0, e1 in zip(bounds[:-1], bounds[1:]):
+        with torch.cuda.stream(s_in):
+            staging["w"][e0:e1].copy_(w[e0:e1], non_blocking=True)
+            ready = torch.cuda.Event()
+            ready.record(s_in)
+        cur.wait_event(ready)
+        _scales_and_sweep(m, staging["w"], buffers, e0, e1)
+        done = torch.cuda.Event()
+        done.record(cur)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(done)
+            out.codes[e0:e1].copy_(buffers.codes[e0:e1], non_blocking=True)
+            if out.loss is not None:
+                out.loss[e0:e1].copy_(buffers.loss[e0:e1], non_blocking=True)
+            if out.wq is not None:
+                out.wq[e0:e1].copy_(buffers.wq[e0:e1], non_blocking=True)
+    cur.wait_stream(s_in)
+    cur.wait_stream(s_out)
     return out
 
 

@@ -657,3 +657,41 @@ def test_multiplier_search_rejects_bad_counts():
         st = lib.lhcal_multiplier_search(3, 1, L._ptr(w), 1, 4, 32, None, None, L._ptr(g), L._ptr(m), n,
                                          L._ptr(codes), None, None, None)
         assert st == L.ERR_INVALID_ARG
+
+
+# ----------------------------------------------------------------------------- host path
+
+@pytest.mark.parametrize("name,kw,chunks", [
+    ("dense", dict(tokens=500, cin=128, rows=64), 8),
+    ("moe", dict(tokens=300, cin=96, rows=24, groups=20, top_k=3), 8),
+    ("moe", dict(tokens=300, cin=96, rows=24, groups=20, top_k=3), 3),
+    ("act", dict(tokens=300, cin=64, rows=40), 8),
+    ("mse", dict(), 1),
+])
+def test_calibrate_host_matches_the_device_path(name, kw, chunks):
+    """calibrate_host (pinned host inputs, grouped layers pipelined over chunks of groups on side
+    streams) returns exactly the codes, losses and fake-quantized weights of calibrate."""
+    mse = name == "mse"
+    layer = P.make_layer("dense" if mse else name, 61, **(dict(tokens=16, cin=64, rows=48) if mse else kw))
+    mode = "mse" if mse else layer.mode
+    d = P.layer_to_device(layer)
+    fused = mode == "act"
+    ref = L.calibrate(mode, d["x"], d["w"], group_offsets=d["offs"], token_ids=d["ids"],
+                      act_gx=d["act_gx"] if fused else None, xq=None)
+    _sync()
+    want = (ref.codes.cpu(), ref.loss.cpu(), ref.wq.cpu())
+    staging = {k: (torch.empty_like(v) if isinstance(v, torch.Tensor) else None) for k, v in d.items()}
+    pin = lambda t: None if t is None else t.cpu().pin_memory()  # noqa: E731
+    buf = L.Buffers(mode, layer.tokens, layer.cin, layer.rows, layer.groups, L.BF16 if layer.dtype == "bf16" else L.F32,
+                    "cuda")
+    out = L.calibrate_host(mode, pin(d["x"]), pin(d["w"]), buf, staging, group_offsets=pin(d["offs"]),
+                           token_ids=pin(d["ids"]), act_gx=d["act_gx"] if fused else None, group_chunks=chunks)
+    torch.cuda.current_stream().synchronize()
+    assert torch.equal(out.codes, want[0])
+    assert torch.equal(out.loss.view(torch.int32), want[1].view(torch.int32))
+    assert torch.equal(out.wq.view(torch.int32), want[2].view(torch.int32))
+    out2 = L.calibrate_host(mode, pin(d["x"]), pin(d["w"]), buf, staging, group_offsets=pin(d["offs"]),
+                            token_ids=pin(d["ids"]), act_gx=d["act_gx"] if fused else None,
+                            out=L.HostOutputs(buf, want_wq=False), group_chunks=chunks)
+    torch.cuda.current_stream().synchronize()
+    assert out2.wq is None and torch.equal(out2.codes, want[0])
