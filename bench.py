@@ -48,7 +48,6 @@ WORKLOAD_TEXT = {
 # dram__bytes_read.sum + dram__bytes_write.sum per launch, from one ncu capture of the current
 # kernel on this workload (summaries in profiles/); workloads without a capture report null.
 SWEEP_TRAFFIC_BYTES = {
-    "dense": 33_871_360 + 143_094_272,   # sweep_tc_kernel, profiles/sweep_tc_kernel_dense.md
     "wmse": 101_576_704 + 166_720_000,   # sweep_diag_kernel, profiles/sweep_diag_kernel_wmse.md
 }
 ACCUM_TRAFFIC_BYTES = {

@@ -301,7 +301,8 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
   // One candidate: A fragment from the elements' packed fp16 grid values; the accumulator starts
   // at rho_k U', so after the 4 MMAs D = v^T H' + rho_k U' and
   //   L = s2_k * sum_n v_n D_n + C' = s^2 v^T H v - 2 s v^T U' + C'.
-  auto evaluate = [&](const uint32_t (&q)[8], int k) {
+  // The lane's share of t for units 0 and 1 (its 4 columns), before the reduction over the quad.
+  auto partials = [&](const uint32_t (&q)[8], int k, float (&tp)[2]) {
     uint32_t afr[4];
 #pragma unroll
     for (int r = 0; r < 4; ++r) afr[r] = (q[kPairLo[r]] | q[kPairLo[r] + 1]) ^ smask[r];
@@ -319,7 +320,13 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
     const float2 v23 = unpack_f16x2(afr[2]), v67 = unpack_f16x2(afr[3]);
     const float2 p0 = __ffma2_rn(v23, make_float2(d1[0], d1[1]), __fmul2_rn(v01, make_float2(d0[0], d0[1])));
     const float2 p1 = __ffma2_rn(v67, make_float2(d1[2], d1[3]), __fmul2_rn(v45, make_float2(d0[2], d0[3])));
-    float t0 = p0.x + p0.y, t1 = p1.x + p1.y;
+    tp[0] = p0.x + p0.y;
+    tp[1] = p1.x + p1.y;
+  };
+  auto evaluate = [&](const uint32_t (&q)[8], int k) {
+    float tp[2];
+    partials(q, k, tp);
+    float t0 = tp[0], t1 = tp[1];
     t0 += __shfl_xor_sync(0xffffffffu, t0, 1);
     t1 += __shfl_xor_sync(0xffffffffu, t1, 1);
     t0 += __shfl_xor_sync(0xffffffffu, t0, 2);
@@ -350,9 +357,9 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
     }
   }
   // From kstart: levels by counting thresholds until the 4th candidate and until the rest is a
-  // multiple of three, then by single-step drops (consecutive scales differ by at most 4/3).
+  // multiple of four, then by single-step drops (consecutive scales differ by at most 4/3).
   int kinc = max(kstart + 1, 3);
-  kinc += (kCand - kinc) % 3;
+  kinc += (kCand - kinc) % 4;
   const uint32_t tab_base = smem_u32(sh.tab);
   uint32_t addr[8];  // shared address of the table entry (k, level) of each element
 #pragma unroll 1
@@ -367,32 +374,77 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
     }
     evaluate(q, k);
   }
+  // Four candidates at a time. A transposed reduction over the quad leaves lane tq with the
+  // full sums of candidate k + tq (the same additions as the per-candidate reduction, so the
+  // same values): after each pair of candidates the lanes tq and tq ^ 1 swap halves (lane tq
+  // keeps the pair's candidate with index bit tq & 1), and after the second pair lanes tq and
+  // tq ^ 2 finish. Each lane tracks the best of its own candidates; the quad merges them after
+  // the loop.
+  const bool b0 = (tq & 1) != 0, b1 = (tq & 2) != 0;
 #pragma unroll 1
-  for (int k = kinc; k < kCand; k += 3) {
+  for (int k = kinc; k < kCand; k += 4) {
+    float hold[2], spair[2][2];
 #pragma unroll
-    for (int u = 0; u < 3; ++u) {
+    for (int c = 0; c < 4; ++c) {
       uint32_t q[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         float t;
-        if (u == 0) t = lds_f32<kTabRowBytes>(addr[i]);
-        else if (u == 1) t = lds_f32<2 * kTabRowBytes>(addr[i]);
-        else t = lds_f32<3 * kTabRowBytes>(addr[i]);
+        if (c == 0) t = lds_f32<kTabRowBytes>(addr[i]);
+        else if (c == 1) t = lds_f32<2 * kTabRowBytes>(addr[i]);
+        else if (c == 2) t = lds_f32<3 * kTabRowBytes>(addr[i]);
+        else t = lds_f32<4 * kTabRowBytes>(addr[i]);
         addr[i] = drop_if_below(addr[i], a[i], t, static_cast<uint32_t>(kEntryBytes));
+        constexpr int kQ0 = 4, kQ1 = 8;  // byte offsets of the low- and high-half fp16 words
         if (i & 1) {
-          if (u == 0) q[i] = lds_u32<kTabRowBytes + 8>(addr[i]);
-          else if (u == 1) q[i] = lds_u32<2 * kTabRowBytes + 8>(addr[i]);
-          else q[i] = lds_u32<3 * kTabRowBytes + 8>(addr[i]);
+          if (c == 0) q[i] = lds_u32<kTabRowBytes + kQ1>(addr[i]);
+          else if (c == 1) q[i] = lds_u32<2 * kTabRowBytes + kQ1>(addr[i]);
+          else if (c == 2) q[i] = lds_u32<3 * kTabRowBytes + kQ1>(addr[i]);
+          else q[i] = lds_u32<4 * kTabRowBytes + kQ1>(addr[i]);
         } else {
-          if (u == 0) q[i] = lds_u32<kTabRowBytes + 4>(addr[i]);
-          else if (u == 1) q[i] = lds_u32<2 * kTabRowBytes + 4>(addr[i]);
-          else q[i] = lds_u32<3 * kTabRowBytes + 4>(addr[i]);
+          if (c == 0) q[i] = lds_u32<kTabRowBytes + kQ0>(addr[i]);
+          else if (c == 1) q[i] = lds_u32<2 * kTabRowBytes + kQ0>(addr[i]);
+          else if (c == 2) q[i] = lds_u32<3 * kTabRowBytes + kQ0>(addr[i]);
+          else q[i] = lds_u32<4 * kTabRowBytes + kQ0>(addr[i]);
         }
       }
-      evaluate(q, k + u);
+      float tp[2];
+      partials(q, k + c, tp);
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        if ((c & 1) == 0) {
+          hold[u] = tp[u];
+        } else {  // candidates (c - 1, c): keep the one with index bit b0, hand over the other
+          spair[c >> 1][u] = (b0 ? tp[u] : hold[u]) + __shfl_xor_sync(0xffffffffu, b0 ? hold[u] : tp[u], 1);
+        }
+      }
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) addr[i] += 3 * kTabRowBytes;
+    for (int i = 0; i < 8; ++i) addr[i] += 4 * kTabRowBytes;
+    const int kk = k + tq;
+    const float s2 = sh.s2[kk];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const float t = (b1 ? spair[1][u] : spair[0][u]) + __shfl_xor_sync(0xffffffffu, b1 ? spair[0][u] : spair[1][u], 2);
+      const float L = fmaf(s2, t, cconst[u]);
+      if (L < best[u]) {
+        best[u] = L;
+        best_k[u] = kk;
+      }
+    }
+  }
+  // Merge the quad's bests: the smallest loss, and on equal losses the lowest candidate.
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      const float ol = __shfl_xor_sync(0xffffffffu, best[u], o);
+      const int ok = __shfl_xor_sync(0xffffffffu, best_k[u], o);
+      if (ol < best[u] || (ol == best[u] && ok < best_k[u])) {
+        best[u] = ol;
+        best_k[u] = ok;
+      }
+    }
   }
 
   // ---- outputs. The winner's loss is recomputed from its fp32 fake-quant weights by the
