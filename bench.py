@@ -48,10 +48,11 @@ WORKLOAD_TEXT = {
 # dram__bytes_read.sum + dram__bytes_write.sum per launch, from one ncu capture of the current
 # kernel on this workload (summaries in profiles/); workloads without a capture report null.
 SWEEP_TRAFFIC_BYTES = {
+    "dense": 33_871_872 + 136_704_512,   # sweep_tc_kernel, profiles/sweep_tc_kernel_dense.md
     "wmse": 101_576_704 + 166_720_000,   # sweep_diag_kernel, profiles/sweep_diag_kernel_wmse.md
 }
 ACCUM_TRAFFIC_BYTES = {
-    "dense": 134_263_808 + 3_650_816,    # accum_mma_kernel (clusters), profiles/accum_mma_kernel_dense.md
+    "dense": 134_265_344 + 3_774_464,    # accum_mma_kernel (clusters), profiles/accum_mma_kernel_dense.md
     "act": 268_573_696 + 5_457_664,      # accum_mma_kernel (quantizer fused), profiles/accum_mma_kernel_act.md
     "wmse": 1_610_820_000 + 8_041_472,   # accum_diag_kernel (+ the partial reduction, not captured)
 }
