@@ -24,12 +24,18 @@ Sources (PR pages of NVIDIA Model-Optimizer):
   description: one Hessian per expert over exactly the tokens routed to it; an
   expert no token reaches gets the plain search.
 
-Readings where the pages are silent (each also listed in the design notes):
+Readings where the pages are silent:
 candidates are E4M3 codes 0x01..0x7E; scale s_k = fp32(v_k * g); E2M1 rounds the
 exact quotient |w|/s_k to nearest, ties to even, clamped at 6; the fake-quant value
 is fp32(q * s_k) with w's sign; ties in loss go to the lowest code; B is the number
 of token rows accumulated; a group with B = 0 gets H = I, P = 0 (DIAG: Imp = 1);
-g = 0 makes every q zero.
+g = 0 makes every q zero. The input quantizer that produces X_q (act_fake_quant) takes a
+per-tensor global scale gx = fp32(amax|X| / 2688) as an input, rounds each block's
+amax / (6 gx) to the nearest E4M3 code and each value to E2M1 on exact quotients, and
+outputs bf16. The "mse" method is the same search with H = I. The 4/6 variant
+normalizes the global scale by 256 instead of 448. The exported per-block amax is
+fp32(6 v g). The amax-multiplier search maps fp32(m * amax_blk) to the nearest E4M3
+code of amax / (6 g), and the first multiplier with the smallest loss wins.
 """
 from __future__ import annotations
 

@@ -1,6 +1,6 @@
 """Comparators and device helpers shared by the GPU parity tests.
 
-Tolerances (BASELINE targets, also stated in the design notes):
+Tolerances (the parity bar for the GPU path):
   * Hessians H / P: relative Frobenius error per 16x16 block <= 1e-4; importance per block
     (16 values) <= 1e-4; an all-zero oracle block requires an exactly zero GPU block.
   * Sweep: codes and fake-quant weights bit-exact for every unit whose oracle gap
