@@ -49,7 +49,7 @@ WORKLOAD_TEXT = {
 # kernel on this workload (summaries in profiles/); workloads without a capture report null.
 SWEEP_TRAFFIC_BYTES = {
     "dense": 33_871_872 + 136_704_512,   # sweep_tc_kernel, profiles/sweep_tc_kernel_dense.md
-    "wmse": 101_576_704 + 166_720_000,   # sweep_diag_kernel, profiles/sweep_diag_kernel_wmse.md
+    "wmse": 101_393_408 + 167_207_936,   # sweep_diag_kernel, profiles/sweep_diag_kernel_wmse.md
 }
 ACCUM_TRAFFIC_BYTES = {
     "dense": 134_265_344 + 3_774_464,    # accum_mma_kernel (clusters), profiles/accum_mma_kernel_dense.md
