@@ -199,6 +199,7 @@ lhcal_status lhcal_global_scale_ex(lhcal_dtype dtype, const void* w, int32_t gro
  *   codes : out [groups, rows, cin/16] uint8, the E4M3 bit pattern of the chosen scale.
  *   wq    : out [groups, rows, cin] fp32 fake-quantized weights (16-byte aligned), or NULL.
  *   loss  : out [groups, rows, cin/16] fp32 winning loss, or NULL.
+ * Sizes: rows <= 65535 * 128, cin / 16 <= 65535, groups <= 65535 (LHCAL_ERR_INVALID_ARG otherwise).
  */
 lhcal_status lhcal_scale_sweep(lhcal_mode mode, lhcal_dtype dtype, const void* w, int32_t groups,
                                int64_t rows, int64_t cin, const float* h, const float* p,

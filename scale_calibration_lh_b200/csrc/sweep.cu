@@ -66,9 +66,9 @@ sweep_diag_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const flo
                   float* __restrict__ loss) {
   __shared__ DiagShared sh;
   const int64_t nblk = cin / kBlock;
-  const int64_t n = blockIdx.y;
+  const int64_t n = blockIdx.x;  // blocks fastest: neighbouring CTAs share rows (see sweep_tc.cu)
   const int64_t e = blockIdx.z;
-  const int64_t rbase = static_cast<int64_t>(blockIdx.x) * kThreads;
+  const int64_t rbase = static_cast<int64_t>(blockIdx.y) * kThreads;
 
   const float gs = __ldg(g + e);
   for (int idx = threadIdx.x; idx < kCand * kLev; idx += kThreads) {
@@ -247,7 +247,7 @@ sweep_diag_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const flo
 lhcal_status launch_sweep(lhcal_mode mode, lhcal_dtype dtype, const void* w, int32_t groups,
                           int64_t rows, int64_t cin, const float* h, const float* p, const float* g,
                           uint8_t* codes, float* wq, float* loss, cudaStream_t stream) {
-  if (rows > static_cast<int64_t>(0x7fffffff) || cin / kBlock > 65535 || groups > 65535)
+  if (ceil_div(rows, kThreads) > 65535 || cin / kBlock > 65535 || groups > 65535)
     return fail(LHCAL_ERR_INVALID_ARG, "scale sweep: grid too large (rows %lld, cin %lld, groups %d)",
                 (long long)rows, (long long)cin, groups);
   // FULL and ACT_AWARE: quadratic form on tensor cores; DIAG: FP32 weighted sum.
@@ -255,7 +255,7 @@ lhcal_status launch_sweep(lhcal_mode mode, lhcal_dtype dtype, const void* w, int
     return launch_sweep_tc(mode, dtype, w, groups, rows, cin, h, p, g, codes, wq, loss, stream);
   if (mode != LHCAL_DIAG && mode != LHCAL_MSE) return fail(LHCAL_ERR_UNSUPPORTED, "scale sweep: unsupported mode");
   if (mode == LHCAL_MSE) h = nullptr;
-  const dim3 grid(static_cast<unsigned>(ceil_div(rows, kThreads)), static_cast<unsigned>(cin / kBlock),
+  const dim3 grid(static_cast<unsigned>(cin / kBlock), static_cast<unsigned>(ceil_div(rows, kThreads)),
                   static_cast<unsigned>(groups));
   if (dtype == LHCAL_BF16)
     sweep_diag_kernel<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(w), rows,

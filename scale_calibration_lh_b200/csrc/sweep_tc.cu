@@ -126,7 +126,9 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
                 float* __restrict__ wq, float* __restrict__ loss) {
   __shared__ TcShared sh;
   const int64_t nblk = cin / kBlock;
-  const int64_t n = blockIdx.y;
+  // Blocks vary fastest across the grid: CTAs running together cover neighbouring blocks of the
+  // same rows, so their W reads are adjacent and their codes / loss writes share DRAM sectors.
+  const int64_t n = blockIdx.x;
   const int64_t e = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, tq = lane & 3;
@@ -147,7 +149,7 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
   }
   // Order the CTA's rows by their smallest |w|, so that the units a warp evaluates together
   // leave the all-clamped candidates at similar scales (see the clamped prefix below).
-  const int64_t rbase = static_cast<int64_t>(blockIdx.x) * kUnitsPerCta;
+  const int64_t rbase = static_cast<int64_t>(blockIdx.y) * kUnitsPerCta;
   if (threadIdx.x < kUnitsPerCta) {
     const int64_t row = rbase + threadIdx.x;
     float m = __int_as_float(0x7f800000);
@@ -515,7 +517,7 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
 lhcal_status launch_sweep_tc(lhcal_mode mode, lhcal_dtype dtype, const void* w, int32_t groups, int64_t rows,
                              int64_t cin, const float* h, const float* p, const float* g, uint8_t* codes,
                              float* wq, float* loss, cudaStream_t stream) {
-  const dim3 grid(static_cast<unsigned>(ceil_div(rows, kUnitsPerCta)), static_cast<unsigned>(cin / kBlock),
+  const dim3 grid(static_cast<unsigned>(cin / kBlock), static_cast<unsigned>(ceil_div(rows, kUnitsPerCta)),
                   static_cast<unsigned>(groups));
   if (dtype == LHCAL_BF16) {
     if (mode == LHCAL_ACT_AWARE)
