@@ -48,7 +48,7 @@ WORKLOAD_TEXT = {
 # dram__bytes_read.sum + dram__bytes_write.sum per launch, from one ncu capture of the current
 # kernel on this workload (summaries in profiles/); workloads without a capture report null.
 SWEEP_TRAFFIC_BYTES = {
-    "dense": 33_880_000 + 123_050_000,   # sweep_tc_kernel, profiles/sweep_tc_kernel_dense.md
+    "dense": 33_938_176 + 30_059_264,    # sweep_tc_kernel, profiles/sweep_tc_kernel_dense.md
     "wmse": 101_393_408 + 167_207_936,   # sweep_diag_kernel, profiles/sweep_diag_kernel_wmse.md
 }
 ACCUM_TRAFFIC_BYTES = {

@@ -57,6 +57,9 @@ struct __align__(16) TcShared {
   float hscale;  // 2^-eH: H' = H * hscale lies below 2^15
   float key[kUnitsPerCta];  // min |w| of each of the CTA's units (rows)
   int perm[kUnitsPerCta];   // the CTA's rows ordered by key
+  // Each warp's 16 units' weights (fp32), rows padded to 17 floats so that the 8 units a warp
+  // reads at once fall in distinct banks. Read by the per-unit set-up and the ACT epilogue.
+  float wst[kTcWarps][kUnitsPerWarp][kBlock + 1];
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -208,16 +211,23 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
     }
   }
 
-  // ---- the warp's 16 units: sorted positions 16 warp + gq (unit 0) and + 8 (unit 1)
-  int64_t ur[2];
-  bool valid[2];
-  float wrow[2][16];
+  // ---- the warp's 16 units: sorted positions 16 warp + gq (unit 0) and + 8 (unit 1). Their
+  // weights go to shared memory (lane l loads half l & 1 of unit l / 2), so that the set-up
+  // below reads them instead of holding 32 of them in registers.
+  float (*wst)[kBlock + 1] = sh.wst[warp];
+  {
+    const int j = lane >> 1, h8 = (lane & 1) * 8;
+    const int64_t row = rbase + sh.perm[warp * kUnitsPerWarp + j];
+    const bool ok = row < rows;
+    float w8[8];
+    if (ok) load8<WT>(w + (e * rows + row) * cin + n * kBlock + h8, w8);
 #pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    ur[u] = rbase + sh.perm[warp * kUnitsPerWarp + gq + 8 * u];
-    valid[u] = ur[u] < rows;
-    load_row16<WT>(w + (e * rows + (valid[u] ? ur[u] : 0)) * cin + n * kBlock, valid[u], wrow[u]);
+    for (int k = 0; k < 8; ++k) wst[j][h8 + k] = ok ? w8[k] : 0.f;
   }
+  __syncwarp();
+  bool valid[2];
+#pragma unroll
+  for (int u = 0; u < 2; ++u) valid[u] = rbase + sh.perm[warp * kUnitsPerWarp + gq + 8 * u] < rows;
   // Lane element i (0..7): unit i / 4, column col_of(i % 4) with columns {2t, 2t+1, 2t+8, 2t+9}.
   auto col_of = [&](int ci) { return 2 * tq + (ci & 1) + 8 * (ci >> 1); };
   float a[8], up[8];
@@ -231,7 +241,8 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
     for (int ci = 0; ci < 4; ++ci) {
       const int c = col_of(ci);
       const int i = 4 * u + ci;
-      const float x = wrow[u][c];
+      const float* wr = wst[gq + 8 * u];
+      const float x = wr[c];
       a[i] = fabsf(x);
       amin[u] = fminf(amin[u], a[i]);
       sgn[i] = __float_as_uint(x) >> 31;
@@ -239,10 +250,11 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
         const float hck = sh.h[c * 16 + k];
-        hw_sym = fmaf(0.5f * (hck + sh.h[k * 16 + c]), wrow[u][k], hw_sym);
-        hw_row = fmaf(hck, wrow[u][k], hw_row);
-        hsg += (__float_as_uint(wrow[u][k]) >> 31) ? -hck : hck;  // (H sign(w))_c
-        if (ACT) pw = fmaf(sh.p[c * 16 + k], wrow[u][k], pw);
+        const float wk = wr[k];
+        hw_sym = fmaf(0.5f * (hck + sh.h[k * 16 + c]), wk, hw_sym);
+        hw_row = fmaf(hck, wk, hw_row);
+        hsg += (__float_as_uint(wk) >> 31) ? -hck : hck;  // (H sign(w))_c
+        if (ACT) pw = fmaf(sh.p[c * 16 + k], wk, pw);
       }
       up[i] = hw_sym - pw;                               // U'_c
       cpart[u] = fmaf(x, hw_row - 2.f * pw, cpart[u]);  // w_c ((H w)_c - 2 (P w)_c)
@@ -455,8 +467,11 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const float4* tab_k = sh.tab + kLev * best_k[i >> 2];
-    wqv[i] = __uint_as_float(__float_as_uint(tab_k[level_direct_tc(tab_k, a[i])].w) | (sgn[i] << 31));
-    dwv[i] = wqv[i] - __uint_as_float(__float_as_uint(a[i]) | (sgn[i] << 31));
+    // The sign bit of element i, from the packed A-register masks (not kept live through the sweep).
+    constexpr int kPairOf[8] = {0, 0, 2, 2, 1, 1, 3, 3};
+    const uint32_t sbit = (smask[kPairOf[i]] >> ((i & 1) ? 31 : 15)) & 1u;
+    wqv[i] = __uint_as_float(__float_as_uint(tab_k[level_direct_tc(tab_k, a[i])].w) | (sbit << 31));
+    dwv[i] = wqv[i] - __uint_as_float(__float_as_uint(a[i]) | (sbit << 31));
   }
 #pragma unroll 1
   for (int u = 0; u < 2; ++u) {
@@ -473,8 +488,9 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
       for (int ci = 0; ci < 4; ++ci)
         dfull[2 * t2 + (ci & 1) + 8 * (ci >> 1)] = __shfl_sync(0xffffffffu, dw[ci], (lane & ~3) | t2);
     }
-    const bool ok = u ? valid[1] : valid[0];
-    const int64_t row = u ? ur[1] : ur[0];
+    // The unit's row, read again from the CTA's ordering (not kept live through the sweep).
+    const int64_t row = rbase + sh.perm[warp * kUnitsPerWarp + gq + 8 * u];
+    const bool ok = row < rows;
     float part = 0.f;
 #pragma unroll
     for (int ci = 0; ci < 4; ++ci) {
@@ -482,16 +498,11 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
       float hd = 0.f;
 #pragma unroll
       for (int k = 0; k < 16; ++k) hd = fmaf(sh.h[c * 16 + k], dfull[k], hd);
-      if (ACT) {  // + 2 (P w)_c, with w reloaded from global memory
-        const WT* wr = w + (e * rows + (ok ? row : 0)) * cin + n * kBlock;
+      if (ACT) {  // + 2 (P w)_c, with w from the warp's shared copy
+        const float* wr = wst[gq + 8 * u];
         float pw = 0.f;
 #pragma unroll
-        for (int k0 = 0; k0 < 16; k0 += 8) {
-          float w8[8];
-          if (ok) load8<WT>(wr + k0, w8);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) pw = fmaf(sh.p[c * 16 + k0 + k], ok ? w8[k] : 0.f, pw);
-        }
+        for (int k = 0; k < 16; ++k) pw = fmaf(sh.p[c * 16 + k], wr[k], pw);
         hd = fmaf(2.f, pw, hd);
       }
       part = fmaf(dw[ci], hd, part);
