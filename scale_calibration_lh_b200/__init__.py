@@ -421,16 +421,18 @@ class CalibrationGraph:
 
         m = _mode_id(mode)
         groups, rows, cin = (int(v) for v in w.shape)
-        self.buffers = buffers or Buffers(m, int(x.shape[0]), cin, rows, groups, _dtype_id(x), x.device)
+        dev = w.device
+        tokens = 0 if x is None else int(x.shape[0])  # MSE reads no activations
+        self.buffers = buffers or Buffers(m, tokens, cin, rows, groups, _dtype_id(w if x is None else x), dev)
         args = dict(xq=xq, group_offsets=group_offsets, token_ids=token_ids, buffers=self.buffers, act_gx=act_gx)
         calibrate(m, x, w, **args)
-        torch.cuda.synchronize(x.device)
+        torch.cuda.synchronize(dev)
         self.graph = torch.cuda.CUDAGraph()
-        side = torch.cuda.Stream(device=x.device)
-        side.wait_stream(torch.cuda.current_stream(x.device))
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
         with torch.cuda.graph(self.graph, stream=side, capture_error_mode="thread_local"):
             calibrate(m, x, w, **args)
-        torch.cuda.current_stream(x.device).wait_stream(side)
+        torch.cuda.current_stream(dev).wait_stream(side)
 
     def replay(self):
         self.graph.replay()

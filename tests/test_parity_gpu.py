@@ -416,6 +416,29 @@ def test_graph_replay_matches_eager_calls():
         assert torch.equal(out.h.view(torch.int32), eager.h.view(torch.int32))
 
 
+@pytest.mark.parametrize("mode", ["act", "mse"])
+def test_graph_replay_fused_quantizer_and_mse(mode):
+    """The captured path with the input quantizer fused (X and gx in; the token splits reduce
+    through the workspace), and the statistics-free MSE sweep."""
+    layers = [P.make_layer("act" if mode == "act" else "dense", s, tokens=900, cin=256, rows=64) for s in (31, 32)]
+    devs = [P.layer_to_device(ly) for ly in layers]
+    x, w = devs[0]["x"].clone(), devs[0]["w"].clone()
+    gx = devs[0]["act_gx"].clone() if mode == "act" else None
+    graph = L.CalibrationGraph(mode, None if mode == "mse" else x, w, act_gx=gx)
+    for d in (devs[1], devs[0]):
+        x.copy_(d["x"])
+        w.copy_(d["w"])
+        if gx is not None:
+            gx.copy_(d["act_gx"])
+        out = graph.replay()
+        eager = L.calibrate(mode, None if mode == "mse" else d["x"], d["w"], act_gx=d["act_gx"] if gx is not None else None)
+        _sync()
+        assert torch.equal(out.codes, eager.codes)
+        assert torch.equal(out.loss.view(torch.int32), eager.loss.view(torch.int32))
+        if mode == "act":
+            assert torch.equal(out.p.view(torch.int32), eager.p.view(torch.int32))
+
+
 # ----------------------------------------------------------------------------- input quantizer
 
 def _act_x(tokens, cin, seed):
