@@ -718,3 +718,38 @@ def test_calibrate_host_matches_the_device_path(name, kw, chunks):
                             out=L.HostOutputs(buf, want_wq=False), group_chunks=chunks)
     torch.cuda.current_stream().synchronize()
     assert out2.wq is None and torch.equal(out2.codes, want[0])
+
+
+# ----------------------------------------------------------------------------- more edge cases (2)
+
+def test_fused_act_quant_grouped_with_empty_experts():
+    """20 tokens routed to 2 of 16 experts each: most experts get no token and fall back to
+    H = I, P = 0 after finalisation; their raw sums must be exact zeros."""
+    layer = synth.make_layer("moe", 71, tokens=20, cin=48, rows=16, groups=16, top_k=2)
+    assert np.any(np.diff(layer.group_offsets) == 0)
+    layer.mode = "act"
+    P.act_inputs(layer)
+    _run_and_check(layer, fused=True)
+
+
+@pytest.mark.parametrize("n_mult", [1, 1024])
+def test_multiplier_search_counts(n_mult):
+    layer = P.make_layer("dense", 72, tokens=300, cin=64, rows=50)
+    G, R, C = layer.groups, layer.rows, layer.cin
+    w32 = layer.w_f32()
+    g = np.array([O.global_scale(w32[0])], np.float32)
+    hs, _, counts = O.accumulate("full", layer.x_f32())
+    h, _ = O.finalize("full", hs, None, counts)
+    h = h.astype(np.float32).astype(np.float64)
+    mult = (np.float32([1.0]) if n_mult == 1 else np.linspace(0.01, 3.0, n_mult).astype(np.float32))
+    d = P.layer_to_device(layer)
+    codes = torch.empty((G, R, C // 16), dtype=torch.uint8, device="cuda")
+    wq = torch.empty((G, R, C), dtype=torch.float32, device="cuda")
+    loss = torch.empty((G, R, C // 16), dtype=torch.float32, device="cuda")
+    L.lhcal_multiplier_search("full", d["w"], P.to_device(h, "f32"), P.to_device(g, "f32"), P.to_device(mult, "f32"),
+                              codes, wq=wq, loss=loss)
+    _sync()
+    units = P.all_units(G, R, C // 16)
+    ref = O.multiplier_search("full", w32, h, None, g, mult, units)
+    gc, gw, gl = P.gather_gpu_units(codes, wq, loss, units)
+    P.check_sweep(gc, gw, gl, ref, f"multiplier search, {n_mult} multipliers")
