@@ -292,8 +292,7 @@ lhcal_status lhcal_multiplier_search(lhcal_mode mode, lhcal_dtype dtype, const v
   if (!valid_sweep_mode(mode) || !valid_dtype(dtype)) return fail(LHCAL_ERR_UNSUPPORTED, "unknown mode or dtype");
   LHCAL_TRY(check_cin(cin));
   LHCAL_TRY(check_groups(groups));
-  if (rows <= 0 || rows > (int64_t)INT32_MAX * 64)
-    return fail(LHCAL_ERR_INVALID_ARG, "rows (%lld) out of range", (long long)rows);
+  if (rows <= 0) return fail(LHCAL_ERR_INVALID_ARG, "rows (%lld) must be positive", (long long)rows);
   if (n_multipliers < 1 || n_multipliers > LHCAL_MAX_MULTIPLIERS)
     return fail(LHCAL_ERR_INVALID_ARG, "n_multipliers (%d) must be in [1, %d]", n_multipliers, LHCAL_MAX_MULTIPLIERS);
   if (mode == LHCAL_MSE && (h != nullptr || p != nullptr)) return fail(LHCAL_ERR_INVALID_ARG, "MSE takes no h or p");
@@ -307,7 +306,7 @@ lhcal_status lhcal_multiplier_search(lhcal_mode mode, lhcal_dtype dtype, const v
   LHCAL_TRY(check_device_ptr(codes, 1, "codes"));
   if (wq != nullptr) LHCAL_TRY(check_device_ptr(wq, 16, "wq"));
   if (loss != nullptr) LHCAL_TRY(check_device_ptr(loss, 4, "loss"));
-  if (ceil_div(rows, 128) > 0x7fffffff) return fail(LHCAL_ERR_INVALID_ARG, "rows too large");
+  if (ceil_div(rows, 128) > 0x7fffffff) return fail(LHCAL_ERR_INVALID_ARG, "rows (%lld) too large", (long long)rows);
   return launch_multiplier_search(mode, dtype, w, groups, rows, cin, h, p, g, multipliers, n_multipliers, codes, wq,
                                   loss, static_cast<cudaStream_t>(stream));
 }
