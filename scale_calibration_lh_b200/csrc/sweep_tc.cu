@@ -27,6 +27,12 @@
 // each element's level falls by at most one per candidate from the 4th on. Each table entry
 // also carries the fp16 bits of its grid value, pre-placed for the low or the high half of
 // a packed pair, so building the A fragment is one OR (and a sign XOR) per pair.
+//
+// Work per candidate. Candidates below the warp's first unclamped one take a closed form;
+// the rest go four per loop trip, and the quad's four lanes share the reduction of four
+// candidates (a transposed reduction: lane t ends with candidate k + t) and keep their own
+// bests, merged after the loop. The per-unit set-up reads the units' weights from shared
+// memory, and the grid runs the 16-column blocks fastest.
 #include "common.cuh"
 #include "quant_tables.cuh"
 
