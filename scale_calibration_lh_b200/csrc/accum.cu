@@ -15,9 +15,12 @@
 //    wasted MACs. bf16 x bf16 products are exact in the fp32 accumulator. For P the
 //    difference D = X_q - X (exact in fp32) is split into bf16 hi + lo parts, two more MMAs
 //    each. (Forming P as H - X_q^T X instead would cost two MMAs fewer, but the cancellation
-//    multiplies the accumulation error by |H| / |P|, which exceeds 100 on real blocks.) Dense: token ranges are split across CTAs and partials go to the workspace,
-//    reduced in a fixed order by reduce_partials_kernel. Grouped: one CTA per (group, slab)
-//    gathers its routed rows through the CSR and writes the group's blocks directly.
+//    multiplies the accumulation error by |H| / |P|, which exceeds 100 on real blocks.)
+//    Dense layers with enough slabs to fill a wave: clusters of up to 8 CTAs split a slab's
+//    tokens and reduce in distributed shared memory. Narrower dense layers: token splits write
+//    partials to the workspace, which reduce_partials_kernel sums in a fixed order. Grouped
+//    (MoE): a CTA walks a run of consecutive experts of its slab with one pipeline, gathering
+//    the routed rows through the CSR, and writes each expert's sums after its last tile.
 //    Activation-aware with the input quantizer fused (QUANT): only X streams in; each warp
 //    turns its block's 64 x 16 slice of the tile into X_q in shared memory (act_quant.cuh)
 //    and synchronises only with itself before the MMAs, so X is read from HBM once.
