@@ -79,9 +79,14 @@ amax_kernel(const T* __restrict__ w, int64_t per_group, uint32_t* __restrict__ a
   const T* base = w + e * per_group;
   const int64_t n8 = per_group / 8;
   uint32_t m = 0;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    m = max(m, abs_bits8<T>(base + i * 8));
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (; i + 3 * stride < n8; i += 4 * stride) {  // four independent 16-byte loads in flight
+    const uint32_t a = abs_bits8<T>(base + i * 8), b = abs_bits8<T>(base + (i + stride) * 8);
+    const uint32_t c = abs_bits8<T>(base + (i + 2 * stride) * 8), d = abs_bits8<T>(base + (i + 3 * stride) * 8);
+    m = max(m, max(max(a, b), max(c, d)));
+  }
+  for (; i < n8; i += stride) m = max(m, abs_bits8<T>(base + i * 8));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
   __shared__ uint32_t red[kAmaxThreads / 32];
