@@ -141,3 +141,17 @@ def test_multiplier_search_validates_without_gpu(lib):
     assert f(0, 1, None, 1, 4, 32, None, None, None, None, 2000, None, None, None, None) == L.ERR_INVALID_ARG
     assert b"n_multipliers" in lib.lhcal_last_error_string()
     assert f(1, 1, None, 1, 4, 32, None, None, None, None, 8, None, None, None, None) == L.ERR_INVALID_ARG  # no p
+
+
+def test_buffers_size_the_workspace_for_either_activation_aware_entry_point(lib):
+    """Buffers (host-only sizing, CPU tensors here) cover both the two-tensor and the fused
+    activation-aware accumulations, and the statistics-free MSE mode allocates no H."""
+    for tokens, cin in ((32768, 4096), (3000, 1024), (700, 96)):
+        b = L.Buffers("act", tokens, cin, 8, 1, L.BF16, "cpu")
+        need = max(L.lhcal_accumulate_workspace("act", L.BF16, tokens, cin, 1),
+                   L.lhcal_accumulate_act_quant_workspace(L.BF16, tokens, cin, 1))
+        have = 0 if b.workspace is None else b.workspace.numel() * b.workspace.element_size()
+        assert have >= need and b.p is not None
+    m = L.Buffers("mse", 0, 64, 8, 2, L.BF16, "cpu")
+    assert m.h is None and m.p is None and m.workspace is None
+    assert tuple(m.codes.shape) == (2, 8, 4) and tuple(m.wq.shape) == (2, 8, 64)
