@@ -4,8 +4,12 @@
 One step = the whole hot path over one layer: Hessian accumulation (OVERWRITE), token
 counts, finalisation, per-group global scale, and the exhaustive 126-candidate FP8 scale
 sweep writing codes, fake-quantized weights and losses. Inputs are resident in HBM when
-the timed region starts; they are larger than the 126 MB L2 for every bench workload, so
-no L2 flush runs between steps.
+the timed region starts; each step's inputs (X and W together) exceed the 126 MB L2 for
+every bench workload, so no L2 flush runs between steps.
+
+e2e: the same step through calibrate_host from pinned host buffers, inputs copied in and
+the result (codes and losses) copied out every step. The activation-aware workload also
+reports the two-tensor accumulation (X_q resident) beside its fused step.
 
   python bench.py [--gpus N --steps K --warmup W --workload dense|act|wmse|moe]
   python bench.py --impl reference ...   (the CPU oracle, timed on a bounded sample)
@@ -416,7 +420,7 @@ def run_lhcal(args, rank, world, local_rank):
         "data": "synthetic",
         "config": {"workload": WORKLOAD_TEXT[args.workload], "name": args.workload, "tokens": T, "cin": C,
                    "rows": R, "groups": G, "mode": layer.mode, "input_dtype": layer.dtype,
-                   "l2": "no flush: inputs larger than L2 (126 MB)",
+                   "l2": "no flush: each step's inputs (X and W) exceed the 126 MB L2",
                    "parallelism": f"{world} independent layers, one per GPU (no collective)"},
         "roofline": {"kernel": "sweep_diag_kernel" if layer.mode == "diag" else "sweep_tc_kernel", "bound": "alu", "achieved": achieved_ops / 1e12,
                      "peak": peak_ops / 1e12, "unit": "Tops/s", "frac": achieved_ops / peak_ops,
