@@ -2,8 +2,9 @@
 
 Argument marshalling only: every step runs in the CUDA library. Functions carry the C
 names (``lhcal_accumulate`` ...) and take torch tensors, passing their device pointers,
-sizes and the current CUDA stream. A missing or unloadable library raises at import of
-the first call; there is no fallback.
+sizes and the current CUDA stream. Since the C layer sees only pointers, each wrapper first
+checks every tensor's dtype, density and element count against the sizes it passes. A
+missing or unloadable library raises at import of the first call; there is no fallback.
 """
 from __future__ import annotations
 
@@ -95,6 +96,66 @@ def _ld(t, cin: int) -> int:
     return int(t.stride(0)) if t.shape[0] > 0 else cin
 
 
+def _need(t, name: str, numel: int, dtype=None, dense: bool = True):
+    """Reject a tensor the library would misread. The entry points take bare pointers and
+    infer a dense layout from the sizes, so a short, strided or mistyped buffer would be
+    read or written past its end without an error. None passes (the C layer decides
+    whether the pointer is optional)."""
+    if t is None:
+        return
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if dense and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.numel() < numel:
+        raise ValueError(f"{name} has {t.numel()} elements; the call needs {numel}")
+
+
+def _stats_numel(m: int, groups: int, cin: int) -> int:
+    """fp32 elements of H (or P): [groups, cin/16, 16, 16], or [groups, cin/16, 16] for DIAG."""
+    return groups * (cin // BLOCK) * (BLOCK if m == DIAG else BLOCK * BLOCK)
+
+
+def _check_xq(x, xq):
+    """X_q is read with x's row stride (the two-tensor entry points take one ldx for both)."""
+    if xq is None:
+        return
+    if tuple(xq.shape) != tuple(x.shape) or xq.dtype != x.dtype:
+        raise ValueError(f"xq {tuple(xq.shape)} {xq.dtype} must match x {tuple(x.shape)} {x.dtype}")
+    if x.numel() and (xq.stride(1) != 1 or xq.stride(0) != x.stride(0)):
+        raise ValueError("xq must have x's row stride and unit stride along cin")
+
+
+def _check_stats(m: int, x, h, p, group_offsets, token_ids, groups: int):
+    import torch
+
+    n = _stats_numel(m, groups, int(x.shape[1]))
+    _need(h, "h", n, torch.float32)
+    if m == ACT_AWARE:
+        _need(p, "p", n, torch.float32)
+    _need(group_offsets, "group_offsets", groups + 1, torch.int32)
+    _need(token_ids, "token_ids", 0, torch.int32)
+
+
+def _check_sweep_buffers(m: int | None, w, h, p, g, codes, wq, loss, wq16=None, amax=None):
+    import torch
+
+    groups, rows, cin = (int(v) for v in w.shape)
+    units = groups * rows * (cin // BLOCK)
+    _need(w, "w", 0)
+    if m is not None and m != MSE:
+        n = _stats_numel(m, groups, cin)
+        _need(h, "h", n, torch.float32)
+        if m == ACT_AWARE:
+            _need(p, "p", n, torch.float32)
+    _need(g, "g", groups, torch.float32)
+    _need(codes, "codes", units, torch.uint8)
+    _need(wq, "wq", groups * rows * cin, torch.float32)
+    _need(wq16, "wq16", groups * rows * cin, torch.bfloat16)
+    _need(loss, "loss", units, torch.float32)
+    _need(amax, "amax", units, torch.float32)
+
+
 def _dtype_id(t) -> int:
     import torch
 
@@ -132,6 +193,8 @@ def lhcal_accumulate(mode, x, h, xq=None, p=None, group_offsets=None, token_ids=
     if x.numel() and x.stride(1) != 1:
         raise ValueError("x must have unit stride along cin")
     groups = 1 if group_offsets is None else int(group_offsets.numel()) - 1
+    _check_xq(x, xq)
+    _check_stats(m, x, h, p, group_offsets, token_ids, groups)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(load_library().lhcal_accumulate(
         m, _dtype_id(x), _ptr(x), _ptr(xq), tokens, cin, _ld(x, cin), groups,
@@ -149,10 +212,14 @@ def lhcal_accumulate_act_quant(x, h, p, act_gx, group_offsets=None, token_ids=No
                                workspace=None, stream=None):
     """Activation-aware accumulation with the input quantizer fused: X_q is derived from x (bf16)
     in the kernel with the global scale act_gx (fp32 device scalar); h, p as for ``act``."""
+    import torch
+
     tokens, cin = int(x.shape[0]), int(x.shape[1])
     if x.numel() and x.stride(1) != 1:
         raise ValueError("x must have unit stride along cin")
     groups = 1 if group_offsets is None else int(group_offsets.numel()) - 1
+    _check_stats(ACT_AWARE, x, h, p, group_offsets, token_ids, groups)
+    _need(act_gx, "act_gx", 1, torch.float32)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(load_library().lhcal_accumulate_act_quant(
         _dtype_id(x), _ptr(x), tokens, cin, _ld(x, cin), groups, _ptr(group_offsets), _ptr(token_ids),
@@ -161,7 +228,13 @@ def lhcal_accumulate_act_quant(x, h, p, act_gx, group_offsets=None, token_ids=No
 
 def lhcal_act_fake_quant(x, act_gx, xq, stream=None):
     """X_q = NVFP4 fake quant of bf16 x [tokens, cin] with global scale act_gx, into bf16 xq."""
+    import torch
+
     tokens, cin = int(x.shape[0]), int(x.shape[1])
+    if xq is None or tuple(xq.shape) != tuple(x.shape):
+        raise ValueError("xq must be a tensor shaped like x")
+    _need(xq, "xq", 0, torch.bfloat16, dense=False)  # its own row stride is passed
+    _need(act_gx, "act_gx", 1, torch.float32)
     if x.numel() and (x.stride(1) != 1 or xq.stride(1) != 1):
         raise ValueError("x and xq must have unit stride along cin")
     _check(load_library().lhcal_act_fake_quant(_dtype_id(x), _ptr(x), tokens, cin, _ld(x, cin), _ptr(act_gx),
@@ -185,27 +258,40 @@ def lhcal_accumulate_noalloc(mode, x, h, xq=None, p=None, group_offsets=None, to
     if x.numel() and x.stride(1) != 1:
         raise ValueError("x must have unit stride along cin")
     groups = 1 if group_offsets is None else int(group_offsets.numel()) - 1
+    _check_xq(x, xq)
+    _check_stats(m, x, h, p, group_offsets, token_ids, groups)
     _check(load_library().lhcal_accumulate_noalloc(
         m, _dtype_id(x), _ptr(x), _ptr(xq), tokens, cin, _ld(x, cin), groups,
         _ptr(group_offsets), _ptr(token_ids), flags, _ptr(h), _ptr(p), _stream(stream)))
 
 
 def lhcal_count_tokens(counts, tokens: int = 0, group_offsets=None, flags: int = ACCUM_ADD, stream=None):
+    import torch
+
     groups = 1 if group_offsets is None else int(group_offsets.numel()) - 1
+    _need(counts, "counts", groups, torch.int64)
+    _need(group_offsets, "group_offsets", groups + 1, torch.int32)
     _check(load_library().lhcal_count_tokens(groups, tokens, _ptr(group_offsets), flags, _ptr(counts),
                                              _stream(stream)))
 
 
 def lhcal_finalize(mode, counts, h, p=None, stream=None):
+    import torch
+
     m = _mode_id(mode)
     groups = int(h.shape[0])
     cin = int(h.shape[1]) * BLOCK
+    _need(h, "h", _stats_numel(m, groups, cin), torch.float32)
+    if m == ACT_AWARE:
+        _need(p, "p", _stats_numel(m, groups, cin), torch.float32)
+    _need(counts, "counts", groups, torch.int64)
     _check(load_library().lhcal_finalize(m, groups, cin, _ptr(counts), _ptr(h), _ptr(p), _stream(stream)))
 
 
 def lhcal_global_scale(w, g, stream=None, fp8_max: float | None = None):
     """w: [groups, rows, cin] fp32/bf16; g: fp32 [groups]. fp8_max: 448 (default) or 256 (4/6)."""
     groups, rows, cin = (int(v) for v in w.shape)
+    _check_sweep_buffers(None, w, None, None, g, None, None, None)
     if fp8_max is None:
         _check(load_library().lhcal_global_scale(_dtype_id(w), _ptr(w), groups, rows, cin, _ptr(g), _stream(stream)))
     else:
@@ -215,7 +301,11 @@ def lhcal_global_scale(w, g, stream=None, fp8_max: float | None = None):
 
 def lhcal_multiplier_search(mode, w, h, g, multipliers, codes, wq=None, loss=None, p=None, stream=None):
     """Amax-multiplier search: multipliers fp32 device [M]; other tensors as lhcal_scale_sweep."""
+    import torch
+
     groups, rows, cin = (int(v) for v in w.shape)
+    _check_sweep_buffers(_mode_id(mode), w, h, p, g, codes, wq, loss)
+    _need(multipliers, "multipliers", 0, torch.float32)
     _check(load_library().lhcal_multiplier_search(
         _mode_id(mode), _dtype_id(w), _ptr(w), groups, rows, cin, _ptr(h), _ptr(p), _ptr(g), _ptr(multipliers),
         int(multipliers.numel()), _ptr(codes), _ptr(wq), _ptr(loss), _stream(stream)))
@@ -224,6 +314,7 @@ def lhcal_multiplier_search(mode, w, h, g, multipliers, codes, wq=None, loss=Non
 def lhcal_apply_scales(w, g, codes, wq=None, wq16=None, amax=None, stream=None):
     """Fake-quantized weights (fp32 wq, bf16 wq16) and per-block amax for chosen codes."""
     groups, rows, cin = (int(v) for v in w.shape)
+    _check_sweep_buffers(None, w, None, None, g, codes, wq, None, wq16=wq16, amax=amax)
     _check(load_library().lhcal_apply_scales(_dtype_id(w), _ptr(w), groups, rows, cin, _ptr(g), _ptr(codes),
                                              _ptr(wq), _ptr(wq16), _ptr(amax), _stream(stream)))
 
@@ -231,6 +322,7 @@ def lhcal_apply_scales(w, g, codes, wq=None, wq16=None, amax=None, stream=None):
 def lhcal_scale_sweep(mode, w, h, g, codes, wq=None, loss=None, p=None, stream=None):
     """w [G, R, C]; h/p finalized; g [G]; codes uint8 [G, R, C/16]; wq fp32 [G, R, C]; loss fp32 [G, R, C/16]."""
     groups, rows, cin = (int(v) for v in w.shape)
+    _check_sweep_buffers(_mode_id(mode), w, h, p, g, codes, wq, loss)
     _check(load_library().lhcal_scale_sweep(
         _mode_id(mode), _dtype_id(w), _ptr(w), groups, rows, cin, _ptr(h), _ptr(p), _ptr(g), _ptr(codes),
         _ptr(wq), _ptr(loss), _stream(stream)))

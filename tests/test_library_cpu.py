@@ -155,3 +155,87 @@ def test_buffers_size_the_workspace_for_either_activation_aware_entry_point(lib)
     m = L.Buffers("mse", 0, 64, 8, 2, L.BF16, "cpu")
     assert m.h is None and m.p is None and m.workspace is None
     assert tuple(m.codes.shape) == (2, 8, 4) and tuple(m.wq.shape) == (2, 8, 64)
+
+
+def test_binding_rejects_buffers_the_library_would_misread(lib):
+    """The C entry points take bare pointers, so the binding checks each tensor's dtype, density
+    and size against the call. A consistent call (CPU tensors here) reaches the library, which
+    refuses host pointers with an LhcalError; an inconsistent one stops in the binding first."""
+    import types
+
+    import torch
+
+    s = types.SimpleNamespace(cuda_stream=0)
+    x = torch.zeros((8, 32), dtype=torch.bfloat16)
+    h = torch.zeros((1, 2, 16, 16))
+    p = torch.zeros_like(h)
+    xq = torch.zeros_like(x)
+    with pytest.raises(L.LhcalError):
+        L.lhcal_accumulate("act", x, h, xq=xq, p=p, stream=s)
+    wide = torch.zeros((8, 48), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="row stride"):  # one ldx serves x and xq
+        L.lhcal_accumulate("act", x, h, xq=wide[:, :32], p=p, stream=s)
+    with pytest.raises(ValueError, match="must match"):
+        L.lhcal_accumulate("act", x, h, xq=xq.float(), p=p, stream=s)
+    with pytest.raises(ValueError, match="needs 512"):
+        L.lhcal_accumulate("full", x, h[:, :1], stream=s)
+    with pytest.raises(ValueError, match="needs 512"):
+        L.lhcal_accumulate_noalloc("act", x, h, xq=xq, p=p[:, :1], stream=s)
+    with pytest.raises(TypeError, match="float32"):
+        L.lhcal_accumulate("full", x, h.double(), stream=s)
+    with pytest.raises(L.LhcalError):  # DIAG statistics are [groups, cin/16, 16]
+        L.lhcal_accumulate("diag", x, torch.zeros((1, 2, 16)), stream=s)
+    offs = torch.tensor([0, 4, 8], dtype=torch.int32)
+    with pytest.raises(ValueError, match="needs 1024"):  # two groups
+        L.lhcal_accumulate("full", x, h, group_offsets=offs, token_ids=torch.zeros(8, dtype=torch.int32), stream=s)
+    with pytest.raises(TypeError, match="int32"):
+        L.lhcal_accumulate("full", x, torch.zeros((2, 2, 16, 16)), group_offsets=offs.long(),
+                           token_ids=torch.zeros(8, dtype=torch.int32), stream=s)
+    gx = torch.ones(1)
+    with pytest.raises(L.LhcalError):
+        L.lhcal_accumulate_act_quant(x, h, p, gx, stream=s)
+    with pytest.raises(TypeError, match="act_gx"):
+        L.lhcal_accumulate_act_quant(x, h, p, gx.double(), stream=s)
+    # The quantizer's output carries its own row stride, so a strided xq is fine there.
+    with pytest.raises(L.LhcalError):
+        L.lhcal_act_fake_quant(x, gx, wide[:, :32], stream=s)
+    with pytest.raises(ValueError, match="shaped like x"):
+        L.lhcal_act_fake_quant(x, gx, wide, stream=s)
+    with pytest.raises(TypeError, match="bfloat16"):
+        L.lhcal_act_fake_quant(x, gx, xq.float(), stream=s)
+    counts = torch.zeros(1, dtype=torch.int64)
+    with pytest.raises(TypeError, match="int64"):
+        L.lhcal_count_tokens(counts.int(), tokens=8, stream=s)
+    with pytest.raises(TypeError, match="int64"):
+        L.lhcal_finalize("full", counts.int(), h, stream=s)
+    with pytest.raises(ValueError, match="p has"):
+        L.lhcal_finalize("act", counts, h, p=p[:, :1], stream=s)
+
+    w = torch.zeros((2, 4, 32), dtype=torch.bfloat16)
+    hw = torch.zeros((2, 2, 16, 16))
+    g = torch.zeros(2)
+    codes = torch.zeros((2, 4, 2), dtype=torch.uint8)
+    wq = torch.zeros((2, 4, 32))
+    loss = torch.zeros((2, 4, 2))
+    with pytest.raises(L.LhcalError):
+        L.lhcal_scale_sweep("full", w, hw, g, codes, wq=wq, loss=loss, stream=s)
+    with pytest.raises(ValueError, match="w must be contiguous"):
+        L.lhcal_scale_sweep("full", w.transpose(1, 2).contiguous().transpose(1, 2), hw, g, codes, stream=s)
+    with pytest.raises(TypeError, match="uint8"):
+        L.lhcal_scale_sweep("full", w, hw, g, codes.to(torch.int8), stream=s)
+    with pytest.raises(ValueError, match="wq has"):
+        L.lhcal_scale_sweep("full", w, hw, g, codes, wq=wq[:1], stream=s)
+    with pytest.raises(ValueError, match="h has"):
+        L.lhcal_scale_sweep("act", w, hw[:1], g, codes, p=hw, stream=s)
+    with pytest.raises(ValueError, match="g has"):
+        L.lhcal_global_scale(w, g[:1], stream=s)
+    with pytest.raises(L.LhcalError):  # MSE reads no statistics
+        L.lhcal_scale_sweep("mse", w, None, g, codes, stream=s)
+    with pytest.raises(TypeError, match="multipliers"):
+        L.lhcal_multiplier_search("full", w, hw, g, torch.ones(4, dtype=torch.float64), codes, stream=s)
+    with pytest.raises(TypeError, match="wq16"):
+        L.lhcal_apply_scales(w, g, codes, wq16=wq, stream=s)
+    with pytest.raises(ValueError, match="amax has"):
+        L.lhcal_apply_scales(w, g, codes, amax=loss[:1], stream=s)
+    with pytest.raises(L.LhcalError):
+        L.lhcal_apply_scales(w, g, codes, wq=wq, wq16=wq.bfloat16(), amax=loss, stream=s)
