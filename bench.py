@@ -165,7 +165,7 @@ def algorithmic(layer):
     units = G * R * nblk
     ops = 126 * OPS_PER_CANDIDATE[layer.mode]
     hsz = G * nblk * (16 if layer.mode == "diag" else 256) * 4
-    xb = T * C * 2
+    xb = T * C * (4 if layer.dtype == "f32" else 2)
     if layer.mode == "act":  # X read once: X_q is derived from it inside the kernel
         acc_bytes = xb + 2 * hsz
     elif layer.token_ids is not None:

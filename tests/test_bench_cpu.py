@@ -1,0 +1,57 @@
+"""bench.py's host arithmetic: the roofline numerators at the workloads' full sizes.
+
+The units, sweep instructions and accumulation bytes that the bench divides by its measured
+times are checked here against figures worked out by hand from the shapes, so a change to the
+shapes or to the byte accounting cannot move a reported fraction unnoticed. The layers are
+shape-only stand-ins (nothing is generated), since the formula reads only sizes and routing.
+"""
+import types
+
+import numpy as np
+import pytest
+
+import bench
+from scale_calibration_lh_b200 import synth
+
+
+def _shape_only(name):
+    tokens, cin, rows, groups = synth.FULL_SIZES[name]
+    routed = groups > 1
+    return types.SimpleNamespace(
+        tokens=tokens, cin=cin, rows=rows, groups=groups, mode=synth.MODES[name],
+        dtype="f32" if name == "tiny" else "bf16",
+        token_ids=np.empty(tokens * synth.MOE_TOP_K, np.int32) if routed else None,
+        group_offsets=np.empty(groups + 1, np.int32) if routed else None)
+
+
+# name: (units, FP32 instructions per unit, accumulation bytes). Units = groups x rows x cin/16.
+# Per candidate: 136 FMA for the symmetric 16x16 quadratic (80 is the diagonal form's 32), 48 for
+# scale, dequantise and subtract, 16 for the cross term; times 126 candidates. Bytes: X once
+# (bf16, or fp32 for the tiny layer), each statistic written once (16x16 or 16 fp32 per block
+# and group), plus the CSR routing for the grouped layer. The activation-aware layer reads X
+# alone, its X_q being derived in the kernel, and writes H and P.
+EXPECTED = {
+    "tiny": (32 * 4, 126 * 184, 256 * 64 * 4 + 4 * 1024),
+    "dense": (4096 * 256, 126 * 184, 16384 * 4096 * 2 + 256 * 1024),
+    "act": (12288 * 256, 126 * 200, 32768 * 4096 * 2 + 2 * 256 * 1024),
+    "wmse": (4096 * 768, 126 * 80, 65536 * 12288 * 2 + 768 * 64),
+    "moe": (512 * 1280 * 160, 126 * 184, 16384 * 2560 * 2 + 512 * 160 * 1024 + 163840 * 4 + 513 * 4),
+}
+
+
+@pytest.mark.parametrize("name", sorted(EXPECTED))
+def test_roofline_numerators_at_full_size(name):
+    assert bench.algorithmic(_shape_only(name)) == EXPECTED[name]
+
+
+def test_numerators_in_the_units_quoted_for_each_workload():
+    # Per-workload figures as quoted: 1.05 M / 3.15 M / 3.15 M / 104.9 M units; 134.5 MB,
+    # 1.611 GB and 168.4 MB of accumulation traffic (the activation-aware figure is X alone).
+    u, _, b = bench.algorithmic(_shape_only("dense"))
+    assert (u, b) == (1_048_576, 134_479_872)
+    u, _, b = bench.algorithmic(_shape_only("wmse"))
+    assert (u, b) == (3_145_728, 1_610_661_888)
+    u, _, b = bench.algorithmic(_shape_only("moe"))
+    assert (u, b) == (104_857_600, 168_429_572)
+    u, _, b = bench.algorithmic(_shape_only("act"))
+    assert (u, b) == (3_145_728, 268_959_744)
