@@ -55,3 +55,44 @@ def test_numerators_in_the_units_quoted_for_each_workload():
     assert (u, b) == (104_857_600, 168_429_572)
     u, _, b = bench.algorithmic(_shape_only("act"))
     assert (u, b) == (3_145_728, 268_959_744)
+
+
+def _run_bench(args, env_extra=None):
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, **(env_extra or {}))
+    return subprocess.run([sys.executable, os.path.join(root, "bench.py")] + args, capture_output=True, text=True,
+                          timeout=600, cwd=root, env=env)
+
+
+def test_reference_arm_prints_one_contract_line():
+    """The reference arm times the oracle on a bounded sample and prints one JSON line with the
+    keys the benchmark contract names, in the native arm's metric and unit."""
+    import json
+
+    r = _run_bench(["--impl", "reference", "--steps", "1", "--warmup", "3"])
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == bench.UNIT
+    assert d["higher_is_better"] is True and d["steps"] == 1 and d["warmup"] == 3 and d["n_gpus"] == 1
+    assert d["value"] > 0 and d["ms_per_step"] > 0 and d["vs_baseline"] is None
+    assert d["dtype"] == "f64" and d["data"] == "synthetic" and "workload" in d["config"]
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_print_nothing():
+    r = _run_bench(["--impl", "reference", "--steps", "1", "--warmup", "3"],
+                   {"RANK": "1", "LOCAL_RANK": "1", "WORLD_SIZE": "2"})
+    assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_warmup_below_three_is_refused():
+    r = _run_bench(["--impl", "reference", "--steps", "1", "--warmup", "2"])
+    assert r.returncode != 0 and "warmup" in r.stderr
