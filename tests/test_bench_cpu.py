@@ -1,9 +1,12 @@
-"""bench.py's host arithmetic: the roofline numerators at the workloads' full sizes.
+"""bench.py's host logic, without a GPU.
 
-The units, sweep instructions and accumulation bytes that the bench divides by its measured
-times are checked here against figures worked out by hand from the shapes, so a change to the
-shapes or to the byte accounting cannot move a reported fraction unnoticed. The layers are
-shape-only stand-ins (nothing is generated), since the formula reads only sizes and routing.
+- The roofline numerators at the workloads' full sizes. The units, sweep instructions and
+  accumulation bytes that the bench divides by its measured times are checked against
+  figures worked out by hand from the shapes, so a change to the shapes or to the byte
+  accounting cannot move a reported fraction unnoticed. The layers are shape-only stand-ins
+  (nothing is generated), since the formula reads only sizes and routing.
+- The reference arm's JSON line, and the silence of its non-zero ranks.
+- The clock sampler, against a fake NVML (it only reads).
 """
 import types
 
@@ -96,3 +99,65 @@ def test_reference_arm_other_ranks_print_nothing():
 def test_warmup_below_three_is_refused():
     r = _run_bench(["--impl", "reference", "--steps", "1", "--warmup", "2"])
     assert r.returncode != 0 and "warmup" in r.stderr
+
+
+def _fake_nvml(clocks, reasons, seen, fail=False):
+    import itertools
+
+    ck, rs = itertools.cycle(clocks), itertools.cycle(reasons)
+
+    def init():
+        if fail:
+            raise RuntimeError("driver not loaded")
+
+    def handle(i):
+        seen.append(i)
+        return ("handle", i)
+
+    return types.SimpleNamespace(
+        NVML_CLOCK_SM=0, nvmlInit=init, nvmlDeviceGetHandleByIndex=handle,
+        nvmlDeviceGetMaxClockInfo=lambda h, c: 1965,
+        nvmlDeviceGetClockInfo=lambda h, c: next(ck),
+        nvmlDeviceGetCurrentClocksEventReasons=lambda h: next(rs),
+        nvmlClocksEventReasonHwSlowdown=0x8, nvmlClocksEventReasonHwThermalSlowdown=0x40,
+        nvmlClocksEventReasonSwThermalSlowdown=0x20, nvmlClocksEventReasonHwPowerBrakeSlowdown=0x80,
+        nvmlClocksEventReasonSwPowerCap=0x4)
+
+
+def _sample(sampler, n=12):
+    import time
+
+    sampler.start()
+    t0 = time.time()
+    while len(sampler.samples) < n and time.time() - t0 < 10:
+        time.sleep(0.005)
+    return sampler.stop()
+
+
+def test_clock_sampler_reports_median_clock_and_decoded_reasons(monkeypatch):
+    """Read-only NVML polling, checked against a fake NVML: median and minimum SM clock, the
+    union of the active reasons by name, and the physical index behind CUDA_VISIBLE_DEVICES."""
+    import sys
+
+    seen = []
+    monkeypatch.setitem(sys.modules, "pynvml", _fake_nvml([1800, 1965, 1965], [0x4, 0x0, 0x4 | 0x8], seen))
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "3,5")
+    out = _sample(bench.ClockSampler(1, period_s=0.001))
+    assert seen == [5]
+    assert out["sm_mhz"] == 1965 and out["sm_min_mhz"] == 1800 and out["sm_max_mhz"] == 1965
+    assert out["reasons"] == ["hw_slowdown", "sw_power_cap"] and out["samples"] >= 12
+
+
+def test_clock_sampler_without_nvml_says_so(monkeypatch):
+    import sys
+
+    monkeypatch.setitem(sys.modules, "pynvml", _fake_nvml([1965], [0], [], fail=True))
+    out = _sample(bench.ClockSampler(0), n=0)
+    assert out["sm_mhz"] is None and out["reasons"][0].startswith("nvml unavailable")
+
+
+def test_clock_reason_names_exist_in_the_installed_nvml_binding():
+    pynvml = pytest.importorskip("pynvml")
+    for _, const in bench.ClockSampler.REASONS:
+        assert isinstance(getattr(pynvml, const, None), int), const
+    assert callable(pynvml.nvmlDeviceGetCurrentClocksEventReasons)
