@@ -16,7 +16,6 @@ import pytest
 torch = pytest.importorskip("torch")
 
 import scale_calibration_lh_b200 as L  # noqa: E402
-from scale_calibration_lh_b200 import synth  # noqa: E402
 from tests import parity as P  # noqa: E402
 
 pytestmark = pytest.mark.gpu
