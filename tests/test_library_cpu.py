@@ -239,3 +239,17 @@ def test_binding_rejects_buffers_the_library_would_misread(lib):
         L.lhcal_apply_scales(w, g, codes, amax=loss[:1], stream=s)
     with pytest.raises(L.LhcalError):
         L.lhcal_apply_scales(w, g, codes, wq=wq, wq16=wq.bfloat16(), amax=loss, stream=s)
+
+
+def test_zero_token_calls_validate_as_the_header_states(lib):
+    """tokens = 0: one group accepts a NULL x (the next check to fail here is h, a host pointer
+    without a GPU); a grouped call still needs x; the two-tensor ACT_AWARE call still needs xq."""
+    host = ctypes.create_string_buffer(4096)
+    addr = ctypes.c_void_p((ctypes.addressof(host) + 255) // 256 * 256)
+    st = _call_accumulate(lib, tokens=0, x=None, h=addr, flags=1)
+    assert st in (L.ERR_INVALID_ARG, L.ERR_DEVICE_MISMATCH)
+    assert lib.lhcal_last_error_string().startswith(b"h")
+    st = _call_accumulate(lib, tokens=0, x=None, groups=2, offs=addr, ids=addr, h=addr, flags=1)
+    assert st == L.ERR_INVALID_ARG and lib.lhcal_last_error_string() == b"x is NULL"
+    st = _call_accumulate(lib, mode=L.ACT_AWARE, tokens=0, x=None, xq=None, h=addr, p=addr, flags=1)
+    assert st == L.ERR_INVALID_ARG and b"needs xq" in lib.lhcal_last_error_string()
