@@ -1,0 +1,205 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case plants one mistake in the oracle, on the CPU, by wrapping one of its functions: a
+dropped factor, a transposed or negated operand, another tie rule, a missing normalisation, an
+off-by-one candidate set. It then runs the pins named for that mistake. At least one pin must
+fail with an AssertionError; a crash does not count. The oracle resolves its helpers through
+the module at call time, so a mistake planted in ``e2m1_round`` also reaches ``fake_quant``,
+the sweep and the input quantizer. The pins' own references (exact rationals, ml_dtypes,
+torch's float8 decode) are built apart from the oracle and stay as they are.
+"""
+import numpy as np
+import pytest
+
+from oracle import lhcal_oracle as O
+from tests import test_golden as golden
+from tests import test_oracle_pins as pins
+
+# E2M1 midpoints and the two grid values around each.
+_MID = {0.25: (0.0, 0.5), 0.75: (0.5, 1.0), 1.25: (1.0, 1.5), 1.75: (1.5, 2.0), 2.5: (2.0, 3.0),
+        3.5: (3.0, 4.0), 5.0: (4.0, 6.0)}
+
+
+def _e2m1_on_ties(choose):
+    """E2M1 rounding whose exact ties take choose(lo, hi, even_choice) instead of the even value."""
+    def factory(orig):
+        def mutant(u):
+            u64 = np.minimum(np.asarray(u, dtype=np.float64), 6.0)
+            out = np.array(orig(u), dtype=np.float64, copy=True)
+            for m, (lo, hi) in _MID.items():
+                out = np.where(u64 == m, choose(lo, hi, out), out)
+            return out
+        return mutant
+    return factory
+
+
+def _e2m1_of_fp32_quotient(orig):
+    return lambda u: orig(np.asarray(u, dtype=np.float64).astype(np.float32).astype(np.float64))
+
+
+def _e4m3_ties_up(orig):
+    vals = np.concatenate([[0.0], O.e4m3_value(O.candidate_codes())])
+
+    def mutant(r):
+        r64 = np.asarray(r, dtype=np.float64)
+        out = np.asarray(orig(r))
+        hi = np.clip(np.searchsorted(vals, r64, side="left"), 1, len(vals) - 1)
+        return np.where(r64 == (vals[hi - 1] + vals[hi]) / 2, hi, out).astype(np.int64)
+    return mutant
+
+
+def _e4m3_truncating(orig):
+    vals = np.concatenate([[0.0], O.e4m3_value(O.candidate_codes())])
+
+    def mutant(r):
+        r64 = np.asarray(r, dtype=np.float64)
+        down = np.clip(np.searchsorted(vals, r64, side="right") - 1, 0, len(vals) - 1)
+        return np.where(r64 >= 448.0, len(vals) - 1, down).astype(np.int64)
+    return mutant
+
+
+def _act_hessians(change):
+    def factory(orig):
+        def mutant(x, xq):
+            h, p = orig(x, xq)
+            return change(h, p, x, orig)
+        return mutant
+    return factory
+
+
+def _cross_term(change):
+    def factory(orig):
+        def mutant(mode, w_blk, h_blk, p_blk, g):
+            if mode == "act":
+                p_blk = change(np.asarray(p_blk, dtype=np.float64))
+            return orig(mode, w_blk, h_blk, p_blk, g)
+        return mutant
+    return factory
+
+
+def _finalize(change):
+    def factory(orig):
+        def mutant(mode, h, p, counts):
+            hf, pf = orig(mode, h, p, counts)
+            hf = np.array(hf, copy=True)
+            for e, b in enumerate(np.asarray(counts)):
+                change(mode, hf, np.asarray(h, dtype=np.float64), e, int(b))
+            return hf, pf
+        return mutant
+    return factory
+
+
+def _raw_sums(mode, hf, h, e, b):
+    if b > 0 and mode != "diag":
+        hf[e] = h[e]
+
+
+def _diag_divided(mode, hf, h, e, b):
+    if b > 0 and mode == "diag":
+        hf[e] = h[e] / b
+
+
+def _no_fallback(mode, hf, h, e, b):
+    if b == 0:
+        hf[e] = 0.0
+
+
+def _highest_code_on_ties(orig):
+    def mutant(loss):
+        k, best, second = orig(np.asarray(loss)[:, ::-1])
+        return loss.shape[1] - 1 - k, best, second
+    return mutant
+
+
+def _apply_scales_amax_without_six(orig):
+    def mutant(w, g, codes):
+        wq, wq16, amax = orig(w, g, codes)
+        return wq, wq16, amax / 6.0
+    return mutant
+
+
+MUTANTS = {
+    "E2M1 ties to the odd value": (
+        "e2m1_round", _e2m1_on_ties(lambda lo, hi, even: lo + hi - even),
+        [lambda: pins.test_e2m1_midpoints_ties_to_even(0.25, 0), pins.test_fake_quant_exact_ties_and_neighbours,
+         golden.test_e2m1_cases]),
+    "E2M1 ties away from zero": (
+        "e2m1_round", _e2m1_on_ties(lambda lo, hi, even: hi),
+        [lambda: pins.test_e2m1_midpoints_ties_to_even(2.5, 2), pins.test_fake_quant_exact_ties_and_neighbours,
+         golden.test_e2m1_cases]),
+    "E2M1 of the fp32-rounded quotient": (
+        "e2m1_round", _e2m1_of_fp32_quotient, [pins.test_fake_quant_exact_ties_and_neighbours]),
+    "E4M3 ties to the larger code": (
+        "e4m3_round", _e4m3_ties_up,
+        [pins.test_e4m3_round_brute_force_and_library, pins.test_act_fake_quant_hand_worked_ties,
+         golden.test_e4m3_cases]),
+    "E4M3 by truncation": (
+        "e4m3_round", _e4m3_truncating, [pins.test_e4m3_round_brute_force_and_library, golden.test_e4m3_cases]),
+    "candidate codes shifted down by one": (
+        "candidate_codes", lambda orig: (lambda: orig() - 1), [pins.test_e4m3_candidates_match_torch_float8]),
+    "X_q left unrounded to bf16": (
+        "f32_to_bf16_values", lambda orig: (lambda v: np.asarray(v, dtype=np.float32)),
+        [lambda: pins.test_act_fake_quant_brute_force(1.0)]),
+    "fake quant drops the sign": (
+        "fake_quant", lambda orig: (lambda w, s: np.abs(orig(w, s))),
+        [pins.test_fake_quant_negative_zero_and_zero_scale, pins.test_fake_quant_exact_ties_and_neighbours]),
+    "fake quant loses -0": (
+        "fake_quant", lambda orig: (lambda w, s: orig(w, s) + np.float32(0.0)),
+        [pins.test_fake_quant_negative_zero_and_zero_scale]),
+    "P transposed": (
+        "hessian_sum_act", _act_hessians(lambda h, p, x, orig: (h, p.transpose(0, 2, 1))),
+        [pins.test_act_hessians_brute_force_and_properties]),
+    "P negated (X_q^T (X - X_q))": (
+        "hessian_sum_act", _act_hessians(lambda h, p, x, orig: (h, -p)),
+        [pins.test_act_hessians_brute_force_and_properties, pins.test_act_expanded_loss_equals_output_mse_including_negative]),
+    "activation-aware H taken from X": (
+        "hessian_sum_act", _act_hessians(lambda h, p, x, orig: (orig(x, x)[0], p)),
+        [pins.test_act_hessians_brute_force_and_properties, pins.test_act_expanded_loss_equals_output_mse_including_negative]),
+    "cross term without its factor 2": (
+        "candidate_losses", _cross_term(lambda p: 0.5 * p),
+        [pins.test_act_expanded_loss_equals_output_mse_including_negative]),
+    "cross term with P^T w": (
+        "candidate_losses", _cross_term(lambda p: p.transpose(0, 2, 1)),
+        [pins.test_act_expanded_loss_equals_output_mse_including_negative]),
+    "cross term negated": (
+        "candidate_losses", _cross_term(lambda p: -p),
+        [pins.test_act_expanded_loss_equals_output_mse_including_negative]),
+    "H and P left as raw sums (no 1/B)": (
+        "finalize", _finalize(_raw_sums), [pins.test_grouped_accumulate_and_zero_group_fallback]),
+    "importance divided by B": (
+        "finalize", _finalize(_diag_divided), [pins.test_grouped_accumulate_and_zero_group_fallback]),
+    "no fallback for a zero-token group": (
+        "finalize", _finalize(_no_fallback), [pins.test_grouped_accumulate_and_zero_group_fallback]),
+    "importance as a mean over tokens": (
+        "importance_sum", lambda orig: (lambda x: orig(x) / np.asarray(x).shape[0]),
+        [pins.test_hessian_symmetric_psd_and_diag_is_importance]),
+    "global scale over 448 instead of 6 * 448": (
+        "global_scale", lambda orig: (lambda w, fp8_max=448.0: np.float32(orig(w, fp8_max) * 6)),
+        [pins.test_global_scale_is_448_normalized]),
+    "global scale ignores the 4/6 normalization": (
+        "global_scale", lambda orig: (lambda w, fp8_max=448.0: orig(w)),
+        [pins.test_global_scale_four_over_six_is_256_normalized]),
+    "highest code wins a tie": (
+        "argmin_lowest", _highest_code_on_ties, [pins.test_sweep_is_exhaustive_lowest_code_on_ties]),
+    "exported amax without the factor 6": (
+        "apply_scales", _apply_scales_amax_without_six, [pins.test_apply_scales_matches_the_sweep_and_exact_amax]),
+}
+
+
+@pytest.mark.parametrize("name", list(MUTANTS))
+def test_planted_mistake_fails_a_pin(name, monkeypatch):
+    attr, factory, checks = MUTANTS[name]
+    monkeypatch.setattr(O, attr, factory(getattr(O, attr)))
+    caught = 0
+    for check in checks:
+        try:
+            check()
+        except AssertionError:
+            caught += 1
+    assert caught, f"no pin caught: {name}"
+
+
+def test_the_named_pins_pass_on_the_oracle_as_written():
+    for _, _, checks in MUTANTS.values():
+        for check in checks:
+            check()
