@@ -111,6 +111,28 @@ def _highest_code_on_ties(orig):
     return mutant
 
 
+def _gather_from_group_zero(which):
+    def factory(orig):
+        def mutant(mode, w, h, p, g, units):
+            wb, hb, pb, gu = orig(mode, w, h, p, g, units)
+            n = np.asarray(units, dtype=np.int64)[:, 2]
+            if which == "g":
+                gu = np.full_like(gu, np.asarray(g)[0])
+            elif h is not None:
+                hb = np.asarray(h)[0, n]
+            return wb, hb, pb, gu
+        return mutant
+    return factory
+
+
+def _routing_ignored(orig):
+    def mutant(mode, x, xq=None, group_offsets=None, token_ids=None, act_gx=None):
+        if token_ids is not None:
+            token_ids = np.arange(len(token_ids)) % np.asarray(x).shape[0]
+        return orig(mode, x, xq, group_offsets, token_ids, act_gx)
+    return mutant
+
+
 def _apply_scales_amax_without_six(orig):
     def mutant(w, g, codes):
         wq, wq16, amax = orig(w, g, codes)
@@ -181,6 +203,13 @@ MUTANTS = {
         [pins.test_global_scale_four_over_six_is_256_normalized]),
     "highest code wins a tie": (
         "argmin_lowest", _highest_code_on_ties, [pins.test_sweep_is_exhaustive_lowest_code_on_ties]),
+    "every group swept with group 0's global scale": (
+        "gather_units", _gather_from_group_zero("g"), [pins.test_grouped_calibrate_is_each_expert_on_its_own]),
+    "every group swept with group 0's H": (
+        "gather_units", _gather_from_group_zero("h"), [pins.test_grouped_calibrate_is_each_expert_on_its_own]),
+    "grouped accumulation ignores the routing": (
+        "accumulate", _routing_ignored,
+        [pins.test_grouped_accumulate_and_zero_group_fallback, pins.test_grouped_calibrate_is_each_expert_on_its_own]),
     "exported amax without the factor 6": (
         "apply_scales", _apply_scales_amax_without_six, [pins.test_apply_scales_matches_the_sweep_and_exact_amax]),
 }

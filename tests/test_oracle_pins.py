@@ -253,6 +253,29 @@ def test_grouped_accumulate_and_zero_group_fallback():
     np.testing.assert_array_equal(hdf[0], hd[0])  # importance stays a raw sum
 
 
+def test_grouped_calibrate_is_each_expert_on_its_own():
+    """A grouped layer is its experts calibrated one by one: each on its routed rows (PR #2864 /
+    #2840), with a global scale from its own weights, since every expert has its own weight
+    quantizer. Expert 1 gets no token and falls back to H = I."""
+    rng = np.random.default_rng(15)
+    x = rng.normal(size=(20, 32)).astype(np.float32)
+    w = (rng.normal(0, 0.05, (3, 4, 32)) * np.array([1.0, 7.0, 0.2])[:, None, None]).astype(np.float32)
+    off = np.array([0, 6, 6, 13], np.int32)
+    ids = np.concatenate([np.sort(rng.permutation(20)[:6]), np.sort(rng.permutation(20)[:7])]).astype(np.int32)
+    out = O.calibrate("full", x, w, group_offsets=off, token_ids=ids)
+    per = 4 * 2  # units per expert: rows x blocks
+    for e in range(3):
+        one = O.calibrate("full", x[ids[off[e]:off[e + 1]]], w[e:e + 1])
+        assert out["g"][e] == one["g"][0] == O.global_scale(w[e])
+        np.testing.assert_array_equal(out["h"][e], one["h"][0])
+        sl = slice(e * per, (e + 1) * per)
+        np.testing.assert_array_equal(out["codes"][sl], one["codes"])
+        np.testing.assert_array_equal(out["wq"][sl].view(np.int32), one["wq"].view(np.int32))
+        np.testing.assert_array_equal(out["loss"][sl], one["loss"])
+    assert len(set(out["g"].tolist())) == 3
+    np.testing.assert_array_equal(out["h"][1], np.broadcast_to(np.eye(16), (2, 16, 16)))
+
+
 # --------------------------------------------------------------------------- losses and sweep
 
 def _layer(seed, rows=6, cin=16, t=64):
