@@ -133,6 +133,24 @@ def _routing_ignored(orig):
     return mutant
 
 
+def _multiplier_codes(fp32_product=True, signed=True):
+    """The multiplier codes with one step changed; otherwise as the oracle states them."""
+    def factory(orig):
+        def mutant(w_blk, g, multipliers):
+            amax = np.abs(np.asarray(w_blk, dtype=np.float32).astype(np.float64)).max(axis=1)
+            m = np.asarray(multipliers, dtype=np.float32).astype(np.float64)
+            with np.errstate(invalid="ignore"):
+                a = m[None, :] * amax[:, None]
+                if fp32_product:
+                    a = a.astype(np.float32).astype(np.float64)
+            a = np.abs(a) if not signed else np.where(np.isnan(a) | (a < 0), 0.0, a)
+            a = np.where(np.isnan(a), 0.0, a)
+            g64 = np.float64(np.float32(g))
+            return np.zeros(a.shape, dtype=np.int64) if g64 == 0 else O.e4m3_round(a / (6.0 * g64))
+        return mutant
+    return factory
+
+
 def _apply_scales_amax_without_six(orig):
     def mutant(w, g, codes):
         wq, wq16, amax = orig(w, g, codes)
@@ -210,6 +228,11 @@ MUTANTS = {
     "grouped accumulation ignores the routing": (
         "accumulate", _routing_ignored,
         [pins.test_grouped_accumulate_and_zero_group_fallback, pins.test_grouped_calibrate_is_each_expert_on_its_own]),
+    "candidate amax not rounded to fp32": (
+        "multiplier_codes", _multiplier_codes(fp32_product=False),
+        [pins.test_multiplier_codes_round_the_candidate_amax_to_fp32]),
+    "negative multiplier taken by magnitude": (
+        "multiplier_codes", _multiplier_codes(signed=False), [pins.test_multiplier_codes_by_exact_rationals]),
     "exported amax without the factor 6": (
         "apply_scales", _apply_scales_amax_without_six, [pins.test_apply_scales_matches_the_sweep_and_exact_amax]),
 }

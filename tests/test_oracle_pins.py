@@ -496,6 +496,20 @@ def test_multiplier_codes_by_exact_rationals():
     assert np.all(O.multiplier_codes(w, np.float32(0.0), m) == 0)
 
 
+def test_multiplier_codes_round_the_candidate_amax_to_fp32():
+    """The candidate amax is the fp32 product m * amax, as the quantizer holds its amax in fp32.
+    Worked by hand: g = 2^-3, so 6g = 0.75 and the E4M3 tie 1.0625 (between 1.0 = 0x38 and
+    1.125 = 0x39) is a candidate amax of 0.796875. With amax = 1 + 2^-22 and
+    m = 0.796875 - 3 * 2^-24 the exact product is 0.796875 + (0.1875 - 6 * 2^-23) * 2^-24, above
+    the tie by less than half an fp32 ulp (2^-25). It rounds to 0.796875 exactly, and the tie
+    goes to the even code 0x38; the unrounded product would give 0x39."""
+    amax, m = np.float32(1 + 2 ** -22), np.float32(0.796875 - 3 * 2 ** -24)
+    assert float(amax) == 1 + 2 ** -22 and float(m) == 0.796875 - 3 * 2 ** -24
+    w = np.zeros((1, 16), np.float32)
+    w[0, 3] = -amax
+    assert O.multiplier_codes(w, np.float32(0.125), np.array([m, 1.0], np.float32)).tolist() == [[0x38, 0x3B]]
+
+
 @pytest.mark.parametrize("mode", ["full", "diag", "mse"])
 def test_dense_multipliers_reproduce_the_sweep(mode):
     """Multipliers so dense that every code 1..126 is some multiplier's code: the search then
