@@ -151,6 +151,18 @@ def _multiplier_codes(fp32_product=True, signed=True):
     return factory
 
 
+def _loss_scale_signed(orig):
+    def mutant(mode, w_blk, h_blk, p_blk):
+        if mode not in ("full", "act"):
+            return orig(mode, w_blk, h_blk, p_blk)
+        w = np.asarray(w_blk, dtype=np.float64)
+        s = np.einsum("ui,uij,uj->u", w, np.asarray(h_blk, dtype=np.float64), w)
+        if mode == "act":
+            s = s + 2.0 * np.abs(np.einsum("ui,uij,uj->u", w, np.asarray(p_blk, dtype=np.float64), w))
+        return s
+    return mutant
+
+
 def _apply_scales_amax_without_six(orig):
     def mutant(w, g, codes):
         wq, wq16, amax = orig(w, g, codes)
@@ -233,6 +245,17 @@ MUTANTS = {
         [pins.test_multiplier_codes_round_the_candidate_amax_to_fp32]),
     "negative multiplier taken by magnitude": (
         "multiplier_codes", _multiplier_codes(signed=False), [pins.test_multiplier_codes_by_exact_rationals]),
+    "loss scale from signed weights and H": (
+        "loss_scale", _loss_scale_signed, [pins.test_loss_scale_bounds_every_candidate_and_sees_only_magnitudes]),
+    "loss scale without the cross term": (
+        "loss_scale", lambda orig: (lambda mode, w, h, p: orig("full" if mode == "act" else mode, w, h, None)),
+        [pins.test_loss_scale_bounds_every_candidate_and_sees_only_magnitudes]),
+    "input quantizer ignores its global scale": (
+        "act_fake_quant", lambda orig: (lambda x, gx, rows_per_chunk=1024: orig(x, np.float32(1.0), rows_per_chunk)),
+        [lambda: pins.test_act_fake_quant_brute_force(1e-3), pins.test_act_fake_quant_saturates_and_zero_global_scale]),
+    "E4M3 without saturation (NaN code above 448)": (
+        "e4m3_round", lambda orig: (lambda r: np.where(np.asarray(r, dtype=np.float64) > 464.0, 127, orig(r))),
+        [pins.test_e4m3_round_brute_force_and_library, golden.test_e4m3_cases]),
     "exported amax without the factor 6": (
         "apply_scales", _apply_scales_amax_without_six, [pins.test_apply_scales_matches_the_sweep_and_exact_amax]),
 }

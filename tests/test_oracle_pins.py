@@ -456,6 +456,30 @@ def test_loss_scale_bounds_e0_and_equals_it_for_diagonal_h():
     np.testing.assert_allclose(O.loss_scale("diag", w, imp, None), e0d, rtol=1e-13)
 
 
+def test_loss_scale_bounds_every_candidate_and_sees_only_magnitudes():
+    """Rounding to the nearest E2M1 point, or saturating, never moves a weight by more than its
+    magnitude: |dW_i| <= |w_i| for every candidate. Hence |L_k| <= |w|^T |H| |w| (+ 2 |w|^T |P| |w|)
+    = S for all 126 k. S depends on magnitudes only: flipping the signs of weights or of H and P
+    entries leaves it unchanged; and the cross term adds to it whenever P is not zero."""
+    rng = np.random.default_rng(16)
+    w = rng.normal(0, 0.05, (40, 16)).astype(np.float32)
+    a = rng.normal(size=(40, 16, 16))
+    h = a @ a.transpose(0, 2, 1) / 16
+    p = 0.3 * rng.normal(size=(40, 16, 16))
+    g = O.global_scale(w)
+    for mode, pp in (("full", None), ("act", p)):
+        loss, wq, _ = O.candidate_losses(mode, w, h, pp, g)
+        dw = wq.astype(np.float64) - w.astype(np.float64)[:, None, :]
+        assert np.all(np.abs(dw) <= np.abs(w.astype(np.float64))[:, None, :])
+        s = O.loss_scale(mode, w, h, pp)
+        assert np.all(np.abs(loss) <= s[:, None] * (1 + 1e-12))
+        flip = rng.choice([-1.0, 1.0], w.shape).astype(np.float32)
+        hs = h * rng.choice([-1.0, 1.0], h.shape)
+        ps = None if pp is None else pp * rng.choice([-1.0, 1.0], pp.shape)
+        np.testing.assert_array_equal(O.loss_scale(mode, w * flip, hs, ps), s)
+    assert np.all(O.loss_scale("act", w, h, p) > O.loss_scale("full", w, h, None))
+
+
 # --------------------------------------------------------------------------- amax-multiplier search
 
 @pytest.mark.parametrize("mode", ["full", "act", "diag", "mse"])
