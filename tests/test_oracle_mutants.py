@@ -163,6 +163,19 @@ def _loss_scale_signed(orig):
     return mutant
 
 
+def _quadratic_of_wq(orig):
+    def mutant(mode, w_blk, h_blk, p_blk, g):
+        loss, wq, e0 = orig(mode, w_blk, h_blk, p_blk, g)
+        if mode in ("full", "act"):
+            w64, q64 = np.asarray(w_blk, dtype=np.float64), wq.astype(np.float64)
+            loss = np.einsum("uki,uij,ukj->uk", q64, np.asarray(h_blk, dtype=np.float64), q64)
+            if mode == "act":
+                pw = np.einsum("uij,uj->ui", np.asarray(p_blk, dtype=np.float64), w64)
+                loss = loss + 2.0 * np.einsum("uki,ui->uk", q64 - w64[:, None, :], pw)
+        return loss, wq, e0
+    return mutant
+
+
 def _apply_scales_amax_without_six(orig):
     def mutant(w, g, codes):
         wq, wq16, amax = orig(w, g, codes)
@@ -256,6 +269,19 @@ MUTANTS = {
     "E4M3 without saturation (NaN code above 448)": (
         "e4m3_round", lambda orig: (lambda r: np.where(np.asarray(r, dtype=np.float64) > 464.0, 127, orig(r))),
         [pins.test_e4m3_round_brute_force_and_library, golden.test_e4m3_cases]),
+    "DIAG loss weighted by Imp squared": (
+        "candidate_losses",
+        lambda orig: (lambda mode, w, h, p, g: orig(mode, w, np.asarray(h) ** 2 if mode == "diag" else h, p, g)),
+        [pins.test_wmse_equals_full_with_diagonal_hessian]),
+    "MSE loss doubled": (
+        "candidate_losses",
+        lambda orig: (lambda mode, w, h, p, g: orig("diag", w, np.full(np.shape(w), 2.0), None, g)
+                      if mode == "mse" else orig(mode, w, h, p, g)),
+        [pins.test_mse_mode_is_plain_block_mse_by_exact_rationals_and_equals_identity_hessian]),
+    "quadratic form of Wq instead of dW": (
+        "candidate_losses", _quadratic_of_wq,
+        [pins.test_act_expanded_loss_equals_output_mse_including_negative,
+         pins.test_identity_hessian_is_plain_block_mse_by_exact_rationals]),
     "exported amax without the factor 6": (
         "apply_scales", _apply_scales_amax_without_six, [pins.test_apply_scales_matches_the_sweep_and_exact_amax]),
 }
