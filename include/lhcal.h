@@ -127,14 +127,17 @@ lhcal_status lhcal_act_fake_quant(lhcal_dtype dtype, const void* x, int64_t toke
 
 /*
  * Bytes of workspace lhcal_accumulate_act_quant needs for these sizes (0 is possible).
- * Host-only computation; needs no GPU. dtype must be LHCAL_BF16.
+ * Host-only computation; needs no GPU. dtype must be LHCAL_BF16 (LHCAL_ERR_UNSUPPORTED
+ * otherwise); a bad cin, groups or tokens is LHCAL_ERR_INVALID_ARG, as for
+ * lhcal_accumulate_workspace.
  */
 lhcal_status lhcal_accumulate_act_quant_workspace(lhcal_dtype dtype, int64_t tokens, int64_t cin, int32_t groups,
                                                   size_t* bytes);
 
 /*
- * Activation-aware accumulation (lhcal_accumulate with LHCAL_ACT_AWARE) with the input
- * quantizer fused: X_q is not read from memory but derived from x inside the kernel exactly as
+ * Activation-aware accumulation (PR #1976, "What does this PR do?": H and P from the input
+ * quantizer's output X_q; re-review: X_q is what that quantizer produces), i.e. lhcal_accumulate
+ * with LHCAL_ACT_AWARE, with the input quantizer fused: X_q is not read from memory but derived from x inside the kernel exactly as
  * lhcal_act_fake_quant computes it, so the activations are read once. The sums are those of
  * lhcal_act_fake_quant followed by lhcal_accumulate(LHCAL_ACT_AWARE, ...) with that X_q, up to
  * the fp32 summation order (the two may split the tokens differently; grouped sums and equal
@@ -144,6 +147,7 @@ lhcal_status lhcal_accumulate_act_quant_workspace(lhcal_dtype dtype, int64_t tok
  *           it is an input because the quantizer's amax is calibrated before the capture.
  *   other arguments as for lhcal_accumulate with mode LHCAL_ACT_AWARE; the workspace size is
  *   lhcal_accumulate_act_quant_workspace(LHCAL_BF16, tokens, cin, groups).
+ * Errors as for lhcal_accumulate; a NULL act_gx is LHCAL_ERR_INVALID_ARG.
  */
 lhcal_status lhcal_accumulate_act_quant(lhcal_dtype dtype, const void* x, int64_t tokens, int64_t cin,
                                         int64_t ldx, int32_t groups, const int32_t* group_offsets,
@@ -152,9 +156,11 @@ lhcal_status lhcal_accumulate_act_quant(lhcal_dtype dtype, const void* x, int64_
                                         void* stream);
 
 /*
- * Token counts B per group: counts[e] (+)= offsets[e+1] - offsets[e], or counts[0] (+)= tokens
- * when group_offsets is NULL (groups must then be 1). counts: device int64 [groups].
- * flags as for lhcal_accumulate.
+ * Token counts B per group, the B of "/B" (PR #1976) counted per expert over its routed tokens
+ * (PR #2864 / #2840): counts[e] (+)= offsets[e+1] - offsets[e], or counts[0] (+)= tokens when
+ * group_offsets is NULL. counts: device int64 [groups], 8-byte aligned. flags as for
+ * lhcal_accumulate. Errors: groups outside [1, 65535], groups > 1 without group_offsets,
+ * negative tokens or unknown flags are LHCAL_ERR_INVALID_ARG.
  */
 lhcal_status lhcal_count_tokens(int32_t groups, int64_t tokens, const int32_t* group_offsets,
                                 int32_t flags, int64_t* counts, void* stream);
