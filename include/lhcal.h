@@ -93,10 +93,11 @@ lhcal_status lhcal_accumulate_workspace(lhcal_mode mode, lhcal_dtype dtype, int6
  *   workspace: device scratch of at least lhcal_accumulate_workspace() bytes, 256-byte
  *             aligned; may be NULL when that size is 0. Its contents need no initialisation.
  * tokens = 0 with one group: x may be NULL (ACT_AWARE still takes a non-NULL xq, which is not
- * read); OVERWRITE writes zero sums, ADD leaves h and p as they are. A grouped call needs x, group_offsets and token_ids as device pointers
- * even when it routes no token, since the offsets live on the device and the host cannot see
- * that no row will be read; a NULL one is LHCAL_ERR_INVALID_ARG. A caller with an empty
- * grouped batch skips the call (ADD) or zeroes h and p itself (OVERWRITE).
+ * read); OVERWRITE writes zero sums, ADD leaves h and p as they are. A grouped call needs x,
+ * group_offsets and token_ids as device pointers even when it routes no token, since the
+ * offsets live on the device and the host cannot see that no row will be read; a NULL one is
+ * LHCAL_ERR_INVALID_ARG. A caller with an empty grouped batch skips the call (ADD) or zeroes
+ * h and p itself (OVERWRITE).
  * Results are deterministic for fixed sizes (fixed summation order). bf16 products are exact
  * in fp32; sums are fp32.
  */
