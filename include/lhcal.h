@@ -137,9 +137,10 @@ lhcal_status lhcal_accumulate_act_quant_workspace(lhcal_dtype dtype, int64_t tok
 
 /*
  * Activation-aware accumulation (PR #1976, "What does this PR do?": H and P from the input
- * quantizer's output X_q; re-review: X_q is what that quantizer produces), i.e. lhcal_accumulate
- * with LHCAL_ACT_AWARE, with the input quantizer fused: X_q is not read from memory but derived from x inside the kernel exactly as
- * lhcal_act_fake_quant computes it, so the activations are read once. The sums are those of
+ * quantizer's output X_q; re-review: X_q is what that quantizer produces), i.e.
+ * lhcal_accumulate with LHCAL_ACT_AWARE, with the input quantizer fused: X_q is not read from
+ * memory but derived from x inside the kernel exactly as lhcal_act_fake_quant computes it, so
+ * the activations are read once. The sums are those of
  * lhcal_act_fake_quant followed by lhcal_accumulate(LHCAL_ACT_AWARE, ...) with that X_q, up to
  * the fp32 summation order (the two may split the tokens differently; grouped sums and equal
  * splits give identical bits).
