@@ -253,3 +253,17 @@ def test_zero_token_calls_validate_as_the_header_states(lib):
     assert st == L.ERR_INVALID_ARG and lib.lhcal_last_error_string() == b"x is NULL"
     st = _call_accumulate(lib, mode=L.ACT_AWARE, tokens=0, x=None, xq=None, h=addr, p=addr, flags=1)
     assert st == L.ERR_INVALID_ARG and b"needs xq" in lib.lhcal_last_error_string()
+
+
+def test_token_count_and_fused_workspace_errors_as_documented(lib):
+    ct = lib.lhcal_count_tokens
+    for groups, tokens, flags in ((0, 5, 0), (65536, 5, 0), (2, 5, 0), (1, -1, 0), (1, 5, 7)):
+        assert ct(groups, tokens, None, flags, None, None) == L.ERR_INVALID_ARG, (groups, tokens, flags)
+    n = ctypes.c_size_t(0)
+    q = lib.lhcal_accumulate_act_quant_workspace
+    assert q(L.F32, 100, 32, 1, ctypes.byref(n)) == L.ERR_UNSUPPORTED
+    assert q(L.BF16, 100, 24, 1, ctypes.byref(n)) == L.ERR_INVALID_ARG
+    assert q(L.BF16, 100, 32, 0, ctypes.byref(n)) == L.ERR_INVALID_ARG
+    assert q(L.BF16, -1, 32, 1, ctypes.byref(n)) == L.ERR_INVALID_ARG
+    assert q(L.BF16, 100, 32, 1, None) == L.ERR_INVALID_ARG
+    assert q(L.BF16, 0, 32, 1, ctypes.byref(n)) == L.OK
