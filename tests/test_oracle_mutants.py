@@ -282,6 +282,24 @@ MUTANTS = {
         "candidate_losses", _quadratic_of_wq,
         [pins.test_act_expanded_loss_equals_output_mse_including_negative,
          pins.test_identity_hessian_is_plain_block_mse_by_exact_rationals]),
+    "E4M3 subnormals decoded with the normal exponent bias": (
+        "e4m3_value",
+        lambda orig: (lambda code: np.where((np.asarray(code) >> 3) == 0, orig(code) * 8.0, orig(code))),
+        [pins.test_e4m3_candidates_match_torch_float8]),
+    "candidate scales in descending order": (
+        "candidate_scales", lambda orig: (lambda g: orig(g)[::-1].copy()),
+        [pins.test_global_scale_is_448_normalized]),
+    "full Hessian drops the last token": (
+        "hessian_sum_full", lambda orig: (lambda x: orig(np.asarray(x)[:-1])),
+        [pins.test_full_hessian_brute_force]),
+    "codes above 126 applied as zero": (
+        "apply_scales",
+        lambda orig: (lambda w, g, codes: orig(w, g, np.where(np.asarray(codes) > 126, 0, codes).astype(np.uint8))),
+        [pins.test_apply_scales_matches_the_sweep_and_exact_amax]),
+    "losses for scales evaluated on reversed scales": (
+        "losses_for_scales",
+        lambda orig: (lambda mode, w, h, p, s: orig(mode, w, h, p, np.asarray(s)[:, ::-1].copy())),
+        [lambda: pins.test_losses_for_scales_is_candidate_losses_at_the_candidate_scales("full")]),
     "exported amax without the factor 6": (
         "apply_scales", _apply_scales_amax_without_six, [pins.test_apply_scales_matches_the_sweep_and_exact_amax]),
 }
