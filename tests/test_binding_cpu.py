@@ -6,7 +6,9 @@ size. The checks are:
 - each mode's calls, in order: MSE takes no statistics, and ``act`` uses the fused entry point
   only when given the global scale and no X_q;
 - the sizes, flags and pointers each call receives;
-- the binding's own buffer checks accept everything ``calibrate`` allocates.
+- the binding's own buffer checks accept everything ``calibrate`` allocates;
+- ``calibrate_host`` stages the inputs, takes the statistics once and pipelines global scales,
+  sweeps and result copies over chunks of groups (streams and events faked, copies at once).
 """
 import ctypes
 
@@ -120,3 +122,80 @@ def test_diag_statistics_are_one_vector_per_block(fake):
     assert tuple(b.h.shape) == (1, 3, 16) and b.p is None
     (sw,) = fake.args("lhcal_scale_sweep")
     assert sw[0] == L.DIAG and _ptr(sw[6]) == b.h.data_ptr()
+
+
+class _FakeStream:
+    def wait_stream(self, other):
+        pass
+
+    def wait_event(self, event):
+        pass
+
+
+class _FakeEvent:
+    def record(self, stream=None):
+        pass
+
+
+@pytest.fixture
+def fake_streams(monkeypatch):
+    """Streams and events that only accept the ordering calls; copies run on the CPU at once."""
+    import contextlib
+
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda device=None: _FakeStream())
+    monkeypatch.setattr(torch.cuda, "Stream", lambda device=None: _FakeStream())
+    monkeypatch.setattr(torch.cuda, "Event", lambda *a, **k: _FakeEvent())
+    monkeypatch.setattr(torch.cuda, "stream", lambda s: contextlib.nullcontext())
+    monkeypatch.setattr(L, "_side_streams", {})
+
+
+def _host_outputs(b):
+    out = object.__new__(L.HostOutputs)  # plain CPU tensors in place of pinned ones
+    out.codes = torch.full(b.codes.shape, 255, dtype=torch.uint8)
+    out.loss = torch.full(b.loss.shape, -1.0)
+    out.wq = None
+    return out
+
+
+def test_calibrate_host_pipelines_groups_in_chunks(fake, fake_streams):
+    G, R, C, T = 10, 4, 32, 40
+    x = torch.randn(T, C).bfloat16()
+    w = torch.randn(G, R, C).bfloat16()
+    offs = torch.tensor([0, 4, 8, 8, 12, 16, 20, 24, 28, 34, 40], dtype=torch.int32)
+    ids = torch.from_numpy(np.arange(T, dtype=np.int32))
+    b = L.Buffers("full", T, C, R, G, L.BF16, "cpu")
+    b.codes.copy_(torch.arange(b.codes.numel(), dtype=torch.int64).remainder(127).to(torch.uint8).view(b.codes.shape))
+    b.loss.copy_(torch.arange(b.loss.numel(), dtype=torch.float32).view(b.loss.shape))
+    staging = {"x": torch.empty_like(x), "w": torch.empty_like(w), "offs": torch.empty_like(offs),
+               "ids": torch.empty_like(ids)}
+    fake.calls.clear()  # the workspace query of Buffers
+    out = L.calibrate_host("full", x, w, b, staging, group_offsets=offs, token_ids=ids, out=_host_outputs(b),
+                           group_chunks=4)
+    # Statistics once over all tokens from the staged copies, then scale and sweep per chunk.
+    assert fake.names()[:3] == ["lhcal_accumulate", "lhcal_count_tokens", "lhcal_finalize"]
+    (acc,) = fake.args("lhcal_accumulate")
+    assert _ptr(acc[2]) == staging["x"].data_ptr() and _ptr(acc[8]) == staging["offs"].data_ptr() and acc[7] == G
+    assert torch.equal(staging["x"], x) and torch.equal(staging["w"], w) and torch.equal(staging["ids"], ids)
+    bounds = [0, 2, 5, 7, 10]  # groups * j // chunks
+    scales, sweeps = fake.args("lhcal_global_scale"), fake.args("lhcal_scale_sweep")
+    assert [a[2] for a in scales] == [e1 - e0 for e0, e1 in zip(bounds, bounds[1:])]
+    for (e0, _), sc, sw in zip(zip(bounds, bounds[1:]), scales, sweeps):
+        assert _ptr(sc[1]) == staging["w"][e0].data_ptr() and _ptr(sc[5]) == b.g[e0].data_ptr()
+        assert _ptr(sw[2]) == staging["w"][e0].data_ptr() and _ptr(sw[6]) == b.h[e0].data_ptr()
+        assert _ptr(sw[9]) == b.codes[e0].data_ptr() and _ptr(sw[11]) == b.loss[e0].data_ptr()
+    # Every group's results came back.
+    assert torch.equal(out.codes, b.codes) and torch.equal(out.loss, b.loss)
+
+
+def test_calibrate_host_reads_xq_only_when_the_caller_copies_it_in(fake, fake_streams):
+    T, C, R = 48, 32, 8
+    x, w, hxq = torch.randn(T, C).bfloat16(), torch.randn(1, R, C).bfloat16(), torch.randn(T, C).bfloat16()
+    b = L.Buffers("act", T, C, R, 1, L.BF16, "cpu")
+    staging = {"x": torch.empty_like(x), "w": torch.empty_like(w), "xq": torch.empty_like(hxq)}
+    gx = torch.ones(1)
+    L.calibrate_host("act", x, w, b, staging, out=_host_outputs(b), act_gx=gx)
+    assert "lhcal_accumulate_act_quant" in fake.names() and "lhcal_accumulate" not in fake.names()
+    fake.calls.clear()
+    L.calibrate_host("act", x, w, b, staging, hxq=hxq, out=_host_outputs(b))
+    (acc,) = fake.args("lhcal_accumulate")
+    assert _ptr(acc[3]) == staging["xq"].data_ptr() and torch.equal(staging["xq"], hxq)
