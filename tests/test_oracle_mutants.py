@@ -176,6 +176,28 @@ def _quadratic_of_wq(orig):
     return mutant
 
 
+def _act_quant_amax_over_32(orig):
+    """The input quantizer with its block amax taken over two neighbouring blocks (32 values)."""
+    def mutant(x, gx, rows_per_chunk=1024):
+        x64 = np.asarray(x, dtype=np.float64)
+        t, c = x64.shape
+        gx64 = np.float64(np.float32(gx))
+        blk = np.abs(x64).reshape(t, c // 16, 16).max(axis=-1)
+        n2 = blk.shape[1] - blk.shape[1] % 2  # pairs of neighbouring blocks; a lone last block keeps its own
+        pm = np.maximum(blk[:, 0:n2:2], blk[:, 1:n2:2])
+        blk[:, 0:n2:2], blk[:, 1:n2:2] = pm, pm
+        amax = blk[..., None]
+        code = O.e4m3_round(amax / (6.0 * gx64)) if gx64 > 0 else np.zeros(amax.shape, np.int64)
+        v = np.where(code > 0, O.e4m3_value(np.maximum(code, 1)), 0.0)
+        s = (v * gx64).astype(np.float32).astype(np.float64)
+        xb = x64.reshape(t, c // 16, 16)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            u = np.where(s > 0, np.abs(xb) / np.where(s > 0, s, 1.0), 0.0)
+        mag = O.f32_to_bf16_values((O.e2m1_round(u) * s).astype(np.float32))
+        return np.copysign(mag, xb).reshape(t, c).astype(np.float32)
+    return mutant
+
+
 def _apply_scales_amax_without_six(orig):
     def mutant(w, g, codes):
         wq, wq16, amax = orig(w, g, codes)
@@ -300,6 +322,12 @@ MUTANTS = {
         "losses_for_scales",
         lambda orig: (lambda mode, w, h, p, s: orig(mode, w, h, p, np.asarray(s)[:, ::-1].copy())),
         [lambda: pins.test_losses_for_scales_is_candidate_losses_at_the_candidate_scales("full")]),
+    "input quantizer amax over 32 values": (
+        "act_fake_quant", _act_quant_amax_over_32,
+        [lambda: pins.test_act_fake_quant_brute_force(1.0), golden.test_activation_blocks]),
+    "Hessian kept in fp32": (
+        "hessian_sum_full", lambda orig: (lambda x: orig(x).astype(np.float32).astype(np.float64)),
+        [pins.test_full_hessian_brute_force]),
     "exported amax without the factor 6": (
         "apply_scales", _apply_scales_amax_without_six, [pins.test_apply_scales_matches_the_sweep_and_exact_amax]),
 }
