@@ -267,7 +267,8 @@ MUTANTS = {
         "global_scale", lambda orig: (lambda w, fp8_max=448.0: orig(w)),
         [pins.test_global_scale_four_over_six_is_256_normalized]),
     "highest code wins a tie": (
-        "argmin_lowest", _highest_code_on_ties, [pins.test_sweep_is_exhaustive_lowest_code_on_ties]),
+        "argmin_lowest", _highest_code_on_ties,
+        [pins.test_sweep_is_exhaustive_lowest_code_on_ties, golden.test_sweep_winners]),
     "every group swept with group 0's global scale": (
         "gather_units", _gather_from_group_zero("g"), [pins.test_grouped_calibrate_is_each_expert_on_its_own]),
     "every group swept with group 0's H": (
