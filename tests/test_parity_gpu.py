@@ -753,3 +753,30 @@ def test_multiplier_search_counts(n_mult):
     ref = O.multiplier_search("full", w32, h, None, g, mult, units)
     gc, gw, gl = P.gather_gpu_units(codes, wq, loss, units)
     P.check_sweep(gc, gw, gl, ref, f"multiplier search, {n_mult} multipliers")
+
+
+def test_golden_sweep_winners_on_the_gpu():
+    """The hand-derived sweep winners of tests/golden (plain block MSE, one block per group, each
+    group with its own g): the CUDA sweep returns the same codes, zero losses and Wq = W."""
+    from tests import test_golden as G
+
+    cases = G._cases()["sweep"]
+    gs, ws, want = [], [], []
+    for rest in cases:
+        lhs, rhs = rest.split("->")
+        vals = lhs.split()
+        gs.append(np.float32(vals[0]))
+        ws.append(np.array([float(v) for v in vals[1:]], np.float32))
+        code, loss = rhs.split()
+        want.append((int(code, 16), float(loss)))
+    n = len(cases)
+    w = P.to_device(np.stack(ws)[:, None, :], "f32")  # [groups, 1 row, 16]
+    g = P.to_device(np.array(gs, np.float32), "f32")
+    codes = torch.empty((n, 1, 1), dtype=torch.uint8, device="cuda")
+    wq = torch.empty((n, 1, 16), dtype=torch.float32, device="cuda")
+    loss = torch.empty((n, 1, 1), dtype=torch.float32, device="cuda")
+    L.lhcal_scale_sweep("mse", w, None, g, codes, wq=wq, loss=loss)
+    _sync()
+    assert codes.flatten().tolist() == [c for c, _ in want]
+    assert loss.flatten().tolist() == [v for _, v in want]
+    np.testing.assert_array_equal(wq.cpu().numpy().reshape(n, 16).view(np.int32), np.stack(ws).view(np.int32))
