@@ -55,7 +55,8 @@ FP8_MAX = 448.0
 # ---------------------------------------------------------------------------------------
 
 def e4m3_value(code) -> np.ndarray:
-    """Value of an E4M3 byte with sign bit 0 (OCP FP8: 4 exponent bits, bias 7, 3 mantissa bits).
+    """Value of an E4M3 byte with sign bit 0 (OCP FP8: 4 exponent bits, bias 7, 3 mantissa bits);
+    the block-scale format of "Add WMSE weight scale search calibration" (PR #2283), How.
 
     e = code >> 3, m = code & 7; e == 0 is subnormal m * 2^-9, else (1 + m/8) * 2^(e-7).
     Codes 0x01..0x7E are the 126 positive finite non-zero values (0x7F is NaN).
@@ -74,7 +75,8 @@ def candidate_codes() -> np.ndarray:
 
 
 def e2m1_round(u: np.ndarray) -> np.ndarray:
-    """Round non-negative reals to the E2M1 grid {0,.5,1,1.5,2,3,4,6}: nearest, ties to even.
+    """Round non-negative reals to the E2M1 grid {0,.5,1,1.5,2,3,4,6}: nearest, ties to even
+    (the FP4 E2M1 weight format of PR #2283, How; its configuration names round-to-nearest-even).
 
     Values above 6 saturate to 6. "Even" means an even E2M1 code; the grid index
     is the code (exponent << 1 | mantissa), so an even index has mantissa bit 0.
@@ -99,12 +101,14 @@ def global_scale(w: np.ndarray, fp8_max: float = FP8_MAX) -> np.float32:
 
 
 def candidate_scales(g) -> np.ndarray:
-    """s_k = fp32(v_k * g) for the 126 candidates; the fp64 product is exact."""
+    """s_k = fp32(v_k * g) for the 126 candidates; the fp64 product is exact (candidates of
+    PR #2283, How; g of PR #2004, "448-normalized")."""
     return (e4m3_value(candidate_codes()) * np.float64(np.float32(g))).astype(np.float32)
 
 
 def fake_quant(w: np.ndarray, s) -> np.ndarray:
-    """NVFP4 fake quant of fp32 weights with fp32 block scale(s) s (broadcast against w).
+    """NVFP4 fake quant of fp32 weights with fp32 block scale(s) s (broadcast against w): the
+    quant(w) of dW = quant(w) - w in PR #1976, "What does this PR do?".
 
     q = E2M1(|w| / s) on the exact quotient; result fp32(q * s) with the sign of w
     (a negative weight that rounds to 0 gives -0.0). s == 0 gives q = 0.
@@ -124,7 +128,8 @@ def fake_quant(w: np.ndarray, s) -> np.ndarray:
 # ---------------------------------------------------------------------------------------
 
 def e4m3_round(r) -> np.ndarray:
-    """E4M3 code (0..126) of the value nearest to each real r >= 0: ties to the even code.
+    """E4M3 code (0..126) of the value nearest to each real r >= 0: ties to the even code (the
+    block-scale rounding of the input quantizer, PR #1976 re-review).
 
     Code 0 is zero; 1..126 are the positive finite values of ``e4m3_value``, so the even
     code is the one with mantissa bit 0. Anything above 448 saturates to 448 (code 126).
@@ -316,7 +321,8 @@ def candidate_losses(mode: str, w_blk: np.ndarray, h_blk: np.ndarray, p_blk, g) 
 
 
 def argmin_lowest(loss: np.ndarray):
-    """Best candidate per unit scanning codes ascending from best = +inf with strict <.
+    """Best candidate per unit scanning codes ascending from best = +inf with strict < (PR #1976
+    reviews: the best loss starts at +inf and may end negative).
 
     Returns (k* index [U], best loss [U], second-best loss [U]).
     """
@@ -333,7 +339,8 @@ def argmin_lowest(loss: np.ndarray):
 
 
 def sweep_units(mode: str, w_blk, h_blk, p_blk, g):
-    """Sweep U independent units. Returns dict of codes (uint8), wq [U,16], loss, second, e0."""
+    """Sweep U independent units over all 126 candidates (PR #2283, How). Returns dict of codes
+    (uint8), wq [U,16], loss, second, e0."""
     loss, wq, e0 = candidate_losses(mode, w_blk, h_blk, p_blk, g)
     kbest, best, second = argmin_lowest(loss)
     u = np.arange(len(kbest))
@@ -349,7 +356,8 @@ def sweep_units(mode: str, w_blk, h_blk, p_blk, g):
 
 
 def loss_scale(mode: str, w_blk, h_blk, p_blk) -> np.ndarray:
-    """|w|^T |H| |w| (+ 2 |w|^T |P| |w| for ACT; sum Imp w^2 for DIAG) per unit.
+    """|w|^T |H| |w| (+ 2 |w|^T |P| |w| for ACT; sum Imp w^2 for DIAG) per unit. Not a step of
+    the method: the denominator of the parity gate, a reading of this project's.
 
     The magnitude that bounds the rounding error of any Hessian-weighted loss of this block
     evaluated in finite precision; it is >= E0 and equals it for a diagonal H. Parity gaps
@@ -383,7 +391,8 @@ def gather_units(mode: str, w, h, p, g, units):
 
 
 def sweep(mode: str, w, h, p, g, units=None, chunk: int = 512):
-    """Sweep the given units (default: all) of a layer; g has one entry per group.
+    """Sweep the given units (default: all) of a layer; g has one entry per group (one weight
+    quantizer per expert, PR #2864 / #2840).
 
     Returns dict with codes, wq, loss, second, e0 for each unit, in ``units`` order.
     """
@@ -414,7 +423,8 @@ def sweep(mode: str, w, h, p, g, units=None, chunk: int = 512):
 
 
 def losses_for_scales(mode: str, w_blk, h_blk, p_blk, s) -> tuple:
-    """Losses of given block scales: s [U, K] fp32 (0 allowed) for U units.
+    """Losses of given block scales: s [U, K] fp32 (0 allowed) for U units (the losses of
+    ``candidate_losses`` at other scales, for the multiplier search of PR #788).
 
     Same definitions as ``candidate_losses`` (which is this with the 126 candidate scales
     for every unit). Returns (L [U, K], wq [U, K, 16] fp32).
@@ -436,7 +446,8 @@ def losses_for_scales(mode: str, w_blk, h_blk, p_blk, s) -> tuple:
 
 
 def multiplier_codes(w_blk, g, multipliers) -> np.ndarray:
-    """Block-scale codes of the amax-multiplier search: [U, M].
+    """Block-scale codes of the amax-multiplier search (PR #788, Changes table: step size and
+    multipliers): [U, M].
 
     For multiplier m the block's candidate amax is fp32(m * amax_blk) (amax_blk = max |w| of
     the block), and it becomes a block scale as in the NVFP4 quantizer: the E4M3 code nearest to
@@ -536,7 +547,8 @@ def apply_scales(w, g, codes):
 
 
 def calibrate(mode: str, x, w, xq=None, group_offsets=None, token_ids=None, units=None, act_gx=None):
-    """The whole hot path: accumulate, finalize, global scale per group, sweep. MSE has no
+    """The whole hot path (PR #788, #1976, #2283, #2004, #2864): accumulate, finalize, global
+    scale per group, sweep. MSE has no
     statistics: x is ignored and the sweep uses H = I."""
     if mode == "mse":
         w = np.asarray(w, dtype=np.float32)
