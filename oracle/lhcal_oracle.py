@@ -76,7 +76,8 @@ def candidate_codes() -> np.ndarray:
 
 def e2m1_round(u: np.ndarray) -> np.ndarray:
     """Round non-negative reals to the E2M1 grid {0,.5,1,1.5,2,3,4,6}: nearest, ties to even
-    (the FP4 E2M1 weight format of PR #2283, How; its configuration names round-to-nearest-even).
+    (the FP4 E2M1 weight format of PR #2283, How; the pages state no tie rule, and ties to even
+    is the reading taken).
 
     Values above 6 saturate to 6. "Even" means an even E2M1 code; the grid index
     is the code (exponent << 1 | mantissa), so an even index has mantissa bit 0.
