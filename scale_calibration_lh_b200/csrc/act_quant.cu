@@ -69,7 +69,7 @@ lhcal_status launch_act_fake_quant(const void* x, int64_t tokens, int64_t cin, i
                                    void* xq, int64_t ldq, cudaStream_t stream) {
   if (tokens == 0) return LHCAL_OK;
   const int64_t nblk = cin / kBlock;
-  // 100 registers a thread: two CTAs per SM; one wave of them loops over the rows.
+  // 104 registers a thread (ptxas): two CTAs per SM; one wave of them loops over the rows.
   const int64_t blocks = imin64(ceil_div(tokens * nblk, kQuantThreads * kQuantRows), 2 * kNumSms);
   act_quant_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(x), tokens, nblk, ldx, gx, static_cast<__nv_bfloat16*>(xq), ldq);
