@@ -439,6 +439,27 @@ def test_sweep_invariances():
     np.testing.assert_array_equal(d1["loss"], d2["loss"])
 
 
+def test_power_of_two_scaling_is_exact():
+    """W -> 2^k W with g -> 2^k g scales every candidate scale exactly, so each quotient |w| / s_k
+    and every E2M1 decision is unchanged: the same codes, Wq scaled by 2^k bit for bit, and
+    losses by 4^k (ACT: H and P fixed, the cross term scales with dW and w alike)."""
+    rng = np.random.default_rng(17)
+    w = (rng.normal(0, 0.05, (1, 24, 32)) * np.exp(rng.normal(0, 1, (1, 24, 1)))).astype(np.float32)
+    a = rng.normal(size=(1, 2, 16, 16))
+    h = a @ a.transpose(0, 1, 3, 2) / 16
+    p = 0.2 * rng.normal(size=(1, 2, 16, 16))
+    imp = np.abs(rng.normal(size=(1, 2, 16))) + 0.1
+    g = np.array([O.global_scale(w[0])], np.float32)
+    for mode, hh, pp in (("full", h, None), ("act", h, p), ("diag", imp, None), ("mse", None, None)):
+        base = O.sweep(mode, w, hh, pp, g)
+        for k in (-3, 1, 5):
+            f = np.float32(2.0 ** k)
+            sc = O.sweep(mode, w * f, hh, pp, g * f)
+            np.testing.assert_array_equal(sc["codes"], base["codes"])
+            np.testing.assert_array_equal(sc["wq"].view(np.int32), (base["wq"] * f).view(np.int32))
+            np.testing.assert_allclose(sc["loss"], base["loss"] * 4.0 ** k, rtol=1e-12, atol=0)
+
+
 def test_loss_scale_bounds_e0_and_equals_it_for_diagonal_h():
     rng = np.random.default_rng(14)
     w = rng.normal(0, 0.05, (50, 16)).astype(np.float32)
