@@ -226,3 +226,39 @@ def make_layer(name: str, seed: int = 0, tokens: int | None = None, cin: int | N
     if name == "moe":
         layer.group_offsets, layer.token_ids = moe_routing(T, G, top_k, seed)
     return layer
+
+
+# --- device placement (torch imported lazily; no step of the method) -------------------------
+
+
+def to_device(a: np.ndarray | None, kind: str, device="cuda"):
+    """Copy a host array to a torch device tensor. kind: 'bf16' (uint16 bit patterns, kept
+    bit for bit), 'f32' or 'i32'."""
+    import torch
+
+    if a is None:
+        return None
+    if kind == "bf16":
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(torch.bfloat16)
+    if kind == "f32":
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+    if kind == "i32":
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
+    raise ValueError(kind)
+
+
+def layer_to_device(layer: Layer, device="cuda") -> dict:
+    """A layer's tensors on the device: x, xq, w, the CSR routing (offs, ids) and the input
+    quantizer's global scale act_gx when the layer carries one (None where absent)."""
+    import torch
+
+    kind = "bf16" if layer.dtype == "bf16" else "f32"
+    gx = layer.meta.get("act_gx")
+    return {
+        "x": to_device(layer.x, kind, device),
+        "xq": to_device(layer.xq, kind, device),
+        "w": to_device(layer.w, kind, device),
+        "offs": to_device(layer.group_offsets, "i32", device),
+        "ids": to_device(layer.token_ids, "i32", device),
+        "act_gx": None if gx is None else torch.tensor([float(gx)], dtype=torch.float32, device=device),
+    }

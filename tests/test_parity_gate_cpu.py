@@ -8,7 +8,8 @@ rejects each of these:
 - anything non-zero where the oracle's block is zero.
 
 It still accepts what it is meant to allow: another code on a tied unit, and an error inside
-the tolerance.
+the tolerance. On a near-tie unit it checks what is unique: the GPU's code must be one of the
+oracle's tied candidates and its fake-quantized weights those of that code, bit for bit.
 """
 import numpy as np
 import pytest
@@ -22,7 +23,8 @@ def _ref():
     x = rng.normal(size=(64, 32)).astype(np.float32)
     w = rng.normal(0, 0.05, (1, 12, 32)).astype(np.float32)
     w[0, 0, :16] = 0.0  # an all-zero block: every candidate ties, so the unit is exempt
-    return O.calibrate("full", x, w)
+    ref = O.calibrate("full", x, w)
+    return P.attach_candidates(ref, "full", w, ref["h"], None, ref["g"])
 
 
 def _copies(ref):
@@ -93,3 +95,52 @@ def test_hessian_gate_per_block_tolerance_and_zero_blocks():
     z[1, 0, 0, 0] = 1e-30
     with pytest.raises(AssertionError, match="oracle block is zero"):
         P.check_hessians(z, h, "zero block")
+
+
+def _near_tie_ref():
+    """A seeded layer with near-tie units (gap <= 1e-5) whose tied codes give different Wq."""
+    rng = np.random.default_rng(40)
+    x = rng.normal(size=(64, 32)).astype(np.float32)
+    w = rng.normal(0, 0.05, (1, 300, 32)).astype(np.float32)
+    ref = O.calibrate("full", x, w)
+    P.attach_candidates(ref, "full", w, ref["h"], None, ref["g"])
+    scale = _scale(ref)
+    ex = np.nonzero((ref["second"] - ref["loss"]) / scale <= P.GAP_TOL)[0]
+    cc, cl, cw = ref["candidates"](ex)
+    for i, u in enumerate(ex):
+        tied = np.nonzero(cl[i] - ref["loss"][u] <= P.GAP_TOL * scale[u])[0]
+        for k in tied:
+            if k + 1 != ref["codes"][u] and not np.array_equal(cw[i, k].view(np.int32), ref["wq"][u].view(np.int32)):
+                untied = int(np.argmax(cl[i]))  # the worst candidate: far outside the tie
+                return ref, int(u), int(k), cw[i, k].copy(), untied, cw[i, untied].copy()
+    raise AssertionError("no near-tie unit with distinct tied weights in the seeded layer")
+
+
+def test_gate_accepts_the_other_tied_code_with_its_own_weights():
+    ref, u, k, wq_k, _, _ = _near_tie_ref()
+    codes, wq, loss = _copies(ref)
+    codes[u], wq[u] = k + 1, wq_k
+    rep = P.check_sweep(codes, wq, loss, ref, "other tied code")
+    assert rep["exempt"] >= 1 and rep["exempt_e0"] >= 0
+
+
+def test_gate_rejects_a_tied_code_paired_with_the_other_codes_weights():
+    ref, u, k, _, _, _ = _near_tie_ref()
+    codes, wq, loss = _copies(ref)
+    codes[u] = k + 1  # weights still those of the oracle's winner
+    with pytest.raises(AssertionError, match="not bit-exact to the oracle's at the GPU's code"):
+        P.check_sweep(codes, wq, loss, ref, "tied code, wrong weights")
+
+
+def test_gate_rejects_a_code_outside_the_tie_on_a_near_tie_unit():
+    ref, u, _, _, bad, wq_bad = _near_tie_ref()
+    codes, wq, loss = _copies(ref)
+    codes[u], wq[u] = bad + 1, wq_bad
+    with pytest.raises(AssertionError, match="not among the oracle's tied candidates"):
+        P.check_sweep(codes, wq, loss, ref, "untied code")
+
+
+def test_gate_needs_the_near_tie_hook():
+    ref = O.calibrate("full", np.ones((4, 16), np.float32), np.ones((1, 2, 16), np.float32))
+    with pytest.raises(AssertionError, match="near-tie hook"):
+        P.check_sweep(*_copies(ref), ref, "no hook")

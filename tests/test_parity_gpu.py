@@ -76,7 +76,7 @@ def _run_and_check(layer, units=None, check_raw=True, fused=False):
     np.testing.assert_array_equal(b2.g.cpu().numpy().view(np.int32), g.view(np.int32))
     if units is None:
         units = P.all_units(G, R, nblk)
-    ref = O.sweep(layer.mode, w32, h, p, g, units)
+    ref = P.oracle_sweep(layer.mode, w32, h, p, g, units)
     gc, gw, gl = P.gather_gpu_units(b2.codes, b2.wq, b2.loss, units)
     report["sweep"] = P.check_sweep(gc, gw, gl, ref, layer.name)
     return report
@@ -202,7 +202,7 @@ def test_sweep_special_weights_with_oracle_hessians(mode):
     assert g[2] == 0
     codes, wq, loss = _sweep_gpu(L.MODE_IDS[mode], w, h, p, g)
     units = P.all_units(G, R, nblk)
-    ref = O.sweep(mode, w, h.astype(np.float64), None if p is None else p.astype(np.float64), g, units)
+    ref = P.oracle_sweep(mode, w, h.astype(np.float64), None if p is None else p.astype(np.float64), g, units)
     gc, gw, gl = P.gather_gpu_units(codes, wq, loss, units)
     P.check_sweep(gc, gw, gl, ref, f"special {mode}")
     # Degenerate units: every candidate ties, the lowest code wins, outputs are signed zeros.
@@ -219,8 +219,48 @@ def test_sweep_identity_hessian_is_plain_mse():
     # Plain block MSE of the GPU's own fake-quant output equals its reported loss.
     mse = ((wq.astype(np.float64) - w.astype(np.float64)) ** 2).reshape(1, 64, 6, 16).sum(-1)
     np.testing.assert_allclose(loss, mse, rtol=1e-5)
-    ref = O.sweep("full", w, h.astype(np.float64), None, g)
+    ref = P.oracle_sweep("full", w, h.astype(np.float64), None, g)
     P.check_sweep(codes.reshape(-1), wq.reshape(-1, 16), loss.reshape(-1), ref, "identity H")
+
+
+def test_act_aware_negative_winning_losses():
+    """Activation-aware losses may be negative: the best loss starts at +inf and the argmin must
+    handle negative values ("Add activation-aware local Hessian scale calibration", PR #1976,
+    both review comments). With X_q = bf16(0.9 X), H ~ 0.81 M and P ~ -0.09 M (M = X^T X / B);
+    each weight block lies at 0.9 x (E2M1 grid value x s_k) for a random candidate k, so at k
+    dW = w / 9 and the objective is about 0.01 w^T M w - 0.02 w^T M w < 0. The whole path (two-tensor
+    accumulation, finalize, global scale, sweep) must match the oracle, and most winning losses
+    must be negative on both sides."""
+    rng = np.random.default_rng(77)
+    T, C, R = 700, 64, 150
+    x = synth.f32_to_bf16_bits((rng.normal(size=(T, C)) * rng.lognormal(0, 1, C)).astype(np.float32))
+    xq = synth.f32_to_bf16_bits(np.float32(0.9) * synth.bf16_bits_to_f32(x))
+    g0 = np.float32(2.0 ** -10)
+    s = O.candidate_scales(g0)
+    grid = np.array([0.5, 1, 1.5, 2, 3, 4, 6])
+    nblk = C // 16
+    k = rng.integers(40, 126, (R, nblk))
+    q = grid[rng.integers(0, len(grid), (R, nblk, 16))]
+    sign = np.where(rng.random((R, nblk, 16)) < 0.5, -1.0, 1.0)
+    w = (0.9 * q * s[k][..., None].astype(np.float64) * sign).astype(np.float32).reshape(1, R, C)
+    w[0, 0, 0] = np.float32(2688.0 * 2.0 ** -10)  # amax: the global scale is exactly g0
+    assert O.global_scale(w[0]) == g0
+    dev = {"x": synth.to_device(x, "bf16"), "xq": synth.to_device(xq, "bf16"), "w": synth.to_device(w, "f32")}
+    b = L.calibrate("act", dev["x"], dev["w"], xq=dev["xq"])
+    _sync()
+    hs, ps, counts = O.accumulate("act", synth.bf16_bits_to_f32(x), synth.bf16_bits_to_f32(xq))
+    h, p = O.finalize("act", hs, ps, counts)
+    P.check_hessians(b.h.cpu().numpy(), h, "negative-loss layer H")
+    P.check_hessians(b.p.cpu().numpy(), p, "negative-loss layer P")
+    np.testing.assert_array_equal(b.g.cpu().numpy(), [g0])
+    units = P.all_units(1, R, nblk)
+    ref = P.oracle_sweep("act", w, h, p, np.array([g0], np.float32), units)
+    gc, gw, gl = P.gather_gpu_units(b.codes, b.wq, b.loss, units)
+    rep = P.check_sweep(gc, gw, gl, ref, "negative-loss layer")
+    assert rep["units"] == R * nblk
+    neg = ref["loss"] < 0
+    assert neg.mean() > 0.9, f"only {neg.mean():.2f} of the oracle's winning losses are negative"
+    assert np.all(gl[neg] < 0), "the GPU's winning loss is not negative where the oracle's is"
 
 
 # ----------------------------------------------------------------------------- accumulate semantics
@@ -334,7 +374,7 @@ def _run_and_check_wmse_full(layer, units):
     w32 = layer.w_f32()
     g = np.array([O.global_scale(w32[0])], np.float32)
     np.testing.assert_array_equal(b.g.cpu().numpy().view(np.int32), g.view(np.int32))
-    ref = O.sweep("diag", w32, h, None, g, units)
+    ref = P.oracle_sweep("diag", w32, h, None, g, units)
     gc, gw, gl = P.gather_gpu_units(b.codes, b.wq, b.loss, units)
     P.check_sweep(gc, gw, gl, ref, "wmse full")
 
@@ -556,7 +596,7 @@ def test_mse_sweep(name, kw):
     g = np.array([O.global_scale(w32[e]) for e in range(G)], np.float32)
     np.testing.assert_array_equal(b.g.cpu().numpy().view(np.int32), g.view(np.int32))
     units = P.all_units(G, R, C // 16)
-    ref = O.sweep("mse", w32, None, None, g, units)
+    ref = P.oracle_sweep("mse", w32, None, None, g, units)
     gc, gw, gl = P.gather_gpu_units(b.codes, b.wq, b.loss, units)
     P.check_sweep(gc, gw, gl, ref, f"{name} mse")
 
@@ -569,7 +609,7 @@ def test_mse_sweep_full_size_weights():
     w32 = layer.w_f32()
     g = np.array([O.global_scale(w32[0])], np.float32)
     units = P.sample_units(1, layer.rows, layer.cin // 16, 3000, seed=2)
-    ref = O.sweep("mse", w32, None, None, g, units)
+    ref = P.oracle_sweep("mse", w32, None, None, g, units)
     gc, gw, gl = P.gather_gpu_units(b.codes, b.wq, b.loss, units)
     P.check_sweep(gc, gw, gl, ref, "dense mse full size")
 
@@ -658,7 +698,7 @@ def test_multiplier_search(mode, name, kw):
                               p=None if p is None else P.to_device(p, "f32"))
     _sync()
     units = P.all_units(G, R, C // 16)
-    ref = O.multiplier_search(mode, w32, h, p, g, mult, units)
+    ref = P.oracle_multiplier_search(mode, w32, h, p, g, mult, units)
     gc, gw, gl = P.gather_gpu_units(codes, wq, loss, units)
     rep = P.check_sweep(gc, gw, gl, ref, f"{name} {mode} multiplier search")
     assert rep["units"] == len(units)
@@ -750,7 +790,7 @@ def test_multiplier_search_counts(n_mult):
                               codes, wq=wq, loss=loss)
     _sync()
     units = P.all_units(G, R, C // 16)
-    ref = O.multiplier_search("full", w32, h, None, g, mult, units)
+    ref = P.oracle_multiplier_search("full", w32, h, None, g, mult, units)
     gc, gw, gl = P.gather_gpu_units(codes, wq, loss, units)
     P.check_sweep(gc, gw, gl, ref, f"multiplier search, {n_mult} multipliers")
 
