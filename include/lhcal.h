@@ -271,7 +271,9 @@ lhcal_status lhcal_apply_scales(lhcal_dtype dtype, const void* w, int32_t groups
  * (lhcal_accumulate_workspace) exceeds it are rejected with LHCAL_ERR_INVALID_ARG before
  * anything is enqueued. The call allocates nothing and frees nothing.
  *   - The first call on each device looks up the scratch's device address (with that device
- *     current); make that first call before any stream capture on the device.
+ *     current); make that first call before any stream capture on the device. The address is
+ *     kept for the rest of the process, so destroying the device's primary context after that
+ *     call (cudaDeviceReset) is not supported: the module would be reloaded at another address.
  *   - All calls on a device share the one scratch array, and it keeps the last call's
  *     contents. The kernels overwrite every partial before reading it, so no clearing is
  *     needed. Calls that can overlap on the GPU (on different streams, or from different

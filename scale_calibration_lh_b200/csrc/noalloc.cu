@@ -20,7 +20,8 @@ void* g_scratch_addr[kMaxDevices] = {};
 
 // Device address of g_noalloc_scratch on the current device. In host code the symbol's name
 // is only a host-side stand-in, so the address must come from the runtime, once per device,
-// with that device current.
+// with that device current. It is cached for the life of the process: a cudaDeviceReset after
+// the first call would reload the module elsewhere, which the header states is unsupported.
 lhcal_status scratch_for_current_device(float** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);

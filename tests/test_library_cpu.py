@@ -42,6 +42,15 @@ def test_status_values_match_header(root_dir):
         assert m and int(m.group(1)) == val, name
 
 
+def test_noalloc_scratch_size_in_python_matches_the_header(root_dir):
+    """The binding's copy of LHCAL_NOALLOC_SCRATCH_BYTES (used to size-check before the call)
+    is the header's value."""
+    text = open(os.path.join(root_dir, "include", "lhcal.h")).read()
+    m = re.search(r"#define\s+LHCAL_NOALLOC_SCRATCH_BYTES\s+\(([^)]*)\)", text)
+    assert m, "LHCAL_NOALLOC_SCRATCH_BYTES not found in lhcal.h"
+    assert eval(m.group(1).replace("u", ""), {}) == L.NOALLOC_SCRATCH_BYTES
+
+
 def test_workspace_query_is_host_only(lib):
     dense = L.lhcal_accumulate_workspace("full", L.BF16, 16384, 2048, 1)
     assert dense > 0 and dense % (128 * 4 * 256) == 0  # whole [splits, N, 16, 16] partials
