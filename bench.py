@@ -1,17 +1,31 @@
 #!/usr/bin/env python
-"""Benchmark: local-Hessian NVFP4 weight-scale calibration of one synthetic layer per GPU.
+"""Benchmark: local-Hessian NVFP4 weight-scale calibration of synthetic layers, one per GPU.
 
 One step = the whole hot path over one layer: Hessian accumulation (OVERWRITE), token
 counts, finalisation, per-group global scale, and the exhaustive 126-candidate FP8 scale
 sweep writing codes, fake-quantized weights and losses. Inputs are resident in HBM when
-the timed region starts; each step's inputs (X and W together) exceed the 126 MB L2 for
-every bench workload, so no L2 flush runs between steps.
+the timed region starts.
 
-e2e: the same step through calibrate_host from pinned host buffers, inputs copied in and
-the result (codes and losses) copied out every step. The activation-aware workload also
-reports the two-tensor accumulation (X_q resident) beside its fused step.
+By default every workload runs, in the order tiny, dense, act, wmse, moe, each timed over
+the same --steps after the same --warmup; the JSON line's headline (value, ms_per_step,
+roofline, e2e, cpu_baseline) is the largest, the fused-MoE gate_up layer, and "workloads"
+holds one record per workload. --workload NAME runs one.
 
-  python bench.py [--gpus N --steps K --warmup W --workload dense|act|wmse|moe]
+Per workload:
+  * the step loop, K steps back to back between two events (inputs above the 126 MB L2: no
+    flush), or, when the inputs fit in L2 (the tiny layer), each step bracketed by its own
+    events with an L2 flush between steps outside them; per-stage events give medians;
+  * roofline: the sweep's FP32 lane-ops of the direct method over its median in-step time,
+    against 148 SMs x 128 lanes x the max SM clock;
+  * roofline_accum: the accumulation launched alone, max(20, K) times, each after a read of a
+    256 MB buffer (which leaves the L2 clean and holding none of X), median of the event times;
+    the in-step accumulation time is reported beside it;
+  * e2e: the same path through calibrate_host from pinned host buffers, inputs copied in and
+    the whole output copied out every step: codes, global scales, losses and the bf16
+    fake-quantized weights; e2e_scales_only leaves the weights on the device;
+  * cpu_baseline (rank 0, one GPU): the CPU oracle timed on a bounded sample.
+
+  python bench.py [--gpus N --steps K --warmup W --workload all|tiny|dense|act|wmse|moe]
   python bench.py --impl reference ...   (the CPU oracle, timed on a bounded sample)
 
 N > 1 runs under torchrun, one independent layer per rank (weak scaling, no collective
@@ -40,7 +54,13 @@ N_SMS = 148
 FP32_LANES_PER_SM = 128
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_SM_MHZ = 1965.0
+L2_BYTES = 126 * 1024 * 1024
+FLUSH_BYTES = 256 * 1024 * 1024
+ORDER = ("tiny", "dense", "act", "wmse", "moe")
+HEADLINE = "moe"  # the largest workload: 104.9 M sweep units
 WORKLOAD_TEXT = {
+    "tiny": "tiny linear local_hessian: X fp32 [256,64] N(0,1), W fp32 [32,64] N(0,0.02), 4 blocks, full 16x16 H, "
+            "126-candidate FP8 sweep (parity-sized; launch-latency-bound)",
     "dense": "dense projection local_hessian: X bf16 [16384,4096] (lognormal column std, 1% outliers x20), "
              "W bf16 [4096,4096], full 16x16 H per block, 126-candidate FP8 sweep",
     "act": "activation-aware gate_up: X bf16 [32768,4096] through the fused NVFP4 input quantizer (X_q derived "
@@ -49,17 +69,10 @@ WORKLOAD_TEXT = {
     "moe": "fused-MoE gate_up: 512 experts, X bf16 [16384,2560] top-10 routed, W bf16 [512,1280,2560], "
            "grouped full H, per-expert global scale",
 }
-# dram__bytes_read.sum + dram__bytes_write.sum per launch, from one ncu capture of the current
-# kernel on this workload (summaries in profiles/); workloads without a capture report null.
-SWEEP_TRAFFIC_BYTES = {
-    "dense": 33_938_176 + 30_059_264,    # sweep_tc_kernel, profiles/sweep_tc_kernel_dense.md
-    "wmse": 101_393_408 + 167_207_936,   # sweep_diag_kernel, profiles/sweep_diag_kernel_wmse.md
-}
-ACCUM_TRAFFIC_BYTES = {
-    "dense": 134_265_344 + 3_774_464,    # accum_mma_kernel (clusters), profiles/accum_mma_kernel_dense.md
-    "act": 268_573_696 + 5_457_664,      # accum_mma_kernel (quantizer fused), profiles/accum_mma_kernel_act.md
-    "wmse": 1_610_820_000 + 8_041_472,   # accum_diag_kernel (+ the partial reduction, not captured)
-}
+# dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu capture of the named
+# kernel on the workload, as committed with its summary; reported as traffic_from_profile,
+# never as a measurement of the run (the bench cannot read DRAM counters).
+PROFILED_TRAFFIC = {}
 
 
 def load_peaks():
@@ -87,6 +100,12 @@ def rank_max(values, device=None):
 def weak_scaling_value(units_per_rank: int, world: int, ms_per_step_max: float) -> float:
     """Whole-job throughput: every rank's units over the slowest rank's step time."""
     return units_per_rank * world / (ms_per_step_max / 1e3)
+
+
+def median(xs):
+    s = sorted(float(x) for x in xs)
+    n = len(s)
+    return s[n // 2] if n % 2 else 0.5 * (s[n // 2 - 1] + s[n // 2])
 
 
 # ------------------------------------------------------------------------------------------ clocks
@@ -185,28 +204,33 @@ def cpu_threads():
         return 1
 
 
+def _as_f32(a, layer):
+    from scale_calibration_lh_b200 import synth
+
+    return a if layer.dtype == "f32" else synth.bf16_bits_to_f32(a)
+
+
 def oracle_sample_step(layer, frac_tokens: float, n_units: int, seed: int = 0):
     """Time the CPU oracle on a bounded sample; returns estimated seconds for the whole layer."""
     import numpy as np
 
     from oracle import lhcal_oracle as O
-    from scale_calibration_lh_b200 import synth
 
     T = layer.tokens
     ts = max(1, int(T * frac_tokens))
     if layer.mode == "act" and "act_gx_oracle" not in layer.meta:
-        layer.meta["act_gx_oracle"] = O.global_scale(synth.bf16_bits_to_f32(layer.x))
+        layer.meta["act_gx_oracle"] = O.global_scale(_as_f32(layer.x, layer))
     t0 = time.perf_counter()
     if layer.token_ids is not None:
         # Grouped: the first groups' routed rows, about ts rows in total.
         off = layer.group_offsets
         gcount = int(np.searchsorted(off, ts, side="right")) - 1
         gcount = max(1, min(gcount, layer.groups))
-        x32 = synth.bf16_bits_to_f32(layer.x)
+        x32 = _as_f32(layer.x, layer)
         O.accumulate(layer.mode, x32, None, off[:gcount + 1], layer.token_ids[:off[gcount]])
         frac = gcount / layer.groups
     else:
-        xs = synth.bf16_bits_to_f32(layer.x[:ts])
+        xs = _as_f32(layer.x[:ts], layer)
         # Activation-aware: the oracle derives X_q with the input quantizer's global scale,
         # computed once over the whole X before the timing starts.
         O.accumulate(layer.mode, xs, None, act_gx=layer.meta.get("act_gx_oracle"))
@@ -215,16 +239,17 @@ def oracle_sample_step(layer, frac_tokens: float, n_units: int, seed: int = 0):
     rng = np.random.default_rng(seed)
     G, R, C = layer.groups, layer.rows, layer.cin
     nb = C // 16
+    n_units = min(n_units, 4 * G * R * nb)
     # Global scale: the first groups (at most 8), scaled to all groups.
     gs = min(G, 8)
     t0 = time.perf_counter()
-    g = np.array([O.global_scale(synth.bf16_bits_to_f32(layer.w[e])) for e in range(gs)], np.float32)
+    g = np.array([O.global_scale(_as_f32(layer.w[e], layer)) for e in range(gs)], np.float32)
     t_g = (time.perf_counter() - t0) * G / gs
     # Sweep: n_units random (row, block) units in one call, as a one-group layer of the sampled rows.
     rows = rng.integers(0, R, n_units)
     blks = rng.integers(0, nb, n_units)
     grp = rng.integers(0, gs, n_units)
-    w_s = synth.bf16_bits_to_f32(layer.w[grp, rows])[None]  # [1, U, C]
+    w_s = _as_f32(layer.w[grp, rows], layer)[None]  # [1, U, C]
     if layer.mode == "diag":
         h = np.abs(rng.normal(size=(1, nb, 16))) + 1.0
     else:
@@ -240,13 +265,19 @@ def oracle_sample_step(layer, frac_tokens: float, n_units: int, seed: int = 0):
 
 # ------------------------------------------------------------------------------------------ arms
 
+def headline_name(args) -> str:
+    return HEADLINE if args.workload == "all" else args.workload
+
+
 def run_reference(args, rank, world):
-    """The CPU oracle (the deliberately slow reference program) on a bounded sample per step."""
+    """The CPU oracle (the deliberately slow reference program) on a bounded sample per step, on
+    the workload that the native arm's headline measures."""
     if rank != 0:
         return
     from scale_calibration_lh_b200 import synth
 
-    layer = synth.make_layer(args.workload, 0)
+    name = headline_name(args)
+    layer = synth.make_layer(name, 0)
     units, _, _ = algorithmic(layer)
     frac, n_units = 1.0 / 64, 512
     for _ in range(args.warmup):
@@ -260,36 +291,53 @@ def run_reference(args, rank, world):
     cores = cpu_threads()
     out = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD_TEXT[args.workload], "name": args.workload},
+        "warmup": args.warmup, "ms_per_step": ms, "ms_per_step_estimated": True, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT[name], "name": name},
+        "estimate": f"each step times the oracle on a sample (accumulation over {sample['tokens']} tokens, the "
+                    f"sweep of {sample['units']} random units) and scales each stage to the whole layer",
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"per step: accumulation over {sample['tokens']} tokens and the sweep of "
-                                   f"{n_units} random units, each scaled to the whole layer"},
+                                   f"{sample['units']} random units, each scaled to the whole layer"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(out), flush=True)
 
 
-def run_lhcal(args, rank, world, local_rank):
+class L2Flush:
+    """Reads a 256 MB device buffer: dirty L2 lines are written back on the way and the L2 is
+    left holding clean lines of this buffer only (a read, not a write, so nothing stays dirty)."""
+
+    def __init__(self, device):
+        import torch
+
+        self.buf = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+
+    def __call__(self):
+        self.buf.sum()
+
+
+def measure_workload(name, args, rank, world, dev, flusher):
+    """Time one workload as the module docstring describes; returns its record (rank 0's view,
+    times already the maximum over ranks)."""
     import numpy as np
     import torch
 
     import scale_calibration_lh_b200 as L
-    from scale_calibration_lh_b200 import build as B
     from scale_calibration_lh_b200 import synth
-    from tests import parity as P
 
-    B.build()
-    L.load_library()
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
     dist = world > 1
-    layer = synth.make_layer(args.workload, rank, rows=args.rows)
-    d = P.layer_to_device(layer, dev)
+
+    def barrier():
+        if dist:
+            torch.distributed.barrier()
+
+    layer = synth.make_layer(name, rank, rows=args.rows)
+    d = synth.layer_to_device(layer, dev)
     mode = L.MODE_IDS[layer.mode]
     G, R, C, T = layer.groups, layer.rows, layer.cin, layer.tokens
-    buf = L.Buffers(mode, T, C, R, G, L.BF16, dev)
+    xdt = L.BF16 if layer.dtype == "bf16" else L.F32
+    buf = L.Buffers(mode, T, C, R, G, xdt, dev)
     stream = torch.cuda.current_stream()
     act_gx = None
     if layer.mode == "act":
@@ -298,37 +346,16 @@ def run_lhcal(args, rank, world, local_rank):
         act_gx = torch.empty(1, dtype=torch.float32, device=dev)
         L.lhcal_global_scale(d["x"].view(1, T, C), act_gx)
 
-    def step():
-        L.calibrate(mode, d["x"], d["w"], xq=d["xq"], group_offsets=d["offs"], token_ids=d["ids"], buffers=buf,
-                    act_gx=act_gx)
-
-    def barrier():
-        if dist:
-            torch.distributed.barrier()
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-
-    # ---- device-resident timed region, with per-stage events on the launching stream
-    clocks = ClockSampler(torch.cuda.current_device())
-    K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
-    L.lhcal_launch_count(reset=True)
-    clocks.start()
-    start.record(stream)
-    for k in range(K):
-        e = ev[k]
-        e[0].record(stream)
+    def accumulate(b):
         if act_gx is not None:
-            L.lhcal_accumulate_act_quant(d["x"], buf.h, buf.p, act_gx, flags=L.ACCUM_OVERWRITE,
-                                         workspace=buf.workspace)
+            L.lhcal_accumulate_act_quant(d["x"], b.h, b.p, act_gx, flags=L.ACCUM_OVERWRITE, workspace=b.workspace)
         else:
-            L.lhcal_accumulate(mode, d["x"], buf.h, xq=d["xq"], p=buf.p, group_offsets=d["offs"],
-                               token_ids=d["ids"], flags=L.ACCUM_OVERWRITE, workspace=buf.workspace)
+            L.lhcal_accumulate(mode, d["x"], b.h, xq=d["xq"], p=b.p, group_offsets=d["offs"], token_ids=d["ids"],
+                               flags=L.ACCUM_OVERWRITE, workspace=b.workspace)
+
+    def step(e):
+        e[0].record(stream)
+        accumulate(buf)
         e[1].record(stream)
         L.lhcal_count_tokens(buf.counts, tokens=T, group_offsets=d["offs"], flags=L.ACCUM_OVERWRITE)
         L.lhcal_finalize(mode, buf.counts, buf.h, p=buf.p)
@@ -337,130 +364,212 @@ def run_lhcal(args, rank, world, local_rank):
         e[3].record(stream)
         L.lhcal_scale_sweep(mode, d["w"], buf.h, buf.g, buf.codes, wq=buf.wq, loss=buf.loss, p=buf.p)
         e[4].record(stream)
+
+    def events(n):
+        return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+    input_bytes = sum(t.numel() * t.element_size() for t in (d["x"], d["w"], d["offs"], d["ids"]) if t is not None)
+    small = input_bytes < L2_BYTES
+    K = args.steps
+    for _ in range(args.warmup):
+        if small:
+            flusher()
+        step(events(5))
+    torch.cuda.synchronize()
+
+    # ---- the step loop
+    clocks = ClockSampler(torch.cuda.current_device())
+    ev = [events(5) for _ in range(K)]
+    start, end = events(2)
+    barrier()
+    torch.cuda.synchronize()
+    L.lhcal_launch_count(reset=True)
+    clocks.start()
+    start.record(stream)
+    for k in range(K):
+        if small:
+            flusher()  # outside the step's own events
+        step(ev[k])
     end.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
     barrier()
     launches = L.lhcal_launch_count()
-    ms_total = start.elapsed_time(end)
+    ms_total = sum(e[0].elapsed_time(e[4]) for e in ev) if small else start.elapsed_time(end)
     stage = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in ev])  # ms
-    t_acc, t_fin, t_g, t_sweep = (float(v) for v in stage.mean(0))
-    ms_total, t_acc, t_sweep = rank_max([ms_total, t_acc, t_sweep], dev)
+    med = [median(stage[:, i]) for i in range(4)]
+    mean = [float(v) for v in stage.mean(0)]
+    ms_total, t_acc_step, t_sweep = rank_max([ms_total, med[0], med[3]], dev)
     ms = ms_total / K
     units, ops, acc_bytes = algorithmic(layer)
-    value = weak_scaling_value(units, world, ms)
+
+    # ---- the accumulation alone, each launch after an L2 flush (median of max(20, K))
+    reps = max(20, K)
+    acc_ev = [events(2) for _ in range(reps)]
+    torch.cuda.synchronize()
+    for a, b in acc_ev:
+        flusher()
+        a.record(stream)
+        accumulate(buf)
+        b.record(stream)
+    torch.cuda.synchronize()
+    (t_acc,) = rank_max([median(a.elapsed_time(b) for a, b in acc_ev)], dev)
 
     # ---- activation-aware: the two-tensor accumulation for comparison. When the capture records
     # X_q next to X (the input-quantizer hook), X_q is already in HBM and the accumulation reads
-    # both. X_q is materialised once here, outside every timed region, and the kernel is timed
-    # launch by launch; the step above (and its value) uses the fused path.
+    # both. X_q is materialised once here, outside every timed region; each launch is timed after
+    # an L2 flush and the median taken, as above; the step (and its value) uses the fused path.
     two_tensor = None
     if act_gx is not None:
         xq_res = torch.empty_like(d["x"])
         L.lhcal_act_fake_quant(d["x"], act_gx, xq_res)
         torch.cuda.synchronize()
-        K3 = max(3, min(K, 20))
-        ev3 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K3)]
+        ev3 = [events(2) for _ in range(reps)]
         for a3, b3 in ev3:
+            flusher()
             a3.record(stream)
             L.lhcal_accumulate(mode, d["x"], buf.h, xq=xq_res, p=buf.p, flags=L.ACCUM_OVERWRITE,
                                workspace=buf.workspace)
             b3.record(stream)
         torch.cuda.synchronize()
-        t3 = float(np.mean([a3.elapsed_time(b3) for a3, b3 in ev3]))
-        (t3,) = rank_max([t3], dev)
-        two_tensor = {"ms": t3, "bytes": 2 * T * C * 2 + 2 * C // 16 * 256 * 4, "launches": K3}
+        (t3,) = rank_max([median(a3.elapsed_time(b3) for a3, b3 in ev3)], dev)
+        two_tensor = {"ms": t3, "bytes": 2 * T * C * 2 + 2 * C // 16 * 256 * 4, "launches": reps}
         del xq_res
 
     # ---- end to end through the public API from pinned host buffers
-    hx = torch.empty(d["x"].shape, dtype=d["x"].dtype, pin_memory=True)
-    hx.copy_(d["x"])
-    hxq = None
-    if d["xq"] is not None:
-        hxq = torch.empty(d["xq"].shape, dtype=d["xq"].dtype, pin_memory=True)
-        hxq.copy_(d["xq"])
-    hw = torch.empty(d["w"].shape, dtype=d["w"].dtype, pin_memory=True)
-    hw.copy_(d["w"])
-    # The step's result read back: the codes (the chosen scales) and the winning losses; the
-    # fake-quantized weights stay on the device (lhcal_apply_scales derives them from the codes).
-    out_host = L.HostOutputs(buf, want_wq=False)
-    hoffs = None if d["offs"] is None else d["offs"].cpu().pin_memory()
-    hids = None if d["ids"] is None else d["ids"].cpu().pin_memory()
+    def pinned(t):
+        if t is None:
+            return None
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t)
+        return h
+
+    hx, hxq, hw = pinned(d["x"]), pinned(d["xq"]), pinned(d["w"])
+    hoffs, hids = pinned(d["offs"]), pinned(d["ids"])
     K2 = max(3, min(K, 10))
+    e2e = {}
+    for label, want_wq16 in (("e2e", True), ("e2e_scales_only", False)):
+        # The whole output: codes, global scales and losses, plus the bf16 fake-quantized weights
+        # (lhcal_apply_scales of the chosen codes) unless the weights stay on the device.
+        b2 = L.Buffers(mode, T, C, R, G, xdt, dev, want_wq=False, want_wq16=want_wq16)
+        out_host = L.HostOutputs(b2, want_wq=False)
 
-    def e2e_step():
-        L.calibrate_host(mode, hx, hw, buf, d, hxq=hxq, group_offsets=hoffs, token_ids=hids, out=out_host,
-                         act_gx=act_gx)
+        def e2e_step():
+            L.calibrate_host(mode, hx, hw, b2, d, hxq=hxq, group_offsets=hoffs, token_ids=hids, out=out_host,
+                             act_gx=act_gx)
 
-    e2e_step()  # warm
-    torch.cuda.synchronize()
-    barrier()
-    e2s, e2e_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2s.record(stream)
-    for _ in range(K2):
-        e2e_step()
-    e2e_.record(stream)
-    torch.cuda.synchronize()
-    ms_e2e = e2s.elapsed_time(e2e_) / K2
-    (ms_e2e,) = rank_max([ms_e2e], dev)
-    h2d = sum(t.numel() * t.element_size() for t in (hx, hw, hxq, hoffs, hids) if t is not None)
-    d2h = out_host.nbytes()
+        e2e_step()  # warm
+        torch.cuda.synchronize()
+        barrier()
+        e2s, e2e_end = events(2)
+        e2s.record(stream)
+        for _ in range(K2):
+            e2e_step()
+        e2e_end.record(stream)
+        torch.cuda.synchronize()
+        (ms_e2e,) = rank_max([e2s.elapsed_time(e2e_end) / K2], dev)
+        h2d = sum(t.numel() * t.element_size() for t in (hx, hw, hxq, hoffs, hids) if t is not None)
+        e2e[label] = {"value": weak_scaling_value(units, world, ms_e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                      "d2h_bytes_per_step": out_host.nbytes(), "ms_per_step": ms_e2e, "steps": K2,
+                      "outputs": "codes, global scales, losses" + (", bf16 fake-quantized weights" if want_wq16
+                                                                   else "; fake-quantized weights stay on the device")}
+        del b2, out_host
 
-    if rank != 0:
-        return
     hbm_gbs, sm_mhz, peak_src = load_peaks()
     peak_ops = N_SMS * FP32_LANES_PER_SM * sm_mhz * 1e6
-    sweep_units = units
-    achieved_ops = sweep_units * ops / (t_sweep / 1e3)
-    traffic = SWEEP_TRAFFIC_BYTES.get(args.workload)
+    achieved_ops = units * ops / (t_sweep / 1e3)
     achieved_gbs = acc_bytes / (t_acc / 1e3) / 1e9
-    out = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
-        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-        "data": "synthetic",
-        "config": {"workload": WORKLOAD_TEXT[args.workload], "name": args.workload, "tokens": T, "cin": C,
-                   "rows": R, "groups": G, "mode": layer.mode, "input_dtype": layer.dtype,
-                   "l2": "no flush: each step's inputs (X and W) exceed the 126 MB L2",
-                   "parallelism": f"{world} independent layers, one per GPU (no collective)"},
-        "roofline": {"kernel": "sweep_diag_kernel" if layer.mode == "diag" else "sweep_tc_kernel", "bound": "alu", "achieved": achieved_ops / 1e12,
-                     "peak": peak_ops / 1e12, "unit": "Tops/s", "frac": achieved_ops / peak_ops,
-                     "traffic": traffic,
-                     "note": f"FP32 lane-ops of the direct method ({ops // 126}/candidate) over the measured sweep "
-                             f"time; peak = {N_SMS} SMs x {FP32_LANES_PER_SM} FP32 lanes x {sm_mhz:.0f} MHz "
+    sweep_kernel = "sweep_diag_kernel" if layer.mode == "diag" else "sweep_tc_kernel"
+    acc_kernel = {"diag": "accum_diag_kernel + reduce_partials_kernel"}.get(layer.mode, "accum_mma_kernel")
+    if layer.dtype == "f32":
+        acc_kernel = "accum_generic_kernel + reduce_partials_kernel"
+    rec = {
+        "name": name, "workload": WORKLOAD_TEXT[name], "tokens": T, "cin": C, "rows": R, "groups": G,
+        "mode": layer.mode, "input_dtype": layer.dtype,
+        "value": weak_scaling_value(units, world, ms), "unit": UNIT, "ms_per_step": ms, "steps": K,
+        "units_per_step": units,
+        "l2": ("inputs fit in the L2: an L2 flush between timed steps, outside each step's events" if small else
+               f"no flush: each step's inputs ({input_bytes / 1e6:.0f} MB of X and W) exceed the 126 MB L2"),
+        "stages_ms": dict(zip(("accumulate", "count_finalize", "global_scale", "sweep"), med)),
+        "stages_ms_mean": dict(zip(("accumulate", "count_finalize", "global_scale", "sweep"), mean)),
+        "roofline": {"kernel": sweep_kernel, "bound": "alu", "achieved": achieved_ops / 1e12,
+                     "peak": peak_ops / 1e12, "unit": "Tops/s", "frac": achieved_ops / peak_ops, "traffic": None,
+                     "traffic_from_profile": PROFILED_TRAFFIC.get((name, sweep_kernel)),
+                     "note": f"FP32 lane-ops of the direct method ({ops // 126}/candidate) over the median in-step "
+                             f"sweep time; peak = {N_SMS} SMs x {FP32_LANES_PER_SM} FP32 lanes x {sm_mhz:.0f} MHz "
                              f"(max clock, {peak_src})"},
-        "roofline_accum": {"kernel": "accumulate (incl. partial reduction)" + (
-                               ", input quantizer fused" if act_gx is not None else ""), "bound": "hbm",
-                           "achieved": achieved_gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": achieved_gbs / hbm_gbs,
-                           "traffic": ACCUM_TRAFFIC_BYTES.get(args.workload), "bytes_per_step": acc_bytes,
-                           "note": f"algorithmic bytes over the measured accumulation time; peak {peak_src}"},
-        "stages_ms": {"accumulate": t_acc, "count_finalize": t_fin, "global_scale": t_g, "sweep": t_sweep},
-        "e2e": {"value": weak_scaling_value(units, world, ms_e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
+        "roofline_accum": {"kernel": acc_kernel + (", input quantizer fused" if act_gx is not None else ""),
+                           "bound": "hbm", "achieved": achieved_gbs, "peak": hbm_gbs, "unit": "GB/s",
+                           "frac": achieved_gbs / hbm_gbs, "traffic": None,
+                           "traffic_from_profile": PROFILED_TRAFFIC.get((name, "accum")),
+                           "bytes_per_step": acc_bytes, "ms": t_acc, "in_step_ms": t_acc_step,
+                           "in_step_frac": acc_bytes / (t_acc_step / 1e3) / 1e9 / hbm_gbs,
+                           "note": f"algorithmic bytes over the median of {reps} launches, each after an L2 flush "
+                                   f"(peak {peak_src}); in_step_ms is the same stage inside the step loop, where it "
+                                   f"follows the previous step's sweep"},
         "gpu_launches": launches,
         "clocks": clk,
     }
+    rec.update(e2e)
+    if small:
+        rec["latency_bound"] = True
     if two_tensor is not None:
         gbs = two_tensor["bytes"] / (two_tensor["ms"] / 1e3) / 1e9
-        out["accumulate_two_tensor"] = {
+        rec["accumulate_two_tensor"] = {
             "ms": two_tensor["ms"], "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,
             "note": "X and X_q both read (X_q materialised beforehand, as the input-quantizer hook provides it); "
-                    f"mean of {two_tensor['launches']} launches timed one by one; not part of value"}
+                    f"median of {two_tensor['launches']} launches, each after an L2 flush; not part of value"}
     if world == 1 and not args.no_cpu_baseline:
         est, sample = oracle_sample_step(layer, 1.0 / 16, 16384)
-        cb_value = units / est
-        out["cpu_baseline"] = {"value": cb_value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+        rec["cpu_baseline"] = {"value": units / est, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                                "sample": f"accumulation over {sample['tokens']} tokens and the sweep of "
                                          f"{sample['units']} random units, each scaled to the whole layer"}
+    del d, buf, hx, hxq, hw, hoffs, hids
+    torch.cuda.empty_cache()
+    return rec
+
+
+def run_lhcal(args, rank, world, local_rank):
+    import torch
+
+    import scale_calibration_lh_b200 as L
+    from scale_calibration_lh_b200 import build as B
+
+    B.build()
+    L.load_library()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    flusher = L2Flush(dev)
+    names = ORDER if args.workload == "all" else (args.workload,)
+    recs = {n: measure_workload(n, args, rank, world, dev, flusher) for n in names}
+    if rank != 0:
+        return
+    head = recs[headline_name(args)]
+    out = {
+        "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": head["workload"], "name": head["name"], "tokens": head["tokens"], "cin": head["cin"],
+                   "rows": head["rows"], "groups": head["groups"], "mode": head["mode"],
+                   "input_dtype": head["input_dtype"], "l2": head["l2"],
+                   "parallelism": f"{world} independent layers, one per GPU (no collective)",
+                   "workloads_run": list(names)},
+        "roofline": head["roofline"], "roofline_accum": head["roofline_accum"], "stages_ms": head["stages_ms"],
+        "e2e": head["e2e"], "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
+    }
+    if "cpu_baseline" in head:
+        out["cpu_baseline"] = head["cpu_baseline"]
+    out["workloads"] = recs
     print(json.dumps(out), flush=True)
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["lhcal", "reference"], default="lhcal")
-    ap.add_argument("--workload", choices=list(WORKLOAD_TEXT), default="dense")
+    ap.add_argument("--workload", choices=["all"] + list(ORDER), default="all")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rows", type=int, default=None,
                     help="weight rows per group instead of the workload's (smaller captures for profiling)")

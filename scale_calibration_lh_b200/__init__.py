@@ -336,7 +336,7 @@ class Buffers:
     """Device buffers for one layer's calibration (allocated by torch, owned by the caller)."""
 
     def __init__(self, mode, tokens: int, cin: int, rows: int, groups: int, x_dtype: int, device,
-                 want_wq: bool = True, want_loss: bool = True):
+                 want_wq: bool = True, want_loss: bool = True, want_wq16: bool = False):
         import torch
 
         self.mode = _mode_id(mode)
@@ -350,6 +350,8 @@ class Buffers:
         self.codes = torch.empty((groups, rows, nblk), dtype=torch.uint8, device=device)
         self.wq = torch.empty((groups, rows, cin), dtype=torch.float32, device=device) if want_wq else None
         self.loss = torch.empty((groups, rows, nblk), dtype=torch.float32, device=device) if want_loss else None
+        # bf16 fake-quantized weights, derived from the chosen codes by lhcal_apply_scales.
+        self.wq16 = torch.empty((groups, rows, cin), dtype=torch.bfloat16, device=device) if want_wq16 else None
         ws = 0 if self.mode == MSE else lhcal_accumulate_workspace(self.mode, x_dtype, tokens, cin, groups)
         if self.mode == ACT_AWARE and x_dtype == BF16:  # either activation-aware entry point
             ws = max(ws, lhcal_accumulate_act_quant_workspace(x_dtype, tokens, cin, groups))
@@ -362,7 +364,8 @@ def calibrate(mode, x, w, xq=None, group_offsets=None, token_ids=None, buffers: 
 
     x [T, C], w [G, R, C] (and for ``act`` either xq or act_gx, the input quantizer's global
     scale from which the kernel derives X_q; CSR routing for grouped layers) are device
-    tensors. Returns the buffers holding h, p, g, codes, wq and loss.
+    tensors. Returns the buffers holding h, p, g, codes, wq and loss (and the bf16 fake-quantized
+    weights wq16 when the buffers have them).
     """
     if stream is not None:  # enqueue everything on the given stream
         import torch
@@ -384,21 +387,25 @@ def calibrate(mode, x, w, xq=None, group_offsets=None, token_ids=None, buffers: 
 
 
 class HostOutputs:
-    """Pinned host copies of a calibration's results: the codes (the chosen block scales) and the
-    winning losses, and the fake-quantized weights when ``want_wq`` (they follow from the codes
-    through lhcal_apply_scales, so a caller may leave them on the device)."""
+    """Pinned host copies of a calibration's results: the codes (the chosen block scales), the
+    per-group global scales and the winning losses, plus the fake-quantized weights that the
+    buffers hold (fp32 ``wq`` when ``want_wq``, bf16 ``wq16`` when the buffers have it)."""
 
     def __init__(self, buffers: Buffers, want_wq: bool = True):
         import torch
 
         self.codes = torch.empty(buffers.codes.shape, dtype=torch.uint8, pin_memory=True)
+        self.g = torch.empty(buffers.g.shape, dtype=torch.float32, pin_memory=True)
         self.wq = (torch.empty(buffers.wq.shape, dtype=torch.float32, pin_memory=True)
                    if want_wq and buffers.wq is not None else None)
+        self.wq16 = (torch.empty(buffers.wq16.shape, dtype=torch.bfloat16, pin_memory=True)
+                     if getattr(buffers, "wq16", None) is not None else None)
         self.loss = None if buffers.loss is None else torch.empty(buffers.loss.shape, dtype=torch.float32,
                                                                    pin_memory=True)
 
     def nbytes(self) -> int:
-        return sum(t.numel() * t.element_size() for t in (self.codes, self.wq, self.loss) if t is not None)
+        return sum(t.numel() * t.element_size() for t in (self.codes, self.g, self.wq, self.wq16, self.loss)
+                   if t is not None)
 
 
 _side_streams: dict = {}
@@ -429,13 +436,16 @@ def _statistics(m, x, buffers, xq=None, group_offsets=None, token_ids=None, act_
 
 
 def _scales_and_sweep(m, w, buffers, e0: int, e1: int):
-    """Global scales and sweep of groups [e0, e1) on the current stream."""
+    """Global scales and sweep of groups [e0, e1) on the current stream, then the bf16
+    fake-quantized weights of the chosen codes when the buffers hold wq16."""
     b = buffers
     sl = slice(e0, e1)
     lhcal_global_scale(w[sl], b.g[sl])
     lhcal_scale_sweep(m, w[sl], None if b.h is None else b.h[sl], b.g[sl], b.codes[sl],
                       wq=None if b.wq is None else b.wq[sl], loss=None if b.loss is None else b.loss[sl],
                       p=None if b.p is None else b.p[sl])
+    if getattr(b, "wq16", None) is not None:
+        lhcal_apply_scales(w[sl], b.g[sl], b.codes[sl], wq16=b.wq16[sl])
 
 
 def calibrate_host(mode, x, w, buffers: Buffers, staging: dict, hxq=None, group_offsets=None, token_ids=None,
@@ -449,7 +459,8 @@ def calibrate_host(mode, x, w, buffers: Buffers, staging: dict, hxq=None, group_
     the current stream computes global scales and sweeps the chunks already resident, and each
     chunk's results are copied out on another side stream as soon as they are ready. A layer
     with one group copies its weights, computes the scale and sweeps. The results land in
-    ``out`` (codes, loss, and wq if requested); the function returns without synchronising,
+    ``out`` (codes, global scales, loss, and the fake-quantized weights it was made for: fp32
+    wq, or bf16 wq16 when the buffers hold it); the function returns without synchronising,
     and the current stream waits for every copy it issued.
     """
     import torch
@@ -488,6 +499,9 @@ def calibrate_host(mode, x, w, buffers: Buffers, staging: dict, hxq=None, group_
         with torch.cuda.stream(s_out):
             s_out.wait_event(done)
             out.codes[e0:e1].copy_(buffers.codes[e0:e1], non_blocking=True)
+            out.g[e0:e1].copy_(buffers.g[e0:e1], non_blocking=True)
+            if out.wq16 is not None:
+                out.wq16[e0:e1].copy_(buffers.wq16[e0:e1], non_blocking=True)
             if out.loss is not None:
                 out.loss[e0:e1].copy_(buffers.loss[e0:e1], non_blocking=True)
             if out.wq is not None:

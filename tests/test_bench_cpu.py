@@ -161,3 +161,19 @@ def test_clock_reason_names_exist_in_the_installed_nvml_binding():
     for _, const in bench.ClockSampler.REASONS:
         assert isinstance(getattr(pynvml, const, None), int), const
     assert callable(pynvml.nvmlDeviceGetCurrentClocksEventReasons)
+
+
+def test_headline_is_the_largest_workload_and_all_run_by_default():
+    """With no --workload every workload runs, and the line's headline is the one with the most
+    sweep units (the fused-MoE layer), so the largest single-GPU configuration is the number."""
+    import argparse
+
+    units = {n: bench.algorithmic(_shape_only(n))[0] for n in synth.WORKLOADS}
+    assert bench.HEADLINE == max(units, key=units.get) == "moe"
+    assert tuple(bench.ORDER) == tuple(synth.WORKLOADS)
+    assert bench.headline_name(argparse.Namespace(workload="all")) == "moe"
+    assert bench.headline_name(argparse.Namespace(workload="dense")) == "dense"
+
+
+def test_median_of_stage_times():
+    assert bench.median([3, 1, 2]) == 2 and bench.median([4, 1, 3, 2]) == 2.5

@@ -153,7 +153,9 @@ def _host_outputs(b):
     out = object.__new__(L.HostOutputs)  # plain CPU tensors in place of pinned ones
     out.codes = torch.full(b.codes.shape, 255, dtype=torch.uint8)
     out.loss = torch.full(b.loss.shape, -1.0)
+    out.g = torch.full(b.g.shape, -1.0)
     out.wq = None
+    out.wq16 = None
     return out
 
 
@@ -184,7 +186,7 @@ def test_calibrate_host_pipelines_groups_in_chunks(fake, fake_streams):
         assert _ptr(sw[2]) == staging["w"][e0].data_ptr() and _ptr(sw[6]) == b.h[e0].data_ptr()
         assert _ptr(sw[9]) == b.codes[e0].data_ptr() and _ptr(sw[11]) == b.loss[e0].data_ptr()
     # Every group's results came back.
-    assert torch.equal(out.codes, b.codes) and torch.equal(out.loss, b.loss)
+    assert torch.equal(out.codes, b.codes) and torch.equal(out.loss, b.loss) and torch.equal(out.g, b.g)
 
 
 def test_calibrate_host_reads_xq_only_when_the_caller_copies_it_in(fake, fake_streams):
