@@ -19,8 +19,10 @@
 //    Dense layers with enough slabs to fill a wave: clusters of up to 8 CTAs split a slab's
 //    tokens and reduce in distributed shared memory. Narrower dense layers: token splits write
 //    partials to the workspace, which reduce_partials_kernel sums in a fixed order. Grouped
-//    (MoE): a CTA walks a run of consecutive experts of its slab with one pipeline, gathering
-//    the routed rows through the CSR, and writes each expert's sums after its last tile.
+//    (MoE): a persistent grid deals the (slab, expert) pairs round-robin in slab-major order, so
+//    that the CTAs in flight share one or two slabs of X in L2; a CTA runs one pipeline through
+//    its pairs, gathering the routed rows through the CSR, and writes each expert's sums after
+//    its last tile.
 //    Activation-aware with the input quantizer fused (QUANT): only X streams in; each warp
 //    turns its block's 64 x 16 slice of the tile into X_q in shared memory (act_quant.cuh)
 //    and synchronises only with itself before the MMAs, so X is read from HBM once.
@@ -187,49 +189,51 @@ __device__ __forceinline__ void load_ids(int32_t* slot, const int32_t* ids, int6
   }
 }
 
-// One CTA owns a 128-column slab and a list of items: dense, one token range (a split, whose
-// sums go to the workspace); grouped, a run of consecutive groups (experts), each summed over
-// its routed rows and written to out at item * out_item_stride. A single cp.async pipeline runs
-// through the tiles of all items, so short items (about 5 tiles per expert) still stream; the
-// accumulators are written out after each item's last tile. accumulate_into: out += sums.
-// QUANT (with ACT): xq is unused and X_q comes from X through the input quantizer with the
-// global scale *act_gx.
+// A CTA works through a list of items, each a (128-column slab, row set) pair. Dense: one item,
+// slab blockIdx.x and token range blockIdx.y (a split, whose sums go to the workspace at
+// split * out_item_stride). Grouped: the (slab, expert) pairs in slab-major order q = slab *
+// groups + expert, dealt round-robin over the persistent grid (CTA c takes q = c, c + gridDim.x,
+// ...), each summed over the expert's routed rows and written at expert * out_item_stride. The
+// CTAs of a wave therefore work on one or two slabs at a time, whose rows (4 MB per slab) stay
+// in L2 while the experts gather them. A single cp.async pipeline runs through the tiles of all
+// items, so short items (about 5 tiles per expert) still stream; the accumulators are written
+// out after each item's last tile. accumulate_into: out += sums. QUANT (with ACT): xq is unused
+// and X_q comes from X through the input quantizer with the global scale *act_gx.
 template <bool ACT, bool QUANT, bool CLUSTER>
 __global__ void __launch_bounds__(kMmaThreads, QUANT ? 3 : 1)
 accum_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ xq,
                  int64_t tokens, int64_t cin, int64_t ldx, const int32_t* __restrict__ group_offsets,
-                 const int32_t* __restrict__ token_ids, int64_t tok_per_split, int64_t items_per_cta,
+                 const int32_t* __restrict__ token_ids, int64_t tok_per_split, int64_t total_items,
                  int64_t groups, float* __restrict__ out_h, float* __restrict__ out_p,
                  int64_t out_item_stride, int accumulate_into, const float* __restrict__ act_gx) {
   static_assert(ACT || !QUANT, "the input quantizer belongs to the activation-aware mode");
   using Cfg = MmaCfg<ACT, QUANT>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t slab = blockIdx.x;
-  const int64_t col0 = slab * kSlabCols;
   const int64_t nblk = cin / kBlock;
-  const int64_t blk = slab * 8 + warp;
-  const bool blk_ok = blk < nblk;
   const bool grouped = group_offsets != nullptr;
 
-  int64_t it0, it1;  // this CTA's items
+  // This CTA's items are it0 <= item < it1. Grouped: item t is the pair q = blockIdx.x + t *
+  // gridDim.x; dense: the one item blockIdx.y (the token split) of slab blockIdx.x.
+  int64_t it0, it1;
   if (grouped) {
-    it0 = static_cast<int64_t>(blockIdx.y) * items_per_cta;
-    it1 = imin64(groups, it0 + items_per_cta);
+    it0 = 0;
+    it1 = total_items > blockIdx.x ? ceil_div(total_items - blockIdx.x, gridDim.x) : 0;
   } else {
     it0 = blockIdx.y;
     it1 = it0 + 1;
   }
-  // Grouped: this CTA's slice of the offsets, staged in shared memory after the pipeline ring.
-  int32_t* offs_s = reinterpret_cast<int32_t*>(smem + Cfg::kSmem);
-  if (grouped) {
-    for (int64_t i = threadIdx.x; i <= it1 - it0; i += kMmaThreads) offs_s[i] = __ldg(group_offsets + it0 + i);
-    __syncthreads();
-  }
+  // Pair indices fit in 32 bits: groups <= 65535 and slabs <= 65535 / 8 (checked by the API).
+  const uint32_t ngroups = static_cast<uint32_t>(groups);
+  auto pair_of = [&](int64_t item) { return blockIdx.x + static_cast<uint32_t>(item) * gridDim.x; };
+  auto slab_of = [&](int64_t item) -> int64_t { return grouped ? pair_of(item) / ngroups : blockIdx.x; };
+  // Index of the item's sums in out (expert, or token split).
+  auto out_of = [&](int64_t item) -> int64_t { return grouped ? pair_of(item) % ngroups : item; };
   auto range = [&](int64_t item, int64_t& b, int64_t& e) {
     if (grouped) {
-      b = offs_s[item - it0];
-      e = offs_s[item - it0 + 1];
+      const uint32_t ex = pair_of(item) % ngroups;
+      b = __ldg(group_offsets + ex);
+      e = __ldg(group_offsets + ex + 1);
     } else {
       b = item * tok_per_split;
       e = imin64(tokens, b + tok_per_split);
@@ -237,11 +241,14 @@ accum_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __res
   };
 
   // Accumulator layout of m16n8: c0,c1 -> (i = lane/4, j = 2*(lane%4) + {0,1}); c2,c3 -> i + 8.
+  // Sums are written with streaming stores: they are not read again by this launch and should
+  // not displace the activation rows that other CTAs are still gathering from L2.
   const int i0 = lane >> 2, j0 = 2 * (lane & 3);
   auto write_out = [&](int64_t item, const float (&ah)[2][4], const float (&ap)[2][4]) {
-    if (!blk_ok) return;
-    float* oh = out_h + item * out_item_stride + blk * 256;
-    float* op = ACT ? out_p + item * out_item_stride + blk * 256 : nullptr;
+    const int64_t blk = slab_of(item) * 8 + warp;
+    if (blk >= nblk) return;
+    float* oh = out_h + out_of(item) * out_item_stride + blk * 256;
+    float* op = ACT ? out_p + out_of(item) * out_item_stride + blk * 256 : nullptr;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
@@ -253,7 +260,7 @@ accum_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __res
           vh.x += o.x;
           vh.y += o.y;
         }
-        *reinterpret_cast<float2*>(oh + idx) = vh;
+        __stcs(reinterpret_cast<float2*>(oh + idx), vh);
         if (ACT) {
           float2 vp = make_float2(ap[nt][2 * half], ap[nt][2 * half + 1]);
           if (accumulate_into) {
@@ -261,7 +268,7 @@ accum_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __res
             vp.x += o.x;
             vp.y += o.y;
           }
-          *reinterpret_cast<float2*>(op + idx) = vp;
+          __stcs(reinterpret_cast<float2*>(op + idx), vp);
         }
       }
     }
@@ -312,7 +319,6 @@ accum_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __res
   int64_t i_tile = 0;
   int64_t p_item = first_nonempty(it0, p_pos, p_end);
   int64_t c_item = first_nonempty(it0, c_pos, c_end);
-  (void)p_item;
   auto issue_ids = [&]() {  // ids of tile i_tile into slot i_tile % S
     if (grouped && i_tile < ntiles) {
       load_ids(ids_ring + (i_tile % S) * kTileTok, token_ids, i_pos, i_end);
@@ -322,8 +328,8 @@ accum_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __res
     ++i_tile;
   };
   auto produce = [&](int64_t tile) {  // data of tile into stage tile % S
-    load_tile<Cfg::kTwo>(smem + (tile % S) * stage_bytes, x, xq, ldx, col0, cin,
-                   grouped ? ids_ring + (tile % S) * kTileTok : nullptr, p_pos, p_end);
+    load_tile<Cfg::kTwo>(smem + (tile % S) * stage_bytes, x, xq, ldx, slab_of(p_item) * kSlabCols, cin,
+                         grouped ? ids_ring + (tile % S) * kTileTok : nullptr, p_pos, p_end);
     p_pos += kTileTok;
     if (p_pos >= p_end) p_item = first_nonempty(p_item + 1, p_pos, p_end);
   };
@@ -441,7 +447,7 @@ accum_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __res
     const int csize = static_cast<int>(cluster.num_blocks());
     const int rank = static_cast<int>(cluster.block_rank());
     for (int b = rank; b < 8; b += csize) {  // blocks of the slab this CTA finishes
-      const int64_t ob = slab * 8 + b;
+      const int64_t ob = static_cast<int64_t>(blockIdx.x) * 8 + b;
       if (ob < nblk) {
         const int t = threadIdx.x;  // 256 threads: one entry of the 16 x 16 block each
         float vh = 0.f, vp = 0.f;
@@ -713,14 +719,11 @@ lhcal_status launch_mma(const void* x, const void* xq, int64_t tokens, int64_t c
   const auto* xb = static_cast<const __nv_bfloat16*>(x);
   const auto* xqb = static_cast<const __nv_bfloat16*>(Cfg::kTwo ? xq : x);
   if (offs != nullptr) {
-    // Runs of experts per CTA so that about one wave of CTAs covers all (slab, expert) items.
-    const int64_t ctas_per_sm = Cfg::kResident;
-    const int64_t per = imax64(1, ceil_div(static_cast<int64_t>(groups) * slabs, ctas_per_sm * kNumSms));
-    const dim3 grid(static_cast<unsigned>(slabs), static_cast<unsigned>(ceil_div(groups, per)));
-    const size_t smem = Cfg::kSmem + static_cast<size_t>(ceil_div((per + 1) * 4, 16) * 16);
-    if (smem > static_cast<size_t>(kMaxDynSmem)) return fail(LHCAL_ERR_UNSUPPORTED, "accumulate: too many groups per CTA");
-    accum_mma_kernel<ACT, QUANT, false><<<grid, kMmaThreads, smem, stream>>>(
-        xb, xqb, tokens, cin, ldx, offs, ids, 0, per, groups, h, p, nblk * 256, accumulate_into, act_gx);
+    // One persistent wave of resident CTAs dealt the (slab, expert) pairs round-robin.
+    const int64_t total = static_cast<int64_t>(groups) * slabs;
+    const int64_t ctas = imin64(total, static_cast<int64_t>(Cfg::kResident) * kNumSms);
+    accum_mma_kernel<ACT, QUANT, false><<<static_cast<unsigned>(ctas), kMmaThreads, Cfg::kSmem, stream>>>(
+        xb, xqb, tokens, cin, ldx, offs, ids, 0, total, groups, h, p, nblk * 256, accumulate_into, act_gx);
     return check_launch("accumulate (grouped, tensor cores)");
   }
   const DensePlan pl = dense_plan(ACT ? LHCAL_ACT_AWARE : LHCAL_FULL, tokens, cin, Cfg::kResident, Cfg::kClusterFill);
