@@ -31,8 +31,18 @@
 // Work per candidate. Candidates below the warp's first unclamped one take a closed form;
 // the rest go four per loop trip, and the quad's four lanes share the reduction of four
 // candidates (a transposed reduction: lane t ends with candidate k + t) and keep their own
-// bests, merged after the loop. The per-unit set-up reads the units' weights from shared
-// memory, and the grid runs the 16-column blocks fastest.
+// bests, merged after the loop. The argmin compares L - C' (C' is the same for all of a
+// unit's candidates); the winner's loss is then recomputed by its definition.
+//
+// Set-up per CTA (128 rows of one block). The rows' weights are staged in shared memory once;
+// each row's first unclamped candidate kfirst comes from a binary search of the top-level
+// thresholds, and a stable counting sort by kfirst (match_any over each warp, per-warp
+// histograms, one scan) orders the rows, so that a warp's 16 units leave the clamped regime
+// together and its first full candidate is the first of its sorted range. U' and H sign(w)
+// are 16-term dot products with rows of (H + H^T) / 2 read four at a time. The grid runs the
+// 16-column blocks fastest.
+#include <cstddef>
+
 #include "common.cuh"
 #include "quant_tables.cuh"
 
@@ -54,19 +64,32 @@ constexpr int kUnitsPerCta = kUnitsPerWarp * kTcWarps;
 constexpr int kEntryBytes = 16;                 // {thr, q16 (low half), q16 << 16, val}
 constexpr int kTabRowBytes = kLev * kEntryBytes;  // one candidate
 
+constexpr int kWStride = kBlock + 4;  // floats per staged weight row (16-byte aligned, see below)
+static_assert(kTcWarps >= 5 && kUnitsPerCta == 128, "the set-up uses warps 0-4 and 4 warps of rows");
+
+// Arrays read with 16-byte loads are declared 16-byte aligned (a member is otherwise aligned
+// only to its element type); the static_asserts after the struct check the offsets.
 struct __align__(16) TcShared {
   float4 tab[kCand * kLev];
+  alignas(16) float h[256];
+  alignas(16) float p[256];
+  alignas(16) float hs[256];  // (H + H^T) / 2
+  // The CTA's 128 rows' weights (fp32), row stride 20 floats (80 bytes): the 8 rows that a
+  // warp's lane groups read at once with 16-byte loads then fall in distinct banks.
+  alignas(16) float wall[kUnitsPerCta][kWStride];
   float rho[kCand];  // -2 / (s_k * 2^eH): scale of U' in the MMA accumulator
   float s2[kCand];   // s_k^2 * 2^eH
-  float h[256];
-  float p[256];
   float hscale;  // 2^-eH: H' = H * hscale lies below 2^15
-  float key[kUnitsPerCta];  // min |w| of each of the CTA's units (rows)
-  int perm[kUnitsPerCta];   // the CTA's rows ordered by key
-  // Each warp's 16 units' weights (fp32), rows padded to 17 floats so that the 8 units a warp
-  // reads at once fall in distinct banks. Read by the per-unit set-up and the ACT epilogue.
-  float wst[kTcWarps][kUnitsPerWarp][kBlock + 1];
+  int kfirst[kUnitsPerCta];  // per row: first candidate with an element below the top level
+  int perm[kUnitsPerCta];    // the CTA's rows in ascending kfirst (stable)
+  int kf_sorted[kUnitsPerCta];
+  int hist[4][kUnitsPerCta];  // per warp of rows, per kfirst value: rows of that warp
+  int base[kUnitsPerCta];     // rows with a smaller kfirst
 };
+static_assert(offsetof(TcShared, tab) % 16 == 0 && offsetof(TcShared, h) % 16 == 0 &&
+                  offsetof(TcShared, p) % 16 == 0 && offsetof(TcShared, hs) % 16 == 0 &&
+                  offsetof(TcShared, wall) % 16 == 0 && (kWStride * sizeof(float)) % 16 == 0,
+              "16-byte shared-memory accesses need 16-byte aligned rows");
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -109,11 +132,13 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t v) {
   return __half22float2(*reinterpret_cast<const __half2*>(&v));
 }
 
-// Level of magnitude a at candidate row k of the table, by counting thresholds.
+// Level of magnitude a at candidate row k of the table: the largest j with a >= thr[k][j], by a
+// three-step binary search (the thresholds rise with j for s > 0; for s = 0 every level's
+// value is 0, so whichever level it returns gives the same fake-quant value).
 __device__ __forceinline__ int level_direct_tc(const float4* tab_k, float a) {
-  int lev = 0;
-#pragma unroll
-  for (int j = 1; j < kLev; ++j) lev += (a >= tab_k[j].x) ? 1 : 0;
+  int lev = (a >= tab_k[4].x) ? 4 : 0;
+  lev += (a >= tab_k[lev + 2].x) ? 2 : 0;
+  lev += (a >= tab_k[lev + 1].x) ? 1 : 0;
   return lev;
 }
 
@@ -142,10 +167,12 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, tq = lane & 3;
 
-  // ---- per-CTA set-up: H (and P) of block n, the H scale, candidate tables
+  // ---- per-CTA set-up: H (and P) of block n, its symmetric part, candidate tables
   const int64_t hblk = e * nblk + n;
   for (int i = threadIdx.x; i < 256; i += kTcThreads) {
-    sh.h[i] = __ldg(h + hblk * 256 + i);
+    const float hv = __ldg(h + hblk * 256 + i);
+    sh.h[i] = hv;
+    sh.hs[i] = 0.5f * (hv + __ldg(h + hblk * 256 + (i & 15) * 16 + (i >> 4)));
     if (ACT) sh.p[i] = __ldg(p + hblk * 256 + i);
   }
   const float gs = __ldg(g + e);
@@ -156,51 +183,88 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
     sh.tab[idx] = make_float4(level_threshold(j, s), __uint_as_float(q16), __uint_as_float(q16 << 16),
                               __fmul_rn(e2m1_grid(j), s));
   }
-  // Order the CTA's rows by their smallest |w|, so that the units a warp evaluates together
-  // leave the all-clamped candidates at similar scales (see the clamped prefix below).
+  for (int i = threadIdx.x; i < 4 * kUnitsPerCta; i += kTcThreads) (&sh.hist[0][0])[i] = 0;
   const int64_t rbase = static_cast<int64_t>(blockIdx.y) * kUnitsPerCta;
+  __syncthreads();
+  // Each of the CTA's rows: weights staged in shared memory, and kfirst, the first candidate at
+  // which one of its 16 weights falls below the top E2M1 level (|w| < thr[k][7]); before it the
+  // unit's loss has a closed form (below). Rows past the end get kCand and sort last.
   if (threadIdx.x < kUnitsPerCta) {
     const int64_t row = rbase + threadIdx.x;
+    const bool ok = row < rows;
+    float wt[16];
+    load_row16<WT>(w + (e * rows + (ok ? row : 0)) * cin + n * kBlock, ok, wt);
     float m = __int_as_float(0x7f800000);
-    if (row < rows) {
-      float wt[16];
-      load_row16<WT>(w + (e * rows + row) * cin + n * kBlock, true, wt);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) m = fminf(m, fabsf(wt[i]));
+    for (int i = 0; i < 16; i += 4) {
+      *reinterpret_cast<float4*>(&sh.wall[threadIdx.x][i]) = make_float4(wt[i], wt[i + 1], wt[i + 2], wt[i + 3]);
+      m = fminf(fminf(fabsf(wt[i]), fabsf(wt[i + 1])), fminf(fminf(fabsf(wt[i + 2]), fabsf(wt[i + 3])), m));
     }
-    sh.key[threadIdx.x] = m;
-  }
-  __syncthreads();
-  if (threadIdx.x < kUnitsPerCta) {
-    const float my = sh.key[threadIdx.x];
-    int rank = 0;
-    for (int j = 0; j < kUnitsPerCta; ++j) {
-      const float kj = sh.key[j];
-      rank += (kj < my || (kj == my && j < static_cast<int>(threadIdx.x))) ? 1 : 0;
+    int lo = 0, hi = kCand;  // first k with m < thr[k][7]
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (m < sh.tab[kLev * mid + 7].x) hi = mid; else lo = mid + 1;
     }
-    sh.perm[rank] = threadIdx.x;
-  }
-  if (warp == 0) {
+    const int kf = ok ? lo : kCand;
+    sh.kfirst[threadIdx.x] = kf;
+    // Stable counting sort by kfirst, step 1: rows of this warp per kfirst value.
+    const uint32_t same = __match_any_sync(0xffffffffu, kf);
+    if (lane == __ffs(same) - 1) sh.hist[warp][kf] = __popc(same);
+  } else if (warp == 4) {
+    // Scale H so that its largest |H'| lies in [2^14, 2^15): below the fp16 maximum.
     uint32_t m = 0;
     for (int i = lane; i < 256; i += 32) m = max(m, __float_as_uint(sh.h[i]) & 0x7fffffffu);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
     if (lane == 0) {
-      // Scale so that the largest |H'| lies in [2^14, 2^15): below the fp16 maximum.
       const int ex = (m == 0u) ? 0 : static_cast<int>(m >> 23) - 127;  // floor(log2 max|H|)
-      const int sh_exp = min(127, max(-126, 14 - ex));
-      sh.hscale = pow2i(sh_exp);
+      sh.hscale = pow2i(min(127, max(-126, 14 - ex)));
     }
   }
   __syncthreads();
-  const float hscale = sh.hscale;
-  const float inv_hscale = 1.0f / hscale;  // exact: a power of two
-  for (int k = threadIdx.x; k < kCand; k += kTcThreads) {
-    const float s = candidate_scale(k, gs);
-    sh.rho[k] = -2.f * hscale / s;
-    sh.s2[k] = (s * s) * inv_hscale;
+  if (warp == 0) {
+    // Step 2: base[v] = rows with kfirst < v (an exclusive scan over the 127 values).
+    int c[4], run = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int v = 4 * lane + j;
+      c[j] = sh.hist[0][v] + sh.hist[1][v] + sh.hist[2][v] + sh.hist[3][v];
+      run += c[j];
+    }
+    int incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    int b = incl - run;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      sh.base[4 * lane + j] = b;
+      b += c[j];
+    }
+  } else if (warp == 1) {
+    const float hscale = sh.hscale;
+    const float inv_hscale = 1.0f / hscale;  // exact: a power of two
+    for (int k = lane; k < kCand; k += 32) {
+      const float s = candidate_scale(k, gs);
+      sh.rho[k] = -2.f * hscale / s;
+      sh.s2[k] = (s * s) * inv_hscale;
+    }
   }
   __syncthreads();
+  if (threadIdx.x < kUnitsPerCta) {
+    // Step 3: position = rows with a smaller kfirst + rows of earlier warps with the same one
+    // + lanes of this warp before this one with the same one (ties keep the row order).
+    const int kf = sh.kfirst[threadIdx.x];
+    const uint32_t same = __match_any_sync(0xffffffffu, kf);
+    int pos = sh.base[kf] + __popc(same & ((1u << lane) - 1u));
+    for (int w2 = 0; w2 < warp; ++w2) pos += sh.hist[w2][kf];
+    sh.perm[pos] = threadIdx.x;
+    sh.kf_sorted[pos] = kf;
+  }
+  __syncthreads();
+  const float hscale = sh.hscale;
 
   // ---- B fragments: H' = H * hscale as fp16 hi + lo. B[k][n] = H'[k][n].
   uint32_t bhi[2][2], blo[2][2];
@@ -217,94 +281,68 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
     }
   }
 
-  // ---- the warp's 16 units: sorted positions 16 warp + gq (unit 0) and + 8 (unit 1). Their
-  // weights go to shared memory (lane l loads half l & 1 of unit l / 2), so that the set-up
-  // below reads them instead of holding 32 of them in registers.
-  float (*wst)[kBlock + 1] = sh.wst[warp];
-  {
-    const int j = lane >> 1, h8 = (lane & 1) * 8;
-    const int64_t row = rbase + sh.perm[warp * kUnitsPerWarp + j];
-    const bool ok = row < rows;
-    float w8[8];
-    if (ok) load8<WT>(w + (e * rows + row) * cin + n * kBlock + h8, w8);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) wst[j][h8 + k] = ok ? w8[k] : 0.f;
-  }
-  __syncwarp();
-  bool valid[2];
-#pragma unroll
-  for (int u = 0; u < 2; ++u) valid[u] = rbase + sh.perm[warp * kUnitsPerWarp + gq + 8 * u] < rows;
+  // ---- the warp's 16 units: sorted positions 16 warp + gq (unit 0) and + 8 (unit 1); the
+  // warp's first candidate to evaluate in full is the smallest kfirst of its units, the first
+  // of its sorted range.
+  const int kstart = sh.kf_sorted[warp * kUnitsPerWarp];
   // Lane element i (0..7): unit i / 4, column col_of(i % 4) with columns {2t, 2t+1, 2t+8, 2t+9}.
   auto col_of = [&](int ci) { return 2 * tq + (ci & 1) + 8 * (ci >> 1); };
   float a[8], up[8];
   uint32_t sgn[8];
-  float cpart[2] = {0.f, 0.f};
-  float pqa[2] = {0.f, 0.f}, pqb[2] = {0.f, 0.f}, amin[2];
+  float pa[2], pb[2];
 #pragma unroll
   for (int u = 0; u < 2; ++u) {
-    amin[u] = __int_as_float(0x7f800000);
+    // The unit's 16 weights and their signs (+-1), then per lane column c of the unit:
+    // U'_c = (Hs w)_c - (P w)_c and (Hs sign(w))_c, as 16-term dot products with the rows of
+    // Hs (and P) read four at a time.
+    const float* wr = sh.wall[sh.perm[warp * kUnitsPerWarp + gq + 8 * u]];
+    float wv[16], sv[16];
+#pragma unroll
+    for (int k = 0; k < 16; k += 4) {
+      const float4 q = *reinterpret_cast<const float4*>(wr + k);
+      wv[k] = q.x; wv[k + 1] = q.y; wv[k + 2] = q.z; wv[k + 3] = q.w;
+    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) sv[k] = copysignf(1.f, wv[k]);
+    float qa = 0.f, qb = 0.f;
 #pragma unroll
     for (int ci = 0; ci < 4; ++ci) {
       const int c = col_of(ci);
       const int i = 4 * u + ci;
-      const float* wr = wst[gq + 8 * u];
-      const float x = wr[c];
-      a[i] = fabsf(x);
-      amin[u] = fminf(amin[u], a[i]);
-      sgn[i] = __float_as_uint(x) >> 31;
-      float hw_sym = 0.f, hw_row = 0.f, pw = 0.f, hsg = 0.f;
+      const float* hr = sh.hs + c * 16;
+      float hw = 0.f, hsg = 0.f, pw = 0.f;
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const float hck = sh.h[c * 16 + k];
-        const float wk = wr[k];
-        hw_sym = fmaf(0.5f * (hck + sh.h[k * 16 + c]), wk, hw_sym);
-        hw_row = fmaf(hck, wk, hw_row);
-        hsg += (__float_as_uint(wk) >> 31) ? -hck : hck;  // (H sign(w))_c
-        if (ACT) pw = fmaf(sh.p[c * 16 + k], wk, pw);
+      for (int k = 0; k < 16; k += 4) {
+        const float4 hq = *reinterpret_cast<const float4*>(hr + k);
+        hw = fmaf(hq.x, wv[k], hw); hw = fmaf(hq.y, wv[k + 1], hw);
+        hw = fmaf(hq.z, wv[k + 2], hw); hw = fmaf(hq.w, wv[k + 3], hw);
+        hsg = fmaf(hq.x, sv[k], hsg); hsg = fmaf(hq.y, sv[k + 1], hsg);
+        hsg = fmaf(hq.z, sv[k + 2], hsg); hsg = fmaf(hq.w, sv[k + 3], hsg);
+        if (ACT) {
+          const float4 pq = *reinterpret_cast<const float4*>(sh.p + c * 16 + k);
+          pw = fmaf(pq.x, wv[k], pw); pw = fmaf(pq.y, wv[k + 1], pw);
+          pw = fmaf(pq.z, wv[k + 2], pw); pw = fmaf(pq.w, wv[k + 3], pw);
+        }
       }
-      up[i] = hw_sym - pw;                               // U'_c
-      cpart[u] = fmaf(x, hw_row - 2.f * pw, cpart[u]);  // w_c ((H w)_c - 2 (P w)_c)
-      const float sc = sgn[i] ? -1.f : 1.f;
-      pqa[u] = fmaf(sc, hsg, pqa[u]);
-      pqb[u] = fmaf(sc, up[i], pqb[u]);
+      const float x = wr[c];  // from shared memory: c depends on the lane
+      const float sc = copysignf(1.f, x);
+      a[i] = fabsf(x);
+      sgn[i] = __float_as_uint(x) >> 31;
+      up[i] = hw - pw;  // U'_c
+      qa = fmaf(sc, hsg, qa);
+      qb = fmaf(sc, up[i], qb);
     }
-  }
-  float cconst[2];
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    float v = cpart[u];
-    v += __shfl_xor_sync(0xffffffffu, v, 1);
-    v += __shfl_xor_sync(0xffffffffu, v, 2);
-    cconst[u] = v;  // C' of the unit
-  }
-  // While every element of a unit is clamped at the top of the grid (|w_i| >= thr[k][7], so
-  // v = 6 sign(w)), its loss is the parabola 36 s^2 sign^T H sign - 12 s sign^T U' + C'.
-  // kfirst = first candidate at which some element of the unit is below the top level.
-  float pa[2], pb[2];
-  int kfirst_lane = kCand;
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    float m = amin[u], qa = pqa[u], qb = pqb[u];
+    // Over the quad: sign^T Hs sign and sign^T U'. While every element of the unit is clamped
+    // at the top of the grid (v = 6 sign(w)), its scale-dependent loss is the parabola
+    // 36 s^2 sign^T H sign - 12 s sign^T U'.
 #pragma unroll
     for (int o = 1; o <= 2; o <<= 1) {
-      m = fminf(m, __shfl_xor_sync(0xffffffffu, m, o));
       qa += __shfl_xor_sync(0xffffffffu, qa, o);
       qb += __shfl_xor_sync(0xffffffffu, qb, o);
     }
     pa[u] = 36.f * qa;
     pb[u] = -12.f * qb;
-    if (valid[u]) {
-      int lo = 0, hi = kCand;  // first k with m < thr[k][7]
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (m < sh.tab[kLev * mid + 7].x) hi = mid; else lo = mid + 1;
-      }
-      kfirst_lane = min(kfirst_lane, lo);
-    }
   }
-  int kstart = kfirst_lane;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) kstart = min(kstart, __shfl_xor_sync(0xffffffffu, kstart, o));
   // Sign masks of the four packed A registers: a0 = (elems 0,1), a1 = (4,5), a2 = (2,3), a3 = (6,7).
   constexpr int kPairLo[4] = {0, 4, 2, 6};
   uint32_t smask[4];
@@ -320,7 +358,9 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
 
   // One candidate: A fragment from the elements' packed fp16 grid values; the accumulator starts
   // at rho_k U', so after the 4 MMAs D = v^T H' + rho_k U' and
-  //   L = s2_k * sum_n v_n D_n + C' = s^2 v^T H v - 2 s v^T U' + C'.
+  //   L - C' = s2_k * sum_n v_n D_n = s^2 v^T H v - 2 s v^T U'.
+  // C' is the same for every candidate of a unit, so the argmin compares L - C'; the winner's
+  // loss is recomputed by its definition after the sweep.
   // The lane's share of t for units 0 and 1 (its 4 columns), before the reduction over the quad.
   auto partials = [&](const uint32_t (&q)[8], int k, float (&tp)[2]) {
     uint32_t afr[4];
@@ -352,7 +392,7 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
     t0 += __shfl_xor_sync(0xffffffffu, t0, 2);
     t1 += __shfl_xor_sync(0xffffffffu, t1, 2);
     const float s2 = sh.s2[k];
-    const float L0 = fmaf(s2, t0, cconst[0]), L1 = fmaf(s2, t1, cconst[1]);
+    const float L0 = s2 * t0, L1 = s2 * t1;
     if (L0 < best[0]) {
       best[0] = L0;
       best_k[0] = k;
@@ -369,7 +409,7 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
     const float sk = sh.tab[kLev * k + 2].w;  // grid value 1 times s_k
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      const float L = fmaf(fmaf(pa[u], sk, pb[u]), sk, cconst[u]);
+      const float L = fmaf(pa[u], sk, pb[u]) * sk;
       if (L < best[u]) {
         best[u] = L;
         best_k[u] = k;
@@ -446,7 +486,7 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const float t = (b1 ? spair[1][u] : spair[0][u]) + __shfl_xor_sync(0xffffffffu, b1 ? spair[0][u] : spair[1][u], 2);
-      const float L = fmaf(s2, t, cconst[u]);
+      const float L = s2 * t;
       if (L < best[u]) {
         best[u] = L;
         best_k[u] = kk;
@@ -504,8 +544,8 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
       float hd = 0.f;
 #pragma unroll
       for (int k = 0; k < 16; ++k) hd = fmaf(sh.h[c * 16 + k], dfull[k], hd);
-      if (ACT) {  // + 2 (P w)_c, with w from the warp's shared copy
-        const float* wr = wst[gq + 8 * u];
+      if (ACT) {  // + 2 (P w)_c, with w from the CTA's shared copy
+        const float* wr = sh.wall[sh.perm[warp * kUnitsPerWarp + gq + 8 * u]];
         float pw = 0.f;
 #pragma unroll
         for (int k = 0; k < 16; ++k) pw = fmaf(sh.p[c * 16 + k], wr[k], pw);
