@@ -114,6 +114,7 @@ constexpr int kSlabCols = 128;    // 8 blocks of 16 columns
 constexpr int kTileTok = 64;
 constexpr int kRowBytes = kSlabCols * 2;              // 256 B per token row of the slab
 constexpr int kTileBytes = kTileTok * kRowBytes;      // 16 KB per tensor per stage
+constexpr int64_t kMaxStagedItems = 1024;             // grouped items per CTA (16 KB of item records)
 
 // Shared memory: the cp.async ring (X_q and X per stage for ACT, X for FULL and QUANT), the
 // token-id ring, and for QUANT the X_q tile the warps write plus the quantizer tables.
@@ -225,15 +226,27 @@ accum_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __res
   }
   // Pair indices fit in 32 bits: groups <= 65535 and slabs <= 65535 / 8 (checked by the API).
   const uint32_t ngroups = static_cast<uint32_t>(groups);
-  auto pair_of = [&](int64_t item) { return blockIdx.x + static_cast<uint32_t>(item) * gridDim.x; };
-  auto slab_of = [&](int64_t item) -> int64_t { return grouped ? pair_of(item) / ngroups : blockIdx.x; };
+  // Grouped: each of this CTA's items as {first row position, end, slab, expert}, staged in
+  // shared memory after the pipeline (every cursor looks them up at each item boundary; a
+  // global load or a division there would stall the whole CTA).
+  int4* items_s = reinterpret_cast<int4*>(smem + Cfg::kSmem);
+  if (grouped) {
+    for (int64_t t = threadIdx.x; t < it1; t += kMmaThreads) {
+      const uint32_t q = blockIdx.x + static_cast<uint32_t>(t) * gridDim.x;
+      const uint32_t ex = q % ngroups;
+      items_s[t] = make_int4(__ldg(group_offsets + ex), __ldg(group_offsets + ex + 1), static_cast<int>(q / ngroups),
+                             static_cast<int>(ex));
+    }
+    __syncthreads();
+  }
+  auto slab_of = [&](int64_t item) -> int64_t { return grouped ? items_s[item].z : blockIdx.x; };
   // Index of the item's sums in out (expert, or token split).
-  auto out_of = [&](int64_t item) -> int64_t { return grouped ? pair_of(item) % ngroups : item; };
+  auto out_of = [&](int64_t item) -> int64_t { return grouped ? items_s[item].w : item; };
   auto range = [&](int64_t item, int64_t& b, int64_t& e) {
     if (grouped) {
-      const uint32_t ex = pair_of(item) % ngroups;
-      b = __ldg(group_offsets + ex);
-      e = __ldg(group_offsets + ex + 1);
+      const int4 r = items_s[item];
+      b = r.x;
+      e = r.y;
     } else {
       b = item * tok_per_split;
       e = imin64(tokens, b + tok_per_split);
@@ -719,10 +732,13 @@ lhcal_status launch_mma(const void* x, const void* xq, int64_t tokens, int64_t c
   const auto* xb = static_cast<const __nv_bfloat16*>(x);
   const auto* xqb = static_cast<const __nv_bfloat16*>(Cfg::kTwo ? xq : x);
   if (offs != nullptr) {
-    // One persistent wave of resident CTAs dealt the (slab, expert) pairs round-robin.
+    // One persistent wave of resident CTAs dealt the (slab, expert) pairs round-robin; more CTAs
+    // (several waves) only when a CTA's item ranges would not fit its shared-memory staging.
     const int64_t total = static_cast<int64_t>(groups) * slabs;
-    const int64_t ctas = imin64(total, static_cast<int64_t>(Cfg::kResident) * kNumSms);
-    accum_mma_kernel<ACT, QUANT, false><<<static_cast<unsigned>(ctas), kMmaThreads, Cfg::kSmem, stream>>>(
+    const int64_t ctas = imin64(total, imax64(static_cast<int64_t>(Cfg::kResident) * kNumSms,
+                                              ceil_div(total, kMaxStagedItems)));
+    const size_t smem = Cfg::kSmem + static_cast<size_t>(ceil_div(total, ctas)) * sizeof(int4);
+    accum_mma_kernel<ACT, QUANT, false><<<static_cast<unsigned>(ctas), kMmaThreads, smem, stream>>>(
         xb, xqb, tokens, cin, ldx, offs, ids, 0, total, groups, h, p, nblk * 256, accumulate_into, act_gx);
     return check_launch("accumulate (grouped, tensor cores)");
   }
