@@ -529,6 +529,95 @@ def measure_workload(name, args, rank, world, dev, flusher):
     return rec
 
 
+def measure_sharded(name, args, rank, world, dev):
+    """One layer shared by the ranks (scale_calibration_lh_b200.sharded): each rank accumulates its
+    token shard, one all-reduce (SUM) of the raw statistics and counts, each rank finalizes and
+    sweeps its row shard (the global scale is the all-reduce MAX of the shards'). A step is one
+    such calibration without gathering the results; value = the layer's units over the slowest
+    rank's step time (strong scaling)."""
+    import torch
+
+    import scale_calibration_lh_b200 as L
+    from scale_calibration_lh_b200 import sharded as S
+    from scale_calibration_lh_b200 import synth
+
+    layer = synth.make_layer(name, 0, rows=args.rows)
+    G, R, C, T = layer.groups, layer.rows, layer.cin, layer.tokens
+    t0, t1 = S.token_range(T, rank, world)
+    r0, r1 = S.row_range(R, rank, world)
+    kind = "bf16" if layer.dtype == "bf16" else "f32"
+    x = synth.to_device(layer.x[t0:t1], kind, dev)
+    w = synth.to_device(layer.w[:, r0:r1], kind, dev)
+    offs = ids = None
+    if layer.group_offsets is not None:
+        o, i = S.shard_routing(torch.from_numpy(layer.group_offsets), torch.from_numpy(layer.token_ids), t0, t1)
+        offs, ids = o.to(dev), i.to(dev)
+    mode = L.MODE_IDS[layer.mode]
+    buf = L.Buffers(mode, t1 - t0, C, r1 - r0, G, L.BF16 if kind == "bf16" else L.F32, dev)
+    act_gx = None
+    if layer.mode == "act":  # the input quantizer's scale, calibrated once: MAX over the ranks' shards
+        act_gx = torch.empty(1, dtype=torch.float32, device=dev)
+        L.lhcal_global_scale(x.view(1, t1 - t0, C), act_gx)
+        torch.distributed.all_reduce(act_gx, op=torch.distributed.ReduceOp.MAX)
+
+    def step():
+        S.calibrate_sharded(layer.mode, x, w, group_offsets=offs, token_ids=ids, act_gx=act_gx, buffers=buf,
+                            gather=False)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.distributed.barrier()
+    torch.cuda.synchronize()
+    L.lhcal_launch_count(reset=True)
+    clocks.start()
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    torch.distributed.barrier()
+    (ms_total,) = rank_max([start.elapsed_time(end)], dev)
+    ms = ms_total / args.steps
+    units, _, _ = algorithmic(layer)
+    return {"name": name, "workload": WORKLOAD_TEXT[name], "tokens": T, "cin": C, "rows": R, "groups": G,
+            "mode": layer.mode, "value": units / (ms / 1e3), "ms_per_step": ms, "units_per_step": units,
+            "gpu_launches": L.lhcal_launch_count(), "clocks": clk,
+            "shard": {"tokens": [t0, t1], "rows": [r0, r1]}}
+
+
+def run_sharded(args, rank, world, local_rank):
+    import torch
+
+    import scale_calibration_lh_b200 as L
+    from scale_calibration_lh_b200 import build as B
+
+    B.build()
+    L.load_library()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    rec = measure_sharded(headline_name(args), args, rank, world, dev)
+    if rank != 0:
+        return
+    out = {
+        "metric": METRIC, "value": rec["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": rec["ms_per_step"], "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": rec["workload"], "name": rec["name"], "tokens": rec["tokens"], "cin": rec["cin"],
+                   "rows": rec["rows"], "groups": rec["groups"], "mode": rec["mode"],
+                   "l2": "no flush: each rank's inputs exceed the 126 MB L2 at the full sizes",
+                   "parallelism": f"one layer over {world} GPUs: tokens and rows sharded, NCCL all-reduce of "
+                                  "the raw statistics and counts, MAX of the global scales"},
+        "e2e": {"value": None, "unit": UNIT, "note": "not measured in the sharded mode"},
+        "gpu_launches": rec["gpu_launches"], "clocks": rec["clocks"], "shard_of_rank0": rec["shard"],
+    }
+    print(json.dumps(out), flush=True)
+
+
 def run_lhcal(args, rank, world, local_rank):
     import torch
 
@@ -571,6 +660,9 @@ def main():
     ap.add_argument("--impl", choices=["lhcal", "reference"], default="lhcal")
     ap.add_argument("--workload", choices=["all"] + list(ORDER), default="all")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", action="store_true",
+                    help="one layer sharded over the ranks (tokens and rows; strong scaling) instead of one "
+                         "layer per rank; runs the headline workload or --workload")
     ap.add_argument("--rows", type=int, default=None,
                     help="weight rows per group instead of the workload's (smaller captures for profiling)")
     args = ap.parse_args()
@@ -582,16 +674,23 @@ def main():
     if args.impl == "reference":
         run_reference(args, rank, world)
         return
-    if world > 1:
+    if world > 1 or args.shard:
         import torch
 
         torch.cuda.set_device(local_rank)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                             device_id=torch.device("cuda", local_rank))
+        if world == 1:  # one rank: a local store, no rendezvous
+            torch.distributed.init_process_group("nccl", store=torch.distributed.HashStore(), rank=0, world_size=1,
+                                                 device_id=torch.device("cuda", local_rank))
+        else:
+            torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                                 device_id=torch.device("cuda", local_rank))
     try:
-        run_lhcal(args, rank, world, local_rank)
+        if args.shard:
+            run_sharded(args, rank, world, local_rank)
+        else:
+            run_lhcal(args, rank, world, local_rank)
     finally:
-        if world > 1:
+        if world > 1 or args.shard:
             import torch
 
             torch.distributed.destroy_process_group()

@@ -12,9 +12,14 @@
 //     U' = ((H + H^T) / 2) w - P w,   C' = w^T H w - 2 w^T P w   (P = 0 for FULL).
 // U' and C' are per-unit constants. v is exact in fp16, so the matrix part v^T H (all 16
 // outputs, for 16 units at once) is one m16n8k16 fp16 MMA per 8 outputs with H split into
-// fp16 hi + lo (H scaled by a power of two into fp16 range): relative error <= 2^-23 per H
-// entry, fp32 accumulation. The loss then differs from the fp32-rounded definition by at most
-// a few 2^-23 of |w|^T |H| |w|, far below the 1e-5 decision gaps that matter.
+// fp16 hi + lo, fp32 accumulation. H is first scaled by a power of two, H' = H 2^eH with the
+// largest |H'| in [2^14, 2^15). Then hi = fp16(H') and lo = fp16(H' - hi) represent an entry to
+// within 2^-22 of itself while lo is an fp16 normal number (|H'| >= about 2^-3, i.e. within
+// 2^17 of the largest entry); smaller entries keep an absolute accuracy of about 2^-25 in H'
+// units (lo reaches the fp16 subnormals), i.e. 2^-39 of the block's largest entry. Against
+// |v|^T |H| |v| both are far below the fp32 rounding of the 16-term products themselves, so
+// the loss differs from the fp32-rounded definition by a few 2^-23 of |w|^T |H| |w|, below the
+// 1e-5 decision gaps that matter. A test runs blocks whose H diagonal spans 2^20.
 //
 // Mapping (mma.sync.m16n8k16, row.col, f16 -> f32): a warp evaluates 16 units (the M rows) of
 // one input block for one candidate per step. Lane (g = lane / 4, t = lane % 4) owns units

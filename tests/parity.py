@@ -205,3 +205,40 @@ def sample_units(groups, rows, nblk, count, seed=0):
     u = np.stack([rng.integers(0, groups, count), rng.integers(0, rows, count), rng.integers(0, nblk, count)], 1)
     corners = np.array([[g, r, n] for g in {0, groups - 1} for r in {0, rows - 1} for n in {0, nblk - 1}])
     return np.concatenate([corners, u])
+
+
+def _sweep_rows_worker(args):
+    """One task of oracle_sweep_parallel (runs in a spawned process)."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import lhcal_oracle as O
+
+    mode, w_rows, h, p, g = args
+    with threadpool_limits(1):
+        return O.sweep(mode, w_rows, h, p, g)
+
+
+def oracle_sweep_parallel(mode: str, w, h, p, g, rows_per_task: int = 64, processes: int | None = None) -> dict:
+    """The oracle's sweep of every unit of a layer (row-major unit order, as all_units), computed
+    by a pool of spawned processes over row chunks; with the near-tie hook for check_sweep."""
+    import os
+    from concurrent.futures import ProcessPoolExecutor
+    from multiprocessing import get_context
+
+    w = np.asarray(w, dtype=np.float32)
+    G, R, C = w.shape
+    tasks = [(mode, w[:, r:r + rows_per_task], h, p, g) for r in range(0, R, rows_per_task)]
+    n = processes or max(1, (os.cpu_count() or 2) - 1)
+    with ProcessPoolExecutor(max_workers=n, mp_context=get_context("spawn")) as ex:
+        parts = list(ex.map(_sweep_rows_worker, tasks))
+    # Each part is [G, rows_chunk, N] in unit order; reassemble to [G, R, N].
+    out = {}
+    for k in parts[0]:
+        if k == "all_losses":
+            continue
+        arrs = [pt[k].reshape((G, -1, C // BLOCK) + pt[k].shape[1:]) for pt in parts]
+        out[k] = np.concatenate(arrs, axis=1).reshape((G * R * (C // BLOCK),) + parts[0][k].shape[1:])
+    return attach_candidates(out, mode, w, h, p, g)
+
+
+BLOCK = 16

@@ -379,6 +379,54 @@ def _run_and_check_wmse_full(layer, units):
     P.check_sweep(gc, gw, gl, ref, "wmse full")
 
 
+@pytest.mark.slow
+def test_dense_whole_layer_every_unit():
+    """All 1,048,576 units of the dense workload (X [16384, 4096], W [4096, 4096]) against the
+    oracle, not a sample: codes and Wq bit-exact outside near-ties, near-ties within the oracle's
+    tie set, every winning loss within 1e-4. The oracle runs in spawned worker processes."""
+    layer = P.make_layer("dense", 0)
+    d = synth.layer_to_device(layer)
+    b = L.calibrate("full", d["x"], d["w"])
+    _sync()
+    hs, _, counts = O.accumulate("full", layer.x_f32())
+    h, _ = O.finalize("full", hs, None, counts)
+    P.check_hessians(b.h.cpu().numpy(), h, "dense whole-layer H")
+    w32 = layer.w_f32()
+    g = np.array([O.global_scale(w32[0])], np.float32)
+    ref = P.oracle_sweep_parallel("full", w32, h, None, g)
+    rep = P.check_sweep(b.codes.cpu().numpy().reshape(-1), b.wq.cpu().numpy().reshape(-1, 16),
+                        b.loss.cpu().numpy().reshape(-1), ref, "dense whole layer")
+    assert rep["units"] == 4096 * 256
+    print("dense whole layer:", rep)
+
+
+def test_sweep_hessian_with_2e20_diagonal_dynamic_range():
+    """The tensor-core sweep scales H by a power of two into fp16 range and splits it into fp16
+    hi + lo: entries far below the largest keep an absolute accuracy (the lo part reaches fp16
+    subnormals), not a relative one. A block Hessian whose diagonal spans 2^0 .. 2^20, with
+    off-diagonal coupling, against the oracle in FULL and activation-aware modes."""
+    rng = np.random.default_rng(12)
+    G, R, C = 1, 256, 64
+    nblk = C // 16
+    w = (rng.normal(0, 0.05, (G, R, C)) * np.exp2(rng.uniform(-6, 0, (G, R, C)))).astype(np.float32)
+    scale = np.exp2(np.linspace(0, 20, 16))  # the diagonal's dynamic range: 2^20
+    h = np.zeros((G, nblk, 16, 16))
+    p = np.zeros((G, nblk, 16, 16))
+    for n in range(nblk):
+        a = rng.normal(size=(16, 16)) * np.sqrt(scale)[:, None] * 0.2
+        h[0, n] = np.diag(scale[rng.permutation(16)]) + a @ a.T / 16
+        p[0, n] = 0.01 * rng.normal(size=(16, 16)) * np.sqrt(np.outer(np.diag(h[0, n]), np.diag(h[0, n])))
+    h32, p32 = h.astype(np.float32), p.astype(np.float32)
+    g = np.array([O.global_scale(w[0])], np.float32)
+    for mode, pp in (("full", None), ("act", p32)):
+        codes, wq, loss = _sweep_gpu(L.MODE_IDS[mode], w, h32, pp, g)
+        units = P.all_units(G, R, nblk)
+        ref = P.oracle_sweep(mode, w, h32.astype(np.float64), None if pp is None else pp.astype(np.float64), g, units)
+        gc, gw, gl = P.gather_gpu_units(codes, wq, loss, units)
+        rep = P.check_sweep(gc, gw, gl, ref, f"2^20 dynamic range {mode}")
+        assert rep["units"] == R * nblk
+
+
 # ----------------------------------------------------------------------------- more edge cases
 
 def test_grouped_add_mode_over_two_batches():
@@ -760,6 +808,54 @@ def test_calibrate_host_matches_the_device_path(name, kw, chunks):
     assert out2.wq is None and torch.equal(out2.codes, want[0])
 
 
+@pytest.mark.slow
+def test_dense_whole_layer_every_unit():
+    """All 1,048,576 units of the dense workload (X [16384, 4096], W [4096, 4096]) against the
+    oracle, not a sample: codes and Wq bit-exact outside near-ties, near-ties within the oracle's
+    tie set, every winning loss within 1e-4. The oracle runs in spawned worker processes."""
+    layer = P.make_layer("dense", 0)
+    d = synth.layer_to_device(layer)
+    b = L.calibrate("full", d["x"], d["w"])
+    _sync()
+    hs, _, counts = O.accumulate("full", layer.x_f32())
+    h, _ = O.finalize("full", hs, None, counts)
+    P.check_hessians(b.h.cpu().numpy(), h, "dense whole-layer H")
+    w32 = layer.w_f32()
+    g = np.array([O.global_scale(w32[0])], np.float32)
+    ref = P.oracle_sweep_parallel("full", w32, h, None, g)
+    rep = P.check_sweep(b.codes.cpu().numpy().reshape(-1), b.wq.cpu().numpy().reshape(-1, 16),
+                        b.loss.cpu().numpy().reshape(-1), ref, "dense whole layer")
+    assert rep["units"] == 4096 * 256
+    print("dense whole layer:", rep)
+
+
+def test_sweep_hessian_with_2e20_diagonal_dynamic_range():
+    """The tensor-core sweep scales H by a power of two into fp16 range and splits it into fp16
+    hi + lo: entries far below the largest keep an absolute accuracy (the lo part reaches fp16
+    subnormals), not a relative one. A block Hessian whose diagonal spans 2^0 .. 2^20, with
+    off-diagonal coupling, against the oracle in FULL and activation-aware modes."""
+    rng = np.random.default_rng(12)
+    G, R, C = 1, 256, 64
+    nblk = C // 16
+    w = (rng.normal(0, 0.05, (G, R, C)) * np.exp2(rng.uniform(-6, 0, (G, R, C)))).astype(np.float32)
+    scale = np.exp2(np.linspace(0, 20, 16))  # the diagonal's dynamic range: 2^20
+    h = np.zeros((G, nblk, 16, 16))
+    p = np.zeros((G, nblk, 16, 16))
+    for n in range(nblk):
+        a = rng.normal(size=(16, 16)) * np.sqrt(scale)[:, None] * 0.2
+        h[0, n] = np.diag(scale[rng.permutation(16)]) + a @ a.T / 16
+        p[0, n] = 0.01 * rng.normal(size=(16, 16)) * np.sqrt(np.outer(np.diag(h[0, n]), np.diag(h[0, n])))
+    h32, p32 = h.astype(np.float32), p.astype(np.float32)
+    g = np.array([O.global_scale(w[0])], np.float32)
+    for mode, pp in (("full", None), ("act", p32)):
+        codes, wq, loss = _sweep_gpu(L.MODE_IDS[mode], w, h32, pp, g)
+        units = P.all_units(G, R, nblk)
+        ref = P.oracle_sweep(mode, w, h32.astype(np.float64), None if pp is None else pp.astype(np.float64), g, units)
+        gc, gw, gl = P.gather_gpu_units(codes, wq, loss, units)
+        rep = P.check_sweep(gc, gw, gl, ref, f"2^20 dynamic range {mode}")
+        assert rep["units"] == R * nblk
+
+
 # ----------------------------------------------------------------------------- more edge cases (2)
 
 def test_fused_act_quant_grouped_with_empty_experts():
@@ -820,3 +916,37 @@ def test_golden_sweep_winners_on_the_gpu():
     assert codes.flatten().tolist() == [c for c, _ in want]
     assert loss.flatten().tolist() == [v for _, v in want]
     np.testing.assert_array_equal(wq.cpu().numpy().reshape(n, 16).view(np.int32), np.stack(ws).view(np.int32))
+
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("dense", dict(tokens=700, cin=256, rows=300)),
+    ("act", dict(tokens=500, cin=128, rows=130)),
+    ("moe", dict(tokens=300, cin=128, rows=40, groups=9, top_k=3)),
+])
+def test_sharded_path_on_one_nccl_rank_equals_calibrate(name, kw):
+    """scale_calibration_lh_b200.sharded (token-sharded statistics, all-reduce, row-sharded sweep,
+    all-gather) run by one NCCL rank through the C ABI: every collective is then an identity, so
+    the results equal calibrate()'s bit for bit. The partition and reductions over two ranks are
+    covered on the CPU (tests/test_sharded_cpu.py)."""
+    import torch.distributed as dist
+
+    from scale_calibration_lh_b200 import sharded as S
+
+    layer = P.make_layer(name, 23, **kw)
+    d = synth.layer_to_device(layer)
+    dist.init_process_group("nccl", store=dist.HashStore(), rank=0, world_size=1,
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        b, res = S.calibrate_sharded(layer.mode, d["x"], d["w"], group_offsets=d["offs"], token_ids=d["ids"],
+                                     act_gx=None)
+        ref = L.calibrate(layer.mode, d["x"], d["w"], group_offsets=d["offs"], token_ids=d["ids"],
+                          act_gx=d["act_gx"] if name == "act" else None)
+        _sync()
+    finally:
+        dist.destroy_process_group()
+    for k in ("h", "p", "counts", "g"):
+        if getattr(ref, k) is not None:
+            assert torch.equal(getattr(b, k), getattr(ref, k)), k
+    assert torch.equal(res["codes"], ref.codes) and torch.equal(res["loss"], ref.loss)
+    assert torch.equal(res["wq"].view(torch.int32), ref.wq.view(torch.int32))
