@@ -18,12 +18,16 @@
 //    {threshold, value} table that a level drop lowers by one entry; the candidate row is an
 //    immediate offset in a loop unrolled by three.
 //  * While all 16 weights of a unit sit at the top grid level (6), its loss is the parabola
-//    36 s^2 sum Imp - 12 s sum Imp |w| + sum Imp w^2. The CTA orders its rows by smallest |w|
-//    so that each warp's units leave that regime together; below the warp's first candidate
-//    with an unclamped element the parabola gives the loss.
+//    36 s^2 sum Imp - 12 s sum Imp |w| + sum Imp w^2. The CTA stages its rows' weights in
+//    shared memory and orders the rows by their first unclamped candidate (a stable counting
+//    sort, row_order.cuh), so that each warp's units leave that regime together; below the
+//    warp's first candidate with an unclamped element the parabola gives the loss.
 //  * Loss: packed f32x2 products, L = sum_i Imp_i (|wq_i| - |w_i|)^2.
+#include <cstddef>
+
 #include "common.cuh"
 #include "quant_tables.cuh"
+#include "row_order.cuh"
 
 namespace lhcal {
 namespace {
@@ -31,12 +35,20 @@ namespace {
 constexpr int kThreads = 128;
 constexpr int kRowBytes = 8 * kLev;  // {thr, val} float2 entries per candidate
 
-struct DiagShared {
+constexpr int kWStride = kBlock + 4;  // floats per staged weight row (16-byte aligned rows)
+
+struct __align__(16) DiagShared {
   float2 tab[kCand * kLev];  // .x threshold, .y fake-quant value, per (candidate, level)
+  alignas(16) float wall[kThreads][kWStride];  // the CTA's rows' weights (fp32)
   float imp[kBlock];
-  float key[kThreads];
-  int perm[kThreads];
+  int kfirst[kThreads];  // per row: first candidate with an element below the top level
+  int perm[kThreads];    // rows in ascending kfirst (row_order.cuh)
+  int kf_sorted[kThreads];
+  int hist[4][kOrderRows];
+  int base[kOrderRows];
 };
+static_assert(kThreads == kOrderRows, "one row per thread");
+static_assert(offsetof(DiagShared, wall) % 16 == 0, "16-byte shared-memory accesses need aligned rows");
 
 // Level of magnitude a at candidate row tab_k, by counting thresholds.
 __device__ __forceinline__ int level_direct(const float2* tab_k, float a) {
@@ -77,27 +89,38 @@ sweep_diag_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const flo
     sh.tab[idx] = make_float2(level_threshold(j, s), __fmul_rn(e2m1_grid(j), s));
   }
   if (threadIdx.x < kBlock) sh.imp[threadIdx.x] = imp ? __ldg(imp + (e * nblk + n) * kBlock + threadIdx.x) : 1.f;
+  for (int i = threadIdx.x; i < 4 * kOrderRows; i += kThreads) (&sh.hist[0][0])[i] = 0;
+  __syncthreads();
+  // Each row: its weights staged in shared memory, and kfirst, the first candidate at which one
+  // of its weights falls below the top E2M1 level; rows past the end get kCand and sort last.
   {
     const int64_t row = rbase + threadIdx.x;
     float m = __int_as_float(0x7f800000);
+    float wt[kBlock];
     if (row < rows) {
-      float wt[kBlock];
       load_w16<WT>(w + (e * rows + row) * cin + n * kBlock, wt);
+    } else {
 #pragma unroll
-      for (int i = 0; i < kBlock; ++i) m = fminf(m, fabsf(wt[i]));
+      for (int i = 0; i < kBlock; ++i) wt[i] = 0.f;
     }
-    sh.key[threadIdx.x] = m;
+#pragma unroll
+    for (int i = 0; i < kBlock; i += 4) {
+      *reinterpret_cast<float4*>(&sh.wall[threadIdx.x][i]) = make_float4(wt[i], wt[i + 1], wt[i + 2], wt[i + 3]);
+      m = fminf(fminf(fabsf(wt[i]), fabsf(wt[i + 1])), fminf(fminf(fabsf(wt[i + 2]), fabsf(wt[i + 3])), m));
+    }
+    int lo = 0, hi = kCand;  // first k with m < thr[k][7]
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (m < sh.tab[kLev * mid + 7].x) hi = mid; else lo = mid + 1;
+    }
+    const int kf = row < rows ? lo : kCand;
+    sh.kfirst[threadIdx.x] = kf;
+    row_order_count(kf, sh.hist);
   }
   __syncthreads();
-  {
-    const float my = sh.key[threadIdx.x];
-    int rank = 0;
-    for (int j = 0; j < kThreads; ++j) {
-      const float kj = sh.key[j];
-      rank += (kj < my || (kj == my && j < static_cast<int>(threadIdx.x))) ? 1 : 0;
-    }
-    sh.perm[rank] = threadIdx.x;
-  }
+  if (threadIdx.x < 32) row_order_scan(sh.hist, sh.base);
+  __syncthreads();
+  row_order_place(sh.kfirst[threadIdx.x], sh.hist, sh.base, sh.perm, sh.kf_sorted);
   __syncthreads();
 
   const int64_t r = rbase + sh.perm[threadIdx.x];
@@ -106,16 +129,18 @@ sweep_diag_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const flo
   const int64_t woff = (e * rows + (valid ? r : 0)) * cin + n * kBlock;
 
   float wv[kBlock];
-  if (valid) {
-    load_w16<WT>(w + woff, wv);
-  } else {
+  {
+    const float* wr = sh.wall[sh.perm[threadIdx.x]];
 #pragma unroll
-    for (int i = 0; i < kBlock; ++i) wv[i] = 0.f;
+    for (int i = 0; i < kBlock; i += 4) {
+      const float4 q = *reinterpret_cast<const float4*>(wr + i);
+      wv[i] = q.x; wv[i + 1] = q.y; wv[i + 2] = q.z; wv[i + 3] = q.w;
+    }
   }
   float2 na2[kBlock / 2];  // -|w|, pairs
   float2 wp[kBlock / 2];   // Imp, pairs
   uint32_t neg = 0;        // bit i: w_i has its sign bit set
-  float pa = 0.f, pb = 0.f, pc = 0.f, amin = __int_as_float(0x7f800000);
+  float pa = 0.f, pb = 0.f, pc = 0.f;
 #pragma unroll
   for (int i = 0; i < kBlock; ++i) {
     const float ai = fabsf(wv[i]), im = sh.imp[i];
@@ -123,7 +148,6 @@ sweep_diag_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const flo
     pa += im;
     pb = fmaf(im, ai, pb);
     pc = fmaf(im * ai, ai, pc);
-    amin = fminf(amin, ai);
   }
 #pragma unroll
   for (int q = 0; q < kBlock / 2; ++q) {
@@ -150,19 +174,9 @@ sweep_diag_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const flo
     }
   };
 
-  // Clamped prefix: first candidate at which some element of the unit leaves level 7.
-  int kfirst = kCand;
-  if (valid) {
-    int lo = 0, hi = kCand;
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if (amin < sh.tab[kLev * mid + 7].x) hi = mid; else lo = mid + 1;
-    }
-    kfirst = lo;
-  }
-  int kstart = kfirst;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) kstart = min(kstart, __shfl_xor_sync(0xffffffffu, kstart, o));
+  // Clamped prefix: the warp's first full candidate is the smallest kfirst of its 32 rows, the
+  // first of its sorted range.
+  const int kstart = sh.kf_sorted[threadIdx.x & ~31];
 #pragma unroll 1
   for (int k = 0; k < kstart; ++k) {
     const float sk = sh.tab[kLev * k + 2].y;  // grid value 1 times s_k

@@ -50,6 +50,7 @@
 
 #include "common.cuh"
 #include "quant_tables.cuh"
+#include "row_order.cuh"
 
 namespace lhcal {
 namespace {
@@ -85,11 +86,11 @@ struct __align__(16) TcShared {
   float rho[kCand];  // -2 / (s_k * 2^eH): scale of U' in the MMA accumulator
   float s2[kCand];   // s_k^2 * 2^eH
   float hscale;  // 2^-eH: H' = H * hscale lies below 2^15
-  int kfirst[kUnitsPerCta];  // per row: first candidate with an element below the top level
-  int perm[kUnitsPerCta];    // the CTA's rows in ascending kfirst (stable)
+  int kfirst[kUnitsPerCta];     // per row: first candidate with an element below the top level
+  int perm[kUnitsPerCta];       // the CTA's rows in ascending kfirst (row_order.cuh)
   int kf_sorted[kUnitsPerCta];
-  int hist[4][kUnitsPerCta];  // per warp of rows, per kfirst value: rows of that warp
-  int base[kUnitsPerCta];     // rows with a smaller kfirst
+  int hist[4][kOrderRows];
+  int base[kOrderRows];
 };
 static_assert(offsetof(TcShared, tab) % 16 == 0 && offsetof(TcShared, h) % 16 == 0 &&
                   offsetof(TcShared, p) % 16 == 0 && offsetof(TcShared, hs) % 16 == 0 &&
@@ -188,7 +189,7 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
     sh.tab[idx] = make_float4(level_threshold(j, s), __uint_as_float(q16), __uint_as_float(q16 << 16),
                               __fmul_rn(e2m1_grid(j), s));
   }
-  for (int i = threadIdx.x; i < 4 * kUnitsPerCta; i += kTcThreads) (&sh.hist[0][0])[i] = 0;
+  for (int i = threadIdx.x; i < 4 * kOrderRows; i += kTcThreads) (&sh.hist[0][0])[i] = 0;
   const int64_t rbase = static_cast<int64_t>(blockIdx.y) * kUnitsPerCta;
   __syncthreads();
   // Each of the CTA's rows: weights staged in shared memory, and kfirst, the first candidate at
@@ -212,9 +213,7 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
     }
     const int kf = ok ? lo : kCand;
     sh.kfirst[threadIdx.x] = kf;
-    // Stable counting sort by kfirst, step 1: rows of this warp per kfirst value.
-    const uint32_t same = __match_any_sync(0xffffffffu, kf);
-    if (lane == __ffs(same) - 1) sh.hist[warp][kf] = __popc(same);
+    row_order_count(kf, sh.hist);
   } else if (warp == 4) {
     // Scale H so that its largest |H'| lies in [2^14, 2^15): below the fp16 maximum.
     uint32_t m = 0;
@@ -228,26 +227,7 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
   }
   __syncthreads();
   if (warp == 0) {
-    // Step 2: base[v] = rows with kfirst < v (an exclusive scan over the 127 values).
-    int c[4], run = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int v = 4 * lane + j;
-      c[j] = sh.hist[0][v] + sh.hist[1][v] + sh.hist[2][v] + sh.hist[3][v];
-      run += c[j];
-    }
-    int incl = run;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
-    }
-    int b = incl - run;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      sh.base[4 * lane + j] = b;
-      b += c[j];
-    }
+    row_order_scan(sh.hist, sh.base);
   } else if (warp == 1) {
     const float hscale = sh.hscale;
     const float inv_hscale = 1.0f / hscale;  // exact: a power of two
@@ -258,16 +238,8 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
     }
   }
   __syncthreads();
-  if (threadIdx.x < kUnitsPerCta) {
-    // Step 3: position = rows with a smaller kfirst + rows of earlier warps with the same one
-    // + lanes of this warp before this one with the same one (ties keep the row order).
-    const int kf = sh.kfirst[threadIdx.x];
-    const uint32_t same = __match_any_sync(0xffffffffu, kf);
-    int pos = sh.base[kf] + __popc(same & ((1u << lane) - 1u));
-    for (int w2 = 0; w2 < warp; ++w2) pos += sh.hist[w2][kf];
-    sh.perm[pos] = threadIdx.x;
-    sh.kf_sorted[pos] = kf;
-  }
+  if (threadIdx.x < kUnitsPerCta)
+    row_order_place(sh.kfirst[threadIdx.x], sh.hist, sh.base, sh.perm, sh.kf_sorted);
   __syncthreads();
   const float hscale = sh.hscale;
 
