@@ -444,11 +444,13 @@ def measure_workload(name, args, rank, world, dev, flusher):
         h.copy_(t)
         return h
 
-    hx, hxq, hw = pinned(d["x"]), pinned(d["xq"]), pinned(d["w"])
-    hoffs, hids = pinned(d["offs"]), pinned(d["ids"])
-    K2 = max(3, min(K, 10))
+    hx = hxq = hw = hoffs = hids = None
     e2e = {}
-    for label, want_wq16 in (("e2e", True), ("e2e_scales_only", False)):
+    if not args.no_e2e:
+        hx, hxq, hw = pinned(d["x"]), pinned(d["xq"]), pinned(d["w"])
+        hoffs, hids = pinned(d["offs"]), pinned(d["ids"])
+    K2 = max(3, min(K, 10))
+    for label, want_wq16 in (() if args.no_e2e else (("e2e", True), ("e2e_scales_only", False))):
         # The whole output: codes, global scales and losses, plus the bf16 fake-quantized weights
         # (lhcal_apply_scales of the chosen codes) unless the weights stay on the device.
         b2 = L.Buffers(mode, T, C, R, G, xdt, dev, want_wq=False, want_wq16=want_wq16)
@@ -644,7 +646,8 @@ def run_lhcal(args, rank, world, local_rank):
                    "parallelism": f"{world} independent layers, one per GPU (no collective)",
                    "workloads_run": list(names)},
         "roofline": head["roofline"], "roofline_accum": head["roofline_accum"], "stages_ms": head["stages_ms"],
-        "e2e": head["e2e"], "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
+        "e2e": head.get("e2e", {"value": None, "unit": UNIT, "note": "not measured (--no-e2e)"}),
+        "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
     }
     if "cpu_baseline" in head:
         out["cpu_baseline"] = head["cpu_baseline"]
@@ -660,6 +663,7 @@ def main():
     ap.add_argument("--impl", choices=["lhcal", "reference"], default="lhcal")
     ap.add_argument("--workload", choices=["all"] + list(ORDER), default="all")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
     ap.add_argument("--shard", action="store_true",
                     help="one layer sharded over the ranks (tokens and rows; strong scaling) instead of one "
                          "layer per rank; runs the headline workload or --workload")

@@ -520,12 +520,25 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
       const int c = col_of(ci);
       float hd = 0.f;
 #pragma unroll
-      for (int k = 0; k < 16; ++k) hd = fmaf(sh.h[c * 16 + k], dfull[k], hd);
+      for (int k = 0; k < 16; k += 4) {  // row c of H, four entries at a time
+        const float4 hq = *reinterpret_cast<const float4*>(sh.h + c * 16 + k);
+        hd = fmaf(hq.x, dfull[k], hd);
+        hd = fmaf(hq.y, dfull[k + 1], hd);
+        hd = fmaf(hq.z, dfull[k + 2], hd);
+        hd = fmaf(hq.w, dfull[k + 3], hd);
+      }
       if (ACT) {  // + 2 (P w)_c, with w from the CTA's shared copy
         const float* wr = sh.wall[sh.perm[warp * kUnitsPerWarp + gq + 8 * u]];
         float pw = 0.f;
 #pragma unroll
-        for (int k = 0; k < 16; ++k) pw = fmaf(sh.p[c * 16 + k], wr[k], pw);
+        for (int k = 0; k < 16; k += 4) {
+          const float4 pq = *reinterpret_cast<const float4*>(sh.p + c * 16 + k);
+          const float4 wq4v = *reinterpret_cast<const float4*>(wr + k);
+          pw = fmaf(pq.x, wq4v.x, pw);
+          pw = fmaf(pq.y, wq4v.y, pw);
+          pw = fmaf(pq.z, wq4v.z, pw);
+          pw = fmaf(pq.w, wq4v.w, pw);
+        }
         hd = fmaf(2.f, pw, hd);
       }
       part = fmaf(dw[ci], hd, part);
