@@ -70,9 +70,20 @@ WORKLOAD_TEXT = {
            "grouped full H, per-expert global scale",
 }
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu capture of the named
-# kernel on the workload, as committed with its summary; reported as traffic_from_profile,
-# never as a measurement of the run (the bench cannot read DRAM counters).
-PROFILED_TRAFFIC = {}
+# kernel on the workload (the kernels as they are now), as committed with its summary; reported
+# as traffic_from_profile, never as a measurement of the run (the bench cannot read DRAM
+# counters). The fused-MoE sweep was captured with 128 rows per expert and is scaled to the
+# 1280 rows of the workload (its traffic, W in and Wq out, grows with the rows).
+PROFILED_TRAFFIC = {
+    ("dense", "sweep_tc_kernel"): {"bytes": 33_872_128 + 23_449_856},
+    ("act", "sweep_tc_kernel"): {"bytes": 101_289_216 + 171_041_792},
+    ("moe", "sweep_tc_kernel"): {"bytes": 10 * (420_447_488 + 678_123_264), "scaled": "x10 from 128 rows per expert"},
+    ("wmse", "sweep_diag_kernel"): {"bytes": 100_809_000 + 163_823_616},
+    ("dense", "accum"): {"bytes": 134_267_136 + 4_176_896},
+    ("act", "accum"): {"bytes": 268_592_384 + 4_254_208},
+    ("moe", "accum"): {"bytes": 86_018_816 + 52_112_896},
+    ("wmse", "accum"): {"bytes": 1_610_622_000 + 7_723_264, "note": "accum_diag_kernel only"},
+}
 
 
 def load_peaks():
