@@ -448,20 +448,29 @@ def _scales_and_sweep(m, w, buffers, e0: int, e1: int):
         lhcal_apply_scales(w[sl], b.g[sl], b.codes[sl], wq16=b.wq16[sl])
 
 
+PIPELINE_CHUNK_BYTES = 64 << 20  # weights per chunk of calibrate_host's pipeline
+SWEEP_TILE_ROWS = 128  # rows of one sweep CTA: row chunks start on multiples of it
+
+
 def calibrate_host(mode, x, w, buffers: Buffers, staging: dict, hxq=None, group_offsets=None, token_ids=None,
-                   out: HostOutputs | None = None, act_gx=None, group_chunks: int = 8) -> HostOutputs:
+                   out: HostOutputs | None = None, act_gx=None, group_chunks: int | None = None,
+                   row_chunks: int = 8) -> HostOutputs:
     """The whole hot path from host tensors (pinned, for asynchronous copies) to host results.
 
     ``staging`` holds device tensors shaped like the inputs under keys "x", "w" and, when
-    used, "xq", "offs", "ids". Activations (and routing) are copied in and the statistics
-    computed on the current stream. A grouped layer (groups > 1) is then pipelined over
-    ``group_chunks`` chunks of groups: each chunk's weights are copied in on a side stream while
-    the current stream computes global scales and sweeps the chunks already resident, and each
-    chunk's results are copied out on another side stream as soon as they are ready. A layer
-    with one group copies its weights, computes the scale and sweeps. The results land in
-    ``out`` (codes, global scales, loss, and the fake-quantized weights it was made for: fp32
-    wq, or bf16 wq16 when the buffers hold it); the function returns without synchronising,
-    and the current stream waits for every copy it issued.
+    used, "xq", "offs", "ids". The weights are copied in on a side stream from the start, in
+    chunks, while the current stream copies the activations (and routing) in and computes the
+    statistics; the weight copies wait only for what was enqueued before this call (an earlier
+    call's sweeps may still read the staged weights). Then, chunk by chunk, the current stream
+    computes global scales and sweeps what is resident, and each chunk's results are copied out
+    on another side stream as soon as they are ready. A grouped layer (groups > 1) is chunked by
+    groups: ``group_chunks`` chunks, by default enough for about 64 MB of weights each (at least
+    8). A layer with one group needs all of its weights for its scale: it is copied in whole and
+    its sweep is split into ``row_chunks`` chunks of rows, starting on multiples of the sweep's
+    128-row tile, so every unit is computed exactly as in one sweep. The results land in ``out``
+    (codes, global scales, loss, and the fake-quantized weights it was made for: fp32 wq, or
+    bf16 wq16 when the buffers hold it); the function returns without synchronising, and the
+    current stream waits for every copy it issued.
     """
     import torch
 
@@ -469,6 +478,26 @@ def calibrate_host(mode, x, w, buffers: Buffers, staging: dict, hxq=None, group_
     if out is None:
         out = HostOutputs(buffers)
     cur = torch.cuda.current_stream()
+    dev = staging["w"].device
+    s_in, s_out = _side_stream(dev, "in"), _side_stream(dev, "out")
+    start = torch.cuda.Event()
+    start.record(cur)
+    s_in.wait_event(start)
+    s_out.wait_event(start)
+    groups, rows = int(w.shape[0]), int(w.shape[1])
+    if groups > 1:
+        n = group_chunks or max(8, -(-w.numel() * w.element_size() // PIPELINE_CHUNK_BYTES))
+        n = max(1, min(n, groups))
+        bounds = [groups * j // n for j in range(n + 1)]
+    else:
+        bounds = [0, 1]
+    ready = []
+    with torch.cuda.stream(s_in):  # every weight chunk, in order, from the start
+        for e0, e1 in zip(bounds[:-1], bounds[1:]):
+            staging["w"][e0:e1].copy_(w[e0:e1], non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(s_in)
+            ready.append(ev)
     if m != MSE:
         staging["x"].copy_(x, non_blocking=True)
         if hxq is not None:
@@ -480,32 +509,38 @@ def calibrate_host(mode, x, w, buffers: Buffers, staging: dict, hxq=None, group_
         _statistics(m, staging["x"], buffers, xq=staging["xq"] if hxq is not None else None,
                     group_offsets=staging.get("offs") if group_offsets is not None else None,
                     token_ids=staging.get("ids") if token_ids is not None else None, act_gx=act_gx)
-    groups = int(w.shape[0])
-    n = max(1, min(group_chunks, groups))
-    bounds = [groups * j // n for j in range(n + 1)]
-    dev = staging["w"].device
-    s_in, s_out = _side_stream(dev, "in"), _side_stream(dev, "out")
-    s_in.wait_stream(cur)
-    s_out.wait_stream(cur)
-    for e0, e1 in zip(bounds[:-1], bounds[1:]):
-        with torch.cuda.stream(s_in):
-            staging["w"][e0:e1].copy_(w[e0:e1], non_blocking=True)
-            ready = torch.cuda.Event()
-            ready.record(s_in)
-        cur.wait_event(ready)
-        _scales_and_sweep(m, staging["w"], buffers, e0, e1)
+
+    def copy_out(e0, e1, r0, r1, with_g):
         done = torch.cuda.Event()
         done.record(cur)
         with torch.cuda.stream(s_out):
             s_out.wait_event(done)
-            out.codes[e0:e1].copy_(buffers.codes[e0:e1], non_blocking=True)
-            out.g[e0:e1].copy_(buffers.g[e0:e1], non_blocking=True)
-            if out.wq16 is not None:
-                out.wq16[e0:e1].copy_(buffers.wq16[e0:e1], non_blocking=True)
-            if out.loss is not None:
-                out.loss[e0:e1].copy_(buffers.loss[e0:e1], non_blocking=True)
-            if out.wq is not None:
-                out.wq[e0:e1].copy_(buffers.wq[e0:e1], non_blocking=True)
+            for name in ("codes", "wq16", "loss", "wq"):
+                dst = getattr(out, name)
+                if dst is not None:
+                    dst[e0:e1, r0:r1].copy_(getattr(buffers, name)[e0:e1, r0:r1], non_blocking=True)
+            if with_g:
+                out.g[e0:e1].copy_(buffers.g[e0:e1], non_blocking=True)
+
+    if groups > 1:
+        for (e0, e1), ev in zip(zip(bounds[:-1], bounds[1:]), ready):
+            cur.wait_event(ev)
+            _scales_and_sweep(m, staging["w"], buffers, e0, e1)
+            copy_out(e0, e1, 0, rows, True)
+    else:
+        cur.wait_event(ready[0])
+        b = buffers
+        lhcal_global_scale(staging["w"], b.g)
+        tiles = -(-rows // SWEEP_TILE_ROWS)
+        k = max(1, min(row_chunks, tiles))
+        rb = [min(rows, SWEEP_TILE_ROWS * (tiles * j // k)) for j in range(k + 1)]
+        for j, (r0, r1) in enumerate(zip(rb[:-1], rb[1:])):
+            wr = staging["w"][:, r0:r1]
+            lhcal_scale_sweep(m, wr, b.h, b.g, b.codes[:, r0:r1], wq=None if b.wq is None else b.wq[:, r0:r1],
+                              loss=None if b.loss is None else b.loss[:, r0:r1], p=b.p)
+            if getattr(b, "wq16", None) is not None:
+                lhcal_apply_scales(wr, b.g, b.codes[:, r0:r1], wq16=b.wq16[:, r0:r1])
+            copy_out(0, 1, r0, r1, j == 0)
     cur.wait_stream(s_in)
     cur.wait_stream(s_out)
     return out

@@ -8,7 +8,8 @@ size. The checks are:
 - the sizes, flags and pointers each call receives;
 - the binding's own buffer checks accept everything ``calibrate`` allocates;
 - ``calibrate_host`` stages the inputs, takes the statistics once and pipelines global scales,
-  sweeps and result copies over chunks of groups (streams and events faked, copies at once).
+  sweeps and result copies over chunks of groups, or, with one group, over chunks of rows that
+  start on multiples of the sweep's 128-row tile (streams and events faked, copies at once).
 """
 import ctypes
 
@@ -187,6 +188,54 @@ def test_calibrate_host_pipelines_groups_in_chunks(fake, fake_streams):
         assert _ptr(sw[9]) == b.codes[e0].data_ptr() and _ptr(sw[11]) == b.loss[e0].data_ptr()
     # Every group's results came back.
     assert torch.equal(out.codes, b.codes) and torch.equal(out.loss, b.loss) and torch.equal(out.g, b.g)
+
+
+def test_calibrate_host_default_group_chunks(fake, fake_streams):
+    G, R, C, T = 10, 4, 32, 40
+    x, w = torch.randn(T, C).bfloat16(), torch.randn(G, R, C).bfloat16()
+    offs = torch.tensor([0, 4, 8, 8, 12, 16, 20, 24, 28, 34, 40], dtype=torch.int32)
+    ids = torch.from_numpy(np.arange(T, dtype=np.int32))
+    b = L.Buffers("full", T, C, R, G, L.BF16, "cpu")
+    staging = {"x": torch.empty_like(x), "w": torch.empty_like(w), "offs": torch.empty_like(offs),
+               "ids": torch.empty_like(ids)}
+    fake.calls.clear()
+    L.calibrate_host("full", x, w, b, staging, group_offsets=offs, token_ids=ids, out=_host_outputs(b))
+    # A few KB of weights: the minimum of 8 chunks, groups * j // 8.
+    assert [a[2] for a in fake.args("lhcal_global_scale")] == [1, 1, 1, 2, 1, 1, 1, 2]  # bounds 0 1 2 3 5 6 7 8 10
+
+
+@pytest.mark.parametrize("rows,row_chunks,expect", [(300, 8, [0, 128, 256, 300]), (1000, 3, [0, 256, 640, 1000]),
+                                                    (100, 8, [0, 100]), (640, 1, [0, 640])])
+def test_calibrate_host_one_group_sweeps_in_row_chunks_on_tile_boundaries(fake, fake_streams, rows, row_chunks,
+                                                                           expect):
+    T, C = 24, 32
+    x, w = torch.randn(T, C).bfloat16(), torch.randn(1, rows, C).bfloat16()
+    b = L.Buffers("full", T, C, rows, 1, L.BF16, "cpu", want_wq16=True)
+    b.codes.copy_(torch.arange(b.codes.numel()).remainder(127).to(torch.uint8).view(b.codes.shape))
+    b.loss.copy_(torch.arange(b.loss.numel(), dtype=torch.float32).view(b.loss.shape))
+    b.wq16.copy_(torch.randn(b.wq16.shape).bfloat16())
+    staging = {"x": torch.empty_like(x), "w": torch.empty_like(w)}
+    out = _host_outputs(b)
+    out.wq16 = torch.zeros(b.wq16.shape, dtype=torch.bfloat16)
+    fake.calls.clear()
+    L.calibrate_host("full", x, w, b, staging, out=out, row_chunks=row_chunks)
+    # One global scale over the whole layer, before any sweep.
+    names = fake.names()
+    assert names.count("lhcal_global_scale") == 1 and names.index("lhcal_global_scale") < names.index(
+        "lhcal_scale_sweep")
+    (sc,) = fake.args("lhcal_global_scale")
+    assert _ptr(sc[1]) == staging["w"].data_ptr() and sc[3] == rows
+    sweeps, apply = fake.args("lhcal_scale_sweep"), fake.args("lhcal_apply_scales")
+    assert [a[4] for a in sweeps] == [r1 - r0 for r0, r1 in zip(expect, expect[1:])]
+    assert [a[3] for a in apply] == [a[4] for a in sweeps]
+    for r0, sw, ap in zip(expect, sweeps, apply):
+        assert r0 % 128 == 0  # every chunk starts on a sweep tile
+        assert _ptr(sw[2]) == staging["w"][0, r0].data_ptr() and _ptr(sw[6]) == b.h.data_ptr()
+        assert _ptr(sw[8]) == b.g.data_ptr() and _ptr(sw[9]) == b.codes[0, r0].data_ptr()
+        assert _ptr(sw[11]) == b.loss[0, r0].data_ptr()
+        assert _ptr(ap[1]) == staging["w"][0, r0].data_ptr() and _ptr(ap[8]) == b.wq16[0, r0].data_ptr()
+    assert torch.equal(out.codes, b.codes) and torch.equal(out.loss, b.loss) and torch.equal(out.g, b.g)
+    assert torch.equal(out.wq16, b.wq16)
 
 
 def test_calibrate_host_reads_xq_only_when_the_caller_copies_it_in(fake, fake_streams):
