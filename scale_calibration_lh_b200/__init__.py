@@ -458,12 +458,12 @@ def calibrate_host(mode, x, w, buffers: Buffers, staging: dict, hxq=None, group_
     """The whole hot path from host tensors (pinned, for asynchronous copies) to host results.
 
     ``staging`` holds device tensors shaped like the inputs under keys "x", "w" and, when
-    used, "xq", "offs", "ids". The weights are copied in on a side stream from the start, in
-    chunks, while the current stream copies the activations (and routing) in and computes the
-    statistics; the weight copies wait only for what was enqueued before this call (an earlier
-    call's sweeps may still read the staged weights). Then, chunk by chunk, the current stream
-    computes global scales and sweeps what is resident, and each chunk's results are copied out
-    on another side stream as soon as they are ready. A grouped layer (groups > 1) is chunked by
+    used, "xq", "offs", "ids". One side stream copies the activations (and routing) in, then the
+    weights in chunks, starting at once: it waits only for what was enqueued before this call (an
+    earlier call's kernels may still read the staging). The current stream computes the
+    statistics as soon as the activations are in, then, chunk by chunk, it computes global
+    scales and sweeps what is resident; each chunk's results are copied out on another side
+    stream as soon as they are ready. A grouped layer (groups > 1) is chunked by
     groups: ``group_chunks`` chunks, by default enough for about 64 MB of weights each (at least
     8). A layer with one group needs all of its weights for its scale: it is copied in whole and
     its sweep is split into ``row_chunks`` chunks of rows, starting on multiples of the sweep's
@@ -491,20 +491,27 @@ def calibrate_host(mode, x, w, buffers: Buffers, staging: dict, hxq=None, group_
         bounds = [groups * j // n for j in range(n + 1)]
     else:
         bounds = [0, 1]
+    # Host-to-device copies run in the order they are issued, whatever their stream: the
+    # activations (and routing) go first, so the statistics start as soon as they are in, and
+    # the weight chunks follow on the same stream without a gap.
     ready = []
-    with torch.cuda.stream(s_in):  # every weight chunk, in order, from the start
+    with torch.cuda.stream(s_in):
+        if m != MSE:
+            staging["x"].copy_(x, non_blocking=True)
+            if hxq is not None:
+                staging["xq"].copy_(hxq, non_blocking=True)
+            if group_offsets is not None:
+                staging["offs"].copy_(group_offsets, non_blocking=True)
+                staging["ids"].copy_(token_ids, non_blocking=True)
+            x_in = torch.cuda.Event()
+            x_in.record(s_in)
         for e0, e1 in zip(bounds[:-1], bounds[1:]):
             staging["w"][e0:e1].copy_(w[e0:e1], non_blocking=True)
             ev = torch.cuda.Event()
             ev.record(s_in)
             ready.append(ev)
     if m != MSE:
-        staging["x"].copy_(x, non_blocking=True)
-        if hxq is not None:
-            staging["xq"].copy_(hxq, non_blocking=True)
-        if group_offsets is not None:
-            staging["offs"].copy_(group_offsets, non_blocking=True)
-            staging["ids"].copy_(token_ids, non_blocking=True)
+        cur.wait_event(x_in)
         # X_q is read only when the caller copies it in; otherwise (act_gx) the kernel derives it.
         _statistics(m, staging["x"], buffers, xq=staging["xq"] if hxq is not None else None,
                     group_offsets=staging.get("offs") if group_offsets is not None else None,
