@@ -379,54 +379,6 @@ def _run_and_check_wmse_full(layer, units):
     P.check_sweep(gc, gw, gl, ref, "wmse full")
 
 
-@pytest.mark.slow
-def test_dense_whole_layer_every_unit():
-    """All 1,048,576 units of the dense workload (X [16384, 4096], W [4096, 4096]) against the
-    oracle, not a sample: codes and Wq bit-exact outside near-ties, near-ties within the oracle's
-    tie set, every winning loss within 1e-4. The oracle runs in spawned worker processes."""
-    layer = P.make_layer("dense", 0)
-    d = synth.layer_to_device(layer)
-    b = L.calibrate("full", d["x"], d["w"])
-    _sync()
-    hs, _, counts = O.accumulate("full", layer.x_f32())
-    h, _ = O.finalize("full", hs, None, counts)
-    P.check_hessians(b.h.cpu().numpy(), h, "dense whole-layer H")
-    w32 = layer.w_f32()
-    g = np.array([O.global_scale(w32[0])], np.float32)
-    ref = P.oracle_sweep_parallel("full", w32, h, None, g)
-    rep = P.check_sweep(b.codes.cpu().numpy().reshape(-1), b.wq.cpu().numpy().reshape(-1, 16),
-                        b.loss.cpu().numpy().reshape(-1), ref, "dense whole layer")
-    assert rep["units"] == 4096 * 256
-    print("dense whole layer:", rep)
-
-
-def test_sweep_hessian_with_2e20_diagonal_dynamic_range():
-    """The tensor-core sweep scales H by a power of two into fp16 range and splits it into fp16
-    hi + lo: entries far below the largest keep an absolute accuracy (the lo part reaches fp16
-    subnormals), not a relative one. A block Hessian whose diagonal spans 2^0 .. 2^20, with
-    off-diagonal coupling, against the oracle in FULL and activation-aware modes."""
-    rng = np.random.default_rng(12)
-    G, R, C = 1, 256, 64
-    nblk = C // 16
-    w = (rng.normal(0, 0.05, (G, R, C)) * np.exp2(rng.uniform(-6, 0, (G, R, C)))).astype(np.float32)
-    scale = np.exp2(np.linspace(0, 20, 16))  # the diagonal's dynamic range: 2^20
-    h = np.zeros((G, nblk, 16, 16))
-    p = np.zeros((G, nblk, 16, 16))
-    for n in range(nblk):
-        a = rng.normal(size=(16, 16)) * np.sqrt(scale)[:, None] * 0.2
-        h[0, n] = np.diag(scale[rng.permutation(16)]) + a @ a.T / 16
-        p[0, n] = 0.01 * rng.normal(size=(16, 16)) * np.sqrt(np.outer(np.diag(h[0, n]), np.diag(h[0, n])))
-    h32, p32 = h.astype(np.float32), p.astype(np.float32)
-    g = np.array([O.global_scale(w[0])], np.float32)
-    for mode, pp in (("full", None), ("act", p32)):
-        codes, wq, loss = _sweep_gpu(L.MODE_IDS[mode], w, h32, pp, g)
-        units = P.all_units(G, R, nblk)
-        ref = P.oracle_sweep(mode, w, h32.astype(np.float64), None if pp is None else pp.astype(np.float64), g, units)
-        gc, gw, gl = P.gather_gpu_units(codes, wq, loss, units)
-        rep = P.check_sweep(gc, gw, gl, ref, f"2^20 dynamic range {mode}")
-        assert rep["units"] == R * nblk
-
-
 # ----------------------------------------------------------------------------- more edge cases
 
 def test_grouped_add_mode_over_two_batches():
@@ -821,435 +773,6 @@ def test_calibrate_host_matches_the_device_path(name, kw, chunks):
     torch.cuda.current_stream().synchronize()
     assert out3.wq is None and torch.equal(out3.codes, want[0])
     assert torch.equal(out3.wq16.view(torch.int16), want[4].view(torch.int16))
-
-
-@pytest.mark.slow
-def test_dense_whole_layer_every_unit():
-    """All 1,048,576 units of the dense workload (X [16384, 4096], W [4096, 4096]) against the
-    oracle, not a sample: codes and Wq bit-exact outside near-ties, near-ties within the oracle's
-    tie set, every winning loss within 1e-4. The oracle runs in spawned worker processes."""
-    layer = P.make_layer("dense", 0)
-    d = synth.layer_to_device(layer)
-    b = L.calibrate("full", d["x"], d["w"])
-    _sync()
-    hs, _, counts = O.accumulate("full", layer.x_f32())
-    h, _ = O.finalize("full", hs, None, counts)
-    P.check_hessians(b.h.cpu().numpy(), h, "dense whole-layer H")
-    w32 = layer.w_f32()
-    g = np.array([O.global_scale(w32[0])], np.float32)
-    ref = P.oracle_sweep_parallel("full", w32, h, None, g)
-    rep = P.check_sweep(b.codes.cpu().numpy().reshape(-1), b.wq.cpu().numpy().reshape(-1, 16),
-                        b.loss.cpu().numpy().reshape(-1), ref, "dense whole layer")
-    assert rep["units"] == 4096 * 256
-    print("dense whole layer:", rep)
-
-
-def test_sweep_hessian_with_2e20_diagonal_dynamic_range():
-    """The tensor-core sweep scales H by a power of two into fp16 range and splits it into fp16
-    hi + lo: entries far below the largest keep an absolute accuracy (the lo part reaches fp16
-    subnormals), not a relative one. A block Hessian whose diagonal spans 2^0 .. 2^20, with
-    off-diagonal coupling, against the oracle in FULL and activation-aware modes."""
-    rng = np.random.default_rng(12)
-    G, R, C = 1, 256, 64
-    nblk = C // 16
-    w = (rng.normal(0, 0.05, (G, R, C)) * np.exp2(rng.uniform(-6, 0, (G, R, C)))).astype(np.float32)
-    scale = np.exp2(np.linspace(0, 20, 16))  # the diagonal's dynamic range: 2^20
-    h = np.zeros((G, nblk, 16, 16))
-    p = np.zeros((G, nblk, 16, 16))
-    for n in range(nblk):
-        a = rng.normal(size=(16, 16)) * np.sqrt(scale)[:, None] * 0.2
-        h[0, n] = np.diag(scale[rng.permutation(16)]) + a @ a.T / 16
-        p[0, n] = 0.01 * rng.normal(size=(16, 16)) * np.sqrt(np.outer(np.diag(h[0, n]), np.diag(h[0, n])))
-    h32, p32 = h.astype(np.float32), p.astype(np.float32)
-    g = np.array([O.global_scale(w[0])], np.float32)
-    for mode, pp in (("full", None), ("act", p32)):
-        codes, wq, loss = _sweep_gpu(L.MODE_IDS[mode], w, h32, pp, g)
-        units = P.all_units(G, R, nblk)
-        ref = P.oracle_sweep(mode, w, h32.astype(np.float64), None if pp is None else pp.astype(np.float64), g, units)
-        gc, gw, gl = P.gather_gpu_units(codes, wq, loss, units)
-        rep = P.check_sweep(gc, gw, gl, ref, f"2^20 dynamic range {mode}")
-        assert rep["units"] == R * nblk
-
-
-# ----------------------------------------------------------------------------- more edge cases
-
-def test_grouped_add_mode_over_two_batches():
-    """Two routed batches added into the same per-expert sums equal one pass over both."""
-    layer = P.make_layer("moe", 15, tokens=200, cin=96, rows=8, groups=16, top_k=3)
-    d = P.layer_to_device(layer)
-    x = d["x"]
-    off = layer.group_offsets
-    ids = layer.token_ids
-    # Batch 1: tokens < 100, batch 2: tokens >= 100 (ids renumbered into each batch's rows).
-    batches = []
-    for lo, hi in ((0, 100), (100, 200)):
-        o, t = [0], []
-        for e in range(16):
-            sel = [int(v) - lo for v in ids[off[e]:off[e + 1]] if lo <= v < hi]
-            t += sel
-            o.append(len(t))
-        batches.append((lo, hi, np.array(o, np.int32), np.array(t, np.int32)))
-    h = torch.full((16, 6, 16, 16), 9.0, dtype=torch.float32, device="cuda")
-    counts = torch.empty(16, dtype=torch.int64, device="cuda")
-    for j, (lo, hi, o, t) in enumerate(batches):
-        flags = L.ACCUM_OVERWRITE if j == 0 else L.ACCUM_ADD
-        do, dt = P.to_device(o, "i32"), P.to_device(t, "i32")
-        L.lhcal_accumulate("full", x[lo:hi], h, group_offsets=do, token_ids=dt, flags=flags)
-        L.lhcal_count_tokens(counts, group_offsets=do, flags=flags)
-    L.lhcal_finalize("full", counts, h)
-    _sync()
-    hs, _, c = _oracle_hessians(layer)
-    hf, _ = O.finalize("full", hs, None, c)
-    np.testing.assert_array_equal(counts.cpu().numpy(), c)
-    P.check_hessians(h.cpu().numpy(), hf, "two-batch grouped H")
-
-
-@pytest.mark.parametrize("mode", ["full", "act", "diag"])
-def test_sweep_optional_outputs_and_determinism(mode):
-    name = {"full": "dense", "act": "act", "diag": "wmse"}[mode]
-    layer = P.make_layer(name, 16, tokens=300, cin=128, rows=200)
-    d = P.layer_to_device(layer)
-    b = L.calibrate(mode, d["x"], d["w"], xq=d["xq"])
-    codes1 = b.codes.clone()
-    wq1 = b.wq.clone()
-    loss1 = b.loss.clone()
-    codes2 = torch.empty_like(codes1)
-    L.lhcal_scale_sweep(mode, d["w"], b.h, b.g, codes2, wq=None, loss=None, p=b.p)
-    codes3 = torch.empty_like(codes1)
-    wq3 = torch.empty_like(wq1)
-    loss3 = torch.empty_like(loss1)
-    L.lhcal_scale_sweep(mode, d["w"], b.h, b.g, codes3, wq=wq3, loss=loss3, p=b.p)
-    _sync()
-    assert torch.equal(codes1, codes2) and torch.equal(codes1, codes3)
-    assert torch.equal(wq1.view(torch.int32), wq3.view(torch.int32))
-    assert torch.equal(loss1.view(torch.int32), loss3.view(torch.int32))
-
-
-def test_diag_sweep_multiple_groups():
-    layer = P.make_layer("moe", 17, tokens=120, cin=64, rows=70, groups=6, top_k=2)
-    layer.mode = "diag"
-    _run_and_check(layer)
-
-
-def test_graph_replay_matches_eager_calls():
-    layer_a = P.make_layer("dense", 18, tokens=700, cin=512, rows=96)
-    layer_b = P.make_layer("dense", 19, tokens=700, cin=512, rows=96)
-    da, db = P.layer_to_device(layer_a), P.layer_to_device(layer_b)
-    x, w = da["x"].clone(), da["w"].clone()
-    graph = L.CalibrationGraph("full", x, w)
-    for d in (db, da):
-        x.copy_(d["x"])
-        w.copy_(d["w"])
-        out = graph.replay()
-        eager = L.calibrate("full", d["x"], d["w"])
-        _sync()
-        assert torch.equal(out.codes, eager.codes)
-        assert torch.equal(out.wq.view(torch.int32), eager.wq.view(torch.int32))
-        assert torch.equal(out.h.view(torch.int32), eager.h.view(torch.int32))
-
-
-@pytest.mark.parametrize("mode", ["act", "mse"])
-def test_graph_replay_fused_quantizer_and_mse(mode):
-    """The captured path with the input quantizer fused (X and gx in; the token splits reduce
-    through the workspace), and the statistics-free MSE sweep."""
-    layers = [P.make_layer("act" if mode == "act" else "dense", s, tokens=900, cin=256, rows=64) for s in (31, 32)]
-    devs = [P.layer_to_device(ly) for ly in layers]
-    x, w = devs[0]["x"].clone(), devs[0]["w"].clone()
-    gx = devs[0]["act_gx"].clone() if mode == "act" else None
-    graph = L.CalibrationGraph(mode, None if mode == "mse" else x, w, act_gx=gx)
-    for d in (devs[1], devs[0]):
-        x.copy_(d["x"])
-        w.copy_(d["w"])
-        if gx is not None:
-            gx.copy_(d["act_gx"])
-        out = graph.replay()
-        eager = L.calibrate(mode, None if mode == "mse" else d["x"], d["w"], act_gx=d["act_gx"] if gx is not None else None)
-        _sync()
-        assert torch.equal(out.codes, eager.codes)
-        assert torch.equal(out.loss.view(torch.int32), eager.loss.view(torch.int32))
-        if mode == "act":
-            assert torch.equal(out.p.view(torch.int32), eager.p.view(torch.int32))
-
-
-# ----------------------------------------------------------------------------- input quantizer
-
-def _act_x(tokens, cin, seed):
-    """bf16 activations drawn like the dense workload, plus blocks that stress the quantizer:
-    all-zero, negative-zero, tiny (small and subnormal scale codes) and huge outlier blocks."""
-    rng = np.random.default_rng(seed)
-    sig = np.exp(rng.normal(0, 1, cin))
-    sig[rng.choice(cin, max(1, cin // 100), replace=False)] *= 20
-    x = rng.normal(size=(tokens, cin)) * sig
-    if tokens >= 4 and cin >= 32:
-        x[0, :16] = 0.0
-        x[1, 16:32] = -0.0
-        x[2, :16] *= 1e-30
-        x[3, 16:32] *= 1e4
-    return synth.f32_to_bf16_bits(x.astype(np.float32))
-
-
-@pytest.mark.parametrize("tokens,cin,pad,gx_factor", [(1, 16, 0, 1.0), (37, 48, 8, 1.0), (300, 4096, 0, 1.0),
-                                                       (129, 256, 24, 1e-3), (129, 256, 0, 1e3),
-                                                       (64, 64, 0, 0.0), (0, 32, 0, 1.0)])
-def test_act_fake_quant_kernel_bit_exact(tokens, cin, pad, gx_factor):
-    xb = _act_x(tokens, cin, 40 + tokens)
-    x32 = synth.bf16_bits_to_f32(xb)
-    gx = np.float32(O.global_scale(x32) * gx_factor) if tokens else np.float32(1.0)
-    want = synth.f32_to_bf16_bits(O.act_fake_quant(x32, gx)) if tokens else np.zeros((0, cin), np.uint16)
-    ld = cin + pad
-    xfull = np.zeros((tokens, ld), np.uint16)
-    xfull[:, :cin] = xb
-    dx = P.to_device(xfull, "bf16")[:, :cin]
-    dq_full = torch.full((tokens, ld), 7.0, dtype=torch.bfloat16, device="cuda")
-    dq = dq_full[:, :cin]
-    L.lhcal_act_fake_quant(dx, torch.tensor([float(gx)], device="cuda"), dq)
-    _sync()
-    got = dq_full.cpu().view(torch.int16).numpy().view(np.uint16)
-    np.testing.assert_array_equal(got[:, :cin], want)
-    assert np.all(got[:, cin:] == np.uint16(0x40E0))  # the padding columns (7.0) are untouched
-
-
-@pytest.mark.parametrize("tokens,cin,rows", [(1000, 256, 40), (70, 48, 24), (2500, 4096, 16), (1, 16, 8)])
-def test_fused_act_quant_accumulation(tokens, cin, rows):
-    """X and gx in, no X_q: split (few slabs), cluster (4096 wide) and ragged cases."""
-    _run_and_check(P.make_layer("act", 31, tokens=tokens, cin=cin, rows=rows), fused=True)
-
-
-def test_fused_act_quant_grouped():
-    layer = synth.make_layer("moe", 32, tokens=300, cin=96, rows=24, groups=12, top_k=3)
-    layer.mode = "act"
-    P.act_inputs(layer)
-    _run_and_check(layer, fused=True)
-
-
-@pytest.mark.parametrize("tokens,cin,grouped,same_order", [(3000, 512, False, True), (2048, 4096, False, False),
-                                                            (400, 160, True, True)])
-def test_fused_equals_quantizer_then_unfused(tokens, cin, grouped, same_order):
-    """The fused kernel's sums equal the standalone quantizer's X_q fed to the two-tensor
-    accumulation: bit for bit where both split the tokens alike (the 512-wide layer, grouped
-    sums), else up to the fp32 summation order (the 4096-wide layer: clusters vs splits)."""
-    if grouped:
-        layer = synth.make_layer("moe", 33, tokens=tokens, cin=cin, rows=4, groups=10, top_k=3)
-        layer.mode = "act"
-        P.act_inputs(layer)
-    else:
-        layer = P.make_layer("act", 33, tokens=tokens, cin=cin, rows=4)
-    d = P.layer_to_device(layer)
-    G = layer.groups
-    shape = (G, cin // 16, 16, 16)
-    ws_bytes = max(L.lhcal_accumulate_workspace("act", L.BF16, tokens, cin, G),
-                   L.lhcal_accumulate_act_quant_workspace(L.BF16, tokens, cin, G))
-    ws = torch.empty(max(ws_bytes // 4, 1), dtype=torch.float32, device="cuda")
-    hf, pf = (torch.full(shape, 1.0, device="cuda") for _ in range(2))
-    L.lhcal_accumulate_act_quant(d["x"], hf, pf, d["act_gx"], group_offsets=d["offs"], token_ids=d["ids"],
-                                 flags=L.ACCUM_OVERWRITE, workspace=ws)
-    xq = torch.empty_like(d["x"])
-    L.lhcal_act_fake_quant(d["x"], d["act_gx"], xq)
-    hu, pu = (torch.full(shape, 2.0, device="cuda") for _ in range(2))
-    L.lhcal_accumulate("act", d["x"], hu, xq=xq, p=pu, group_offsets=d["offs"], token_ids=d["ids"],
-                       flags=L.ACCUM_OVERWRITE, workspace=ws)
-    _sync()
-    if same_order:
-        assert torch.equal(hf.view(torch.int32), hu.view(torch.int32))
-        assert torch.equal(pf.view(torch.int32), pu.view(torch.int32))
-    else:
-        P.check_hessians(hf.cpu().numpy(), hu.cpu().numpy().astype(np.float64), "fused vs unfused H", tol=1e-5)
-        P.check_hessians(pf.cpu().numpy(), pu.cpu().numpy().astype(np.float64), "fused vs unfused P", tol=1e-5)
-    # and the GPU quantizer's X_q is the oracle's
-    np.testing.assert_array_equal(xq.cpu().view(torch.int16).numpy().view(np.uint16), layer.xq)
-
-
-def test_fused_act_quant_rejects_fp32_and_missing_scale():
-    x = torch.zeros((8, 32), dtype=torch.float32, device="cuda")
-    h = torch.zeros((1, 2, 16, 16), device="cuda")
-    p = torch.zeros_like(h)
-    gx = torch.ones(1, device="cuda")
-    with pytest.raises(L.LhcalError) as e:
-        L.lhcal_accumulate_act_quant(x, h, p, gx, flags=L.ACCUM_OVERWRITE)
-    assert e.value.status == L.ERR_UNSUPPORTED
-    with pytest.raises(L.LhcalError) as e:
-        L.lhcal_accumulate_act_quant(x.bfloat16(), h, p, None, flags=L.ACCUM_OVERWRITE)
-    assert e.value.status == L.ERR_INVALID_ARG
-
-
-# ----------------------------------------------------------------------------- mse, 4/6 scale, outputs
-
-@pytest.mark.parametrize("name,kw", [("dense", dict(tokens=16, cin=272, rows=300)), ("tiny", dict()),
-                                     ("moe", dict(tokens=16, cin=64, rows=40, groups=5, top_k=2))])
-def test_mse_sweep(name, kw):
-    """Plain block MSE (H = I): no statistics, the diagonal kernel with unit weights."""
-    layer = synth.make_layer(name, 41, **kw)
-    d = P.layer_to_device(layer)
-    b = L.calibrate("mse", None, d["w"])
-    _sync()
-    assert b.h is None
-    w32 = layer.w_f32()
-    G, R, C = layer.groups, layer.rows, layer.cin
-    g = np.array([O.global_scale(w32[e]) for e in range(G)], np.float32)
-    np.testing.assert_array_equal(b.g.cpu().numpy().view(np.int32), g.view(np.int32))
-    units = P.all_units(G, R, C // 16)
-    ref = P.oracle_sweep("mse", w32, None, None, g, units)
-    gc, gw, gl = P.gather_gpu_units(b.codes, b.wq, b.loss, units)
-    P.check_sweep(gc, gw, gl, ref, f"{name} mse")
-
-
-def test_mse_sweep_full_size_weights():
-    layer = synth.make_layer("dense", 0, tokens=16)
-    d = P.layer_to_device(layer)
-    b = L.calibrate("mse", None, d["w"])
-    _sync()
-    w32 = layer.w_f32()
-    g = np.array([O.global_scale(w32[0])], np.float32)
-    units = P.sample_units(1, layer.rows, layer.cin // 16, 3000, seed=2)
-    ref = P.oracle_sweep("mse", w32, None, None, g, units)
-    gc, gw, gl = P.gather_gpu_units(b.codes, b.wq, b.loss, units)
-    P.check_sweep(gc, gw, gl, ref, "dense mse full size")
-
-
-@pytest.mark.parametrize("name", ["dense", "tiny", "moe"])
-def test_global_scale_fp8_max(name):
-    layer = synth.make_layer(name, 42, tokens=16, rows=64, cin=64, **({"groups": 7, "top_k": 2} if name == "moe" else {}))
-    d = P.layer_to_device(layer)
-    w32 = layer.w_f32()
-    for fp8_max in (448.0, 256.0):
-        g = torch.empty(layer.groups, dtype=torch.float32, device="cuda")
-        L.lhcal_global_scale(d["w"], g, fp8_max=fp8_max)
-        _sync()
-        want = np.array([O.global_scale(w32[e], fp8_max) for e in range(layer.groups)], np.float32)
-        np.testing.assert_array_equal(g.cpu().numpy().view(np.int32), want.view(np.int32))
-    g = torch.empty(layer.groups, dtype=torch.float32, device="cuda")
-    for bad in (0.0, 500.0, 1.0 / 3.0):
-        with pytest.raises(L.LhcalError) as e:
-            L.lhcal_global_scale(d["w"], g, fp8_max=bad)
-        assert e.value.status == L.ERR_INVALID_ARG
-
-
-@pytest.mark.parametrize("name,kw", [("dense", dict(tokens=400, cin=256, rows=96)), ("tiny", dict()),
-                                     ("moe", dict(tokens=80, cin=96, rows=24, groups=6, top_k=2))])
-def test_apply_scales_bit_exact(name, kw):
-    """Fake-quantized weights (fp32, bf16) and per-block amax for the sweep's codes and for
-    arbitrary codes (zero, every candidate, out of range), against the oracle."""
-    layer = synth.make_layer(name, 43, **kw)
-    d = P.layer_to_device(layer)
-    mode = layer.mode
-    b = L.calibrate(mode, d["x"], d["w"], group_offsets=d["offs"], token_ids=d["ids"])
-    G, R, C = layer.groups, layer.rows, layer.cin
-    rng = np.random.default_rng(7)
-    crafted = rng.integers(0, 256, (G, R, C // 16)).astype(np.uint8)
-    crafted.flat[:128] = np.arange(128, dtype=np.uint8)
-    w32 = layer.w_f32()
-    g_host = b.g.cpu().numpy()
-    for codes in (b.codes, P.to_device(crafted, "i32").to(torch.uint8)):
-        wq = torch.empty((G, R, C), dtype=torch.float32, device="cuda")
-        wq16 = torch.empty((G, R, C), dtype=torch.bfloat16, device="cuda")
-        amax = torch.empty((G, R, C // 16), dtype=torch.float32, device="cuda")
-        L.lhcal_apply_scales(d["w"], b.g, codes, wq=wq, wq16=wq16, amax=amax)
-        _sync()
-        rw, rw16, ra = O.apply_scales(w32, g_host, codes.cpu().numpy())
-        np.testing.assert_array_equal(wq.cpu().numpy().view(np.int32), rw.view(np.int32))
-        np.testing.assert_array_equal(wq16.float().cpu().numpy().view(np.int32), rw16.view(np.int32))
-        np.testing.assert_array_equal(amax.cpu().numpy().view(np.int32), ra.view(np.int32))
-    # The sweep's own fake-quantized weights are the apply_scales output for its codes.
-    wq = torch.empty((G, R, C), dtype=torch.float32, device="cuda")
-    L.lhcal_apply_scales(d["w"], b.g, b.codes, wq=wq)
-    _sync()
-    assert torch.equal(wq.view(torch.int32), b.wq.view(torch.int32))
-
-
-# ----------------------------------------------------------------------------- amax-multiplier search
-
-@pytest.mark.parametrize("mode,name,kw", [
-    ("full", "dense", dict(tokens=500, cin=96, rows=150)),
-    ("act", "act", dict(tokens=400, cin=64, rows=130)),
-    ("diag", "wmse", dict(tokens=300, cin=80, rows=140)),
-    ("mse", "dense", dict(tokens=16, cin=48, rows=200)),
-    ("full", "tiny", dict()),
-    ("full", "moe", dict(tokens=60, cin=64, rows=40, groups=5, top_k=2)),
-])
-def test_multiplier_search(mode, name, kw):
-    """Both sides get the oracle's finalized H (and P) rounded to fp32, the same global scales
-    and multipliers 0.5, 0.55, ..., 2.0 (plus 0 and one that reaches the 448 saturation)."""
-    layer = P.make_layer(name, 51, **kw)
-    G, R, C = layer.groups, layer.rows, layer.cin
-    w32 = layer.w_f32()
-    g = np.array([O.global_scale(w32[e]) for e in range(G)], np.float32)
-    h = p = None
-    if mode != "mse":
-        xq = layer.xq_f32() if mode == "act" else None
-        hs, ps, counts = O.accumulate(mode, layer.x_f32(), xq, layer.group_offsets, layer.token_ids)
-        h, p = O.finalize(mode, hs, ps, counts)
-        h = h.astype(np.float32).astype(np.float64)
-        p = None if p is None else p.astype(np.float32).astype(np.float64)
-    mult = np.concatenate([np.arange(0.5, 2.0001, 0.05), [0.0, 5000.0]]).astype(np.float32)
-    d = P.layer_to_device(layer)
-    codes = torch.empty((G, R, C // 16), dtype=torch.uint8, device="cuda")
-    wq = torch.empty((G, R, C), dtype=torch.float32, device="cuda")
-    loss = torch.empty((G, R, C // 16), dtype=torch.float32, device="cuda")
-    L.lhcal_multiplier_search(mode, d["w"], None if h is None else P.to_device(h, "f32"), P.to_device(g, "f32"),
-                              P.to_device(mult, "f32"), codes, wq=wq, loss=loss,
-                              p=None if p is None else P.to_device(p, "f32"))
-    _sync()
-    units = P.all_units(G, R, C // 16)
-    ref = P.oracle_multiplier_search(mode, w32, h, p, g, mult, units)
-    gc, gw, gl = P.gather_gpu_units(codes, wq, loss, units)
-    rep = P.check_sweep(gc, gw, gl, ref, f"{name} {mode} multiplier search")
-    assert rep["units"] == len(units)
-    # Optional outputs: codes alone give the same codes.
-    codes2 = torch.empty_like(codes)
-    L.lhcal_multiplier_search(mode, d["w"], None if h is None else P.to_device(h, "f32"), P.to_device(g, "f32"),
-                              P.to_device(mult, "f32"), codes2, p=None if p is None else P.to_device(p, "f32"))
-    _sync()
-    assert torch.equal(codes, codes2)
-
-
-def test_multiplier_search_rejects_bad_counts():
-    w = torch.zeros((1, 4, 32), dtype=torch.bfloat16, device="cuda")
-    g = torch.ones(1, device="cuda")
-    codes = torch.empty((1, 4, 2), dtype=torch.uint8, device="cuda")
-    for n in (0, 1025):
-        m = torch.ones(max(n, 1), device="cuda")
-        lib = L.load_library()
-        st = lib.lhcal_multiplier_search(3, 1, L._ptr(w), 1, 4, 32, None, None, L._ptr(g), L._ptr(m), n,
-                                         L._ptr(codes), None, None, None)
-        assert st == L.ERR_INVALID_ARG
-
-
-# ----------------------------------------------------------------------------- host path
-
-@pytest.mark.parametrize("name,kw,chunks", [
-    ("dense", dict(tokens=500, cin=128, rows=64), 8),
-    ("moe", dict(tokens=300, cin=96, rows=24, groups=20, top_k=3), 8),
-    ("moe", dict(tokens=300, cin=96, rows=24, groups=20, top_k=3), 3),
-    ("act", dict(tokens=300, cin=64, rows=40), 8),
-    ("mse", dict(), 1),
-])
-def test_calibrate_host_matches_the_device_path(name, kw, chunks):
-    """calibrate_host (pinned host inputs, grouped layers pipelined over chunks of groups on side
-    streams) returns exactly the codes, losses and fake-quantized weights of calibrate."""
-    mse = name == "mse"
-    layer = P.make_layer("dense" if mse else name, 61, **(dict(tokens=16, cin=64, rows=48) if mse else kw))
-    mode = "mse" if mse else layer.mode
-    d = P.layer_to_device(layer)
-    fused = mode == "act"
-    ref = L.calibrate(mode, d["x"], d["w"], group_offsets=d["offs"], token_ids=d["ids"],
-                      act_gx=d["act_gx"] if fused else None, xq=None)
-    _sync()
-    want = (ref.codes.cpu(), ref.loss.cpu(), ref.wq.cpu())
-    staging = {k: (torch.empty_like(v) if isinstance(v, torch.Tensor) else None) for k, v in d.items()}
-    pin = lambda t: None if t is None else t.cpu().pin_memory()  # noqa: E731
-    buf = L.Buffers(mode, layer.tokens, layer.cin, layer.rows, layer.groups, L.BF16 if layer.dtype == "bf16" else L.F32,
-                    "cuda")
-    out = L.calibrate_host(mode, pin(d["x"]), pin(d["w"]), buf, staging, group_offsets=pin(d["offs"]),
-                           token_ids=pin(d["ids"]), act_gx=d["act_gx"] if fused else None, group_chunks=chunks)
-    torch.cuda.current_stream().synchronize()
-    assert torch.equal(out.codes, want[0])
-    assert torch.equal(out.loss.view(torch.int32), want[1].view(torch.int32))
-    assert torch.equal(out.wq.view(torch.int32), want[2].view(torch.int32))
-    out2 = L.calibrate_host(mode, pin(d["x"]), pin(d["w"]), buf, staging, group_offsets=pin(d["offs"]),
-                            token_ids=pin(d["ids"]), act_gx=d["act_gx"] if fused else None,
-                            out=L.HostOutputs(buf, want_wq=False), group_chunks=chunks)
-    torch.cuda.current_stream().synchronize()
-    assert out2.wq is None and torch.equal(out2.codes, want[0])
 
 
 @pytest.mark.slow
