@@ -141,25 +141,65 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
   return static_cast<uint32_t>(r * kRowBytes + ((c ^ (r & 7)) << 4));
 }
 
+constexpr uint32_t kBand = 16 * kRowBytes;  // 16 rows: the swizzle repeats every 8
 
-// Loads one 64-token x 128-column tile (both tensors for ACT). Rows pos0 + r for r < 64 with
-// pos0 + r < end; grouped tiles take the row of position pos0 + r from ids_s[r] (shared
-// memory), dense tiles use the position itself. Rows past end and columns past cin are zeros.
+
+__device__ __forceinline__ void cp_async16_all(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src));
+}
+
+// What a thread copies of each tile: row r = tid / 4 and its 16-byte chunks c = j + 4 m (j = tid
+// % 4, m = 0..3), so that four lanes cover 64 contiguous bytes of the row per copy and the
+// thread needs one row address per tile (the chunks are 64 bytes apart). With x = r & 7, the
+// swizzled chunk c ^ x sits at byte 16 (j ^ (x & 3)) + 64 ((m & 1) ^ (x >> 2)) + 128 (m >> 1) of
+// the row: d0 for even m, d1 for odd m, plus 128 for m >= 2.
+struct TileRow {
+  uint32_t d0, d1;  // swizzled byte offsets of chunks m = 0 and m = 1 in a stage
+  int r;            // tile row
+  int j;            // first chunk
+};
+
+__device__ __forceinline__ TileRow tile_row(int tid) {
+  TileRow t;
+  t.r = tid >> 2;
+  t.j = tid & 3;
+  const int x = t.r & 7;
+  const uint32_t base = static_cast<uint32_t>(t.r * kRowBytes + 16 * (t.j ^ (x & 3)));
+  t.d0 = base + 64 * (x >> 2);
+  t.d1 = base + 64 * (1 - (x >> 2));
+  return t;
+}
+
+// Loads one 64-token x 128-column tile (both tensors for ACT) into the stage at shared address
+// stage: rows pos0 + r with pos0 + r < end, the row of position pos0 + r being ids_s[r] (grouped;
+// shared memory) or the position itself (dense). col is the thread's first element in a row (the
+// slab's first column + 8 j); bit m of cmask says whether chunk m lies inside cin. Rows past end
+// and chunks past cin are zero-filled.
 template <bool TWO>
-__device__ __forceinline__ void load_tile(uint8_t* smem_stage, const __nv_bfloat16* x,
-                                          const __nv_bfloat16* xq, int64_t ldx, int64_t col0,
-                                          int64_t cin, const int32_t* ids_s, int64_t pos0, int64_t end) {
-  const int tid = threadIdx.x;
-  const int c = tid & 15;
-  const bool col_ok = col0 + c * 8 < cin;
+__device__ __forceinline__ void load_tile(uint32_t stage, const TileRow& tr, const __nv_bfloat16* x,
+                                          const __nv_bfloat16* xq, int64_t ldx, int64_t col, uint32_t cmask,
+                                          const int32_t* ids_s, int64_t pos0, int64_t end) {
+  const bool row_ok = pos0 + tr.r < end;
+  const int64_t row = ids_s ? static_cast<int64_t>(ids_s[tr.r]) : pos0 + tr.r;
+  if (row_ok && cmask == 0xfu) {
+    const int64_t off = row * ldx + col;
 #pragma unroll
-  for (int m = 0; m < kTileTok / 16; ++m) {
-    const int r = (tid >> 4) + 16 * m;
-    const int64_t pos = pos0 + r;
-    const bool ok = col_ok && pos < end;
-    const int64_t row = ok ? (ids_s ? static_cast<int64_t>(ids_s[r]) : pos) : 0;
-    const int64_t off = ok ? row * ldx + col0 + c * 8 : 0;
-    const uint32_t dst = smem_u32(smem_stage) + swz(r, c);
+    for (int m = 0; m < 4; ++m) {
+      const uint32_t dst = stage + ((m & 1) ? tr.d1 : tr.d0) + 128 * (m >> 1);
+      if (TWO) {
+        cp_async16_all(dst, xq + off + 32 * m);
+        cp_async16_all(dst + kTileBytes, x + off + 32 * m);
+      } else {
+        cp_async16_all(dst, x + off + 32 * m);
+      }
+    }
+    return;
+  }
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const bool ok = row_ok && ((cmask >> m) & 1u);
+    const int64_t off = ok ? row * ldx + col + 32 * m : 0;
+    const uint32_t dst = stage + ((m & 1) ? tr.d1 : tr.d0) + 128 * (m >> 1);
     if (TWO) {
       cp_async16(dst, xq + off, ok);
       cp_async16(dst + kTileBytes, x + off, ok);
@@ -332,19 +372,41 @@ accum_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __res
   int64_t i_tile = 0;
   int64_t p_item = first_nonempty(it0, p_pos, p_end);
   int64_t c_item = first_nonempty(it0, c_pos, c_end);
+  // Ring slots of the id cursor, the data cursor and the consumer: tile t lives in slot t % S,
+  // kept as wrapping counters (S = 3 would otherwise be a 64-bit division per tile).
+  int i_slot = 0, p_slot = 0, c_slot = 0;
+  auto next_slot = [](int v) { return v + 1 == S ? 0 : v + 1; };
+  const uint32_t ring = smem_u32(smem);
+  const TileRow trow = tile_row(threadIdx.x);
+  // The data cursor's slab: the thread's first element in a row, and which of its chunks lie
+  // inside cin.
+  int64_t p_col = 0;
+  uint32_t p_cmask = 0;
+  auto set_slab = [&]() {
+    p_col = (p_item < it1 ? slab_of(p_item) : 0) * kSlabCols + 8 * trow.j;
+    p_cmask = 0;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) p_cmask |= (p_col + 32 * m < cin ? 1u : 0u) << m;
+  };
+  set_slab();
   auto issue_ids = [&]() {  // ids of tile i_tile into slot i_tile % S
     if (grouped && i_tile < ntiles) {
-      load_ids(ids_ring + (i_tile % S) * kTileTok, token_ids, i_pos, i_end);
+      load_ids(ids_ring + i_slot * kTileTok, token_ids, i_pos, i_end);
       i_pos += kTileTok;
       if (i_pos >= i_end) i_item = first_nonempty(i_item + 1, i_pos, i_end);
     }
     ++i_tile;
+    i_slot = next_slot(i_slot);
   };
-  auto produce = [&](int64_t tile) {  // data of tile into stage tile % S
-    load_tile<Cfg::kTwo>(smem + (tile % S) * stage_bytes, x, xq, ldx, slab_of(p_item) * kSlabCols, cin,
-                         grouped ? ids_ring + (tile % S) * kTileTok : nullptr, p_pos, p_end);
+  auto produce = [&]() {  // data of the next tile into its stage
+    load_tile<Cfg::kTwo>(ring + p_slot * stage_bytes, trow, x, xq, ldx, p_col, p_cmask,
+                         grouped ? ids_ring + p_slot * kTileTok : nullptr, p_pos, p_end);
+    p_slot = next_slot(p_slot);
     p_pos += kTileTok;
-    if (p_pos >= p_end) p_item = first_nonempty(p_item + 1, p_pos, p_end);
+    if (p_pos >= p_end) {
+      p_item = first_nonempty(p_item + 1, p_pos, p_end);
+      set_slab();
+    }
   };
 
   // Ids of the first S - 1 tiles, then the prologue: data of tiles 0..S-2 and ids S-1..2S-3.
@@ -356,23 +418,26 @@ accum_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __res
   for (int s2 = 0; s2 < S - 1; ++s2) {
     __syncthreads();  // the id slot refilled below was read by every thread for tile s2 - 1
     issue_ids();
-    if (s2 < ntiles) produce(s2);
+    if (s2 < ntiles) produce();
     cp_async_commit();
   }
 
   // ldmatrix.x4.trans addressing: lane -> (matrix mi = lane / 8, row rr = lane % 8);
   // matrices: (tok 0-7, cols 0-7), (tok 0-7, cols 8-15), (tok 8-15, cols 0-7), (tok 8-15, cols 8-15).
+  // Rows ts * 16 + lrow agree in their low three bits, so the 16-token steps are whole bands.
   const int mi = lane >> 3, rr = lane & 7;
   const int lrow = ((mi >> 1) << 3) + rr;
   const int lchunk = 2 * warp + (mi & 1);
+  const uint32_t loff = swz(lrow, lchunk);
 
   for (int64_t it = 0; it < ntiles; ++it) {
     cp_async_wait<S - 2>();
     __syncthreads();
     issue_ids();  // tile it + 2S - 2
-    if (it + S - 1 < ntiles) produce(it + S - 1);
+    if (it + S - 1 < ntiles) produce();  // tile it + S - 1
     cp_async_commit();
-    const uint32_t base = smem_u32(smem + (it % S) * stage_bytes);
+    const uint32_t base = ring + c_slot * stage_bytes;
+    c_slot = next_slot(c_slot);
     uint32_t qbase = base;               // X_q (ACT) or X (FULL)
     uint32_t xbase = base + kTileBytes;  // X (ACT)
     if (QUANT) {
@@ -403,7 +468,7 @@ accum_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __res
     }
 #pragma unroll
     for (int ts = 0; ts < kTileTok / 16; ++ts) {
-      const uint32_t off = swz(ts * 16 + lrow, lchunk);
+      const uint32_t off = loff + ts * kBand;
       uint32_t q0, q1, q2, q3;
       ldmatrix_x4_trans(qbase + off, q0, q1, q2, q3);
       mma_bf16(acc_h[0], q0, q1, q2, q3, q0, q2);
