@@ -79,9 +79,9 @@ PROFILED_TRAFFIC = {
     ("act", "sweep_tc_kernel"): {"bytes": 101_289_216 + 171_041_792},
     ("moe", "sweep_tc_kernel"): {"bytes": 10 * (420_447_488 + 678_123_264), "scaled": "x10 from 128 rows per expert"},
     ("wmse", "sweep_diag_kernel"): {"bytes": 100_809_000 + 163_823_616},
-    ("dense", "accum"): {"bytes": 134_267_136 + 4_176_896},
-    ("act", "accum"): {"bytes": 268_592_384 + 4_254_208},
-    ("moe", "accum"): {"bytes": 86_018_816 + 52_112_896},
+    ("dense", "accum"): {"bytes": 134_267_904 + 3_960_064},
+    ("act", "accum"): {"bytes": 268_599_552 + 3_796_736},
+    ("moe", "accum"): {"bytes": 84_716_032 + 49_333_248},
     ("wmse", "accum"): {"bytes": 1_610_622_000 + 7_723_264, "note": "accum_diag_kernel only"},
 }
 
