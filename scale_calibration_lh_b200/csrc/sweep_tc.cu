@@ -47,6 +47,7 @@
 // are 16-term dot products with rows of (H + H^T) / 2 read four at a time. The grid runs the
 // 16-column blocks fastest.
 #include <cstddef>
+#include <type_traits>
 
 #include "common.cuh"
 #include "quant_tables.cuh"
@@ -96,6 +97,39 @@ static_assert(offsetof(TcShared, tab) % 16 == 0 && offsetof(TcShared, h) % 16 ==
                   offsetof(TcShared, p) % 16 == 0 && offsetof(TcShared, hs) % 16 == 0 &&
                   offsetof(TcShared, wall) % 16 == 0 && (kWStride * sizeof(float)) % 16 == 0,
               "16-byte shared-memory accesses need 16-byte aligned rows");
+
+// Pair tables (bf16 weights). A bf16 magnitude a lies below an fp32 threshold t iff it lies
+// below the smallest bf16 value >= t, so the level decisions can be taken on bf16 thresholds,
+// two elements per packed compare. For candidate k and an element pair at levels (l0, l1) (l0
+// the A register's low half), thr2[k][8 l1 + l0] holds both elements' thresholds (bf16, l0 in
+// the low half) and q2[8 l1 + l0] both grid values as fp16 bits (candidate-independent). thr16
+// stages the bf16 thresholds per (k, level) so that a row of eight pairs is one 16-byte load.
+constexpr int kPairs = kLev * kLev;  // 64 level pairs
+constexpr int kPairRowBytes = kPairs * 4;
+struct __align__(16) TcPairShared {
+  uint32_t thr2[kCand * kPairs];
+  uint32_t q2[kPairs];
+  alignas(16) uint16_t thr16[kCand * kLev];
+};
+static_assert(offsetof(TcPairShared, thr16) % 16 == 0, "thr16 rows are read with 16-byte loads");
+
+// Smallest bf16 >= x (x >= 0; +inf stays +inf), as bits.
+__device__ __forceinline__ uint32_t bf16_ceil_bits(float x) {
+  const uint32_t b = __float_as_uint(x);
+  return (b >> 16) + ((b & 0xffffu) != 0u ? 1u : 0u);
+}
+
+// The pair's level step at one candidate: each half of a2 (bf16 magnitudes) below its half of
+// t2 (bf16 thresholds of its current level) drops that element one level, i.e. the pair index
+// 8 l1 + l0 by 1 (low half) and 8 (high half): 4 and 32 bytes of the table address.
+__device__ __forceinline__ void drop_pair(uint32_t& addr, uint32_t a2, uint32_t t2) {
+  asm("{\n\t.reg .pred pl, ph;\n\t"
+      "setp.lt.bf16x2 pl|ph, %1, %2;\n\t"
+      "@pl sub.u32 %0, %0, 4;\n\t"
+      "@ph sub.u32 %0, %0, 32;\n\t}\n"
+      : "+r"(addr)
+      : "r"(a2), "r"(t2));
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -165,6 +199,10 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
                 const float* __restrict__ p, const float* __restrict__ g, uint8_t* __restrict__ codes,
                 float* __restrict__ wq, float* __restrict__ loss) {
   __shared__ TcShared sh;
+  // bf16 weights: the pair tables, in dynamic shared memory (the launch sizes it).
+  constexpr bool kPair = std::is_same<WT, __nv_bfloat16>::value;
+  extern __shared__ __align__(16) uint8_t tc_dyn[];
+  TcPairShared& ps = *reinterpret_cast<TcPairShared*>(tc_dyn);
   const int64_t nblk = cin / kBlock;
   // Blocks vary fastest across the grid: CTAs running together cover neighbouring blocks of the
   // same rows, so their W reads are adjacent and their codes / loss writes share DRAM sectors.
@@ -186,9 +224,12 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
     const int k = idx >> 3, j = idx & 7;
     const float s = candidate_scale(k, gs);
     const uint32_t q16 = e2m1_grid_f16_bits(j);
-    sh.tab[idx] = make_float4(level_threshold(j, s), __uint_as_float(q16), __uint_as_float(q16 << 16),
-                              __fmul_rn(e2m1_grid(j), s));
+    const float thr = level_threshold(j, s);
+    sh.tab[idx] = make_float4(thr, __uint_as_float(q16), __uint_as_float(q16 << 16), __fmul_rn(e2m1_grid(j), s));
+    if (kPair) ps.thr16[idx] = static_cast<uint16_t>(bf16_ceil_bits(thr));
   }
+  if (kPair && threadIdx.x < kPairs)
+    ps.q2[threadIdx.x] = e2m1_grid_f16_bits(threadIdx.x & 7) | (e2m1_grid_f16_bits(threadIdx.x >> 3) << 16);
   for (int i = threadIdx.x; i < 4 * kOrderRows; i += kTcThreads) (&sh.hist[0][0])[i] = 0;
   const int64_t rbase = static_cast<int64_t>(blockIdx.y) * kUnitsPerCta;
   __syncthreads();
@@ -223,6 +264,22 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
     if (lane == 0) {
       const int ex = (m == 0u) ? 0 : static_cast<int>(m >> 23) - 127;  // floor(log2 max|H|)
       sh.hscale = pow2i(min(127, max(-126, 14 - ex)));
+    }
+  }
+  if (kPair) {
+    // Row (k, l1) of the pair table: eight entries (l0 = 0..7), from the bf16 thresholds of
+    // candidate k (one 16-byte load) and the threshold of level l1.
+    for (int kr = threadIdx.x; kr < kCand * kLev; kr += kTcThreads) {
+      const int k = kr >> 3, l1 = kr & 7;
+      const uint4 t8 = *reinterpret_cast<const uint4*>(ps.thr16 + k * kLev);
+      const uint32_t hi = static_cast<uint32_t>(ps.thr16[kr]) << 16;
+      const uint32_t tw[4] = {t8.x, t8.y, t8.z, t8.w};
+      uint32_t e[8];
+#pragma unroll
+      for (int l0 = 0; l0 < 8; ++l0) e[l0] = ((tw[l0 >> 1] >> (16 * (l0 & 1))) & 0xffffu) | hi;
+      uint4* dst = reinterpret_cast<uint4*>(ps.thr2 + k * kPairs + l1 * kLev);
+      dst[0] = make_uint4(e[0], e[1], e[2], e[3]);
+      dst[1] = make_uint4(e[4], e[5], e[6], e[7]);
     }
   }
   __syncthreads();
@@ -339,10 +396,7 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
   // C' is the same for every candidate of a unit, so the argmin compares L - C'; the winner's
   // loss is recomputed by its definition after the sweep.
   // The lane's share of t for units 0 and 1 (its 4 columns), before the reduction over the quad.
-  auto partials = [&](const uint32_t (&q)[8], int k, float (&tp)[2]) {
-    uint32_t afr[4];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) afr[r] = (q[kPairLo[r]] | q[kPairLo[r] + 1]) ^ smask[r];
+  auto partials_afr = [&](const uint32_t (&afr)[4], int k, float (&tp)[2]) {
     const float rk = sh.rho[k];
     const float2 rr = make_float2(rk, rk);
     float2 c0a = __fmul2_rn(rr, u0a), c0b = __fmul2_rn(rr, u0b);
@@ -359,6 +413,12 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
     const float2 p1 = __ffma2_rn(v67, make_float2(d1[2], d1[3]), __fmul2_rn(v45, make_float2(d0[2], d0[3])));
     tp[0] = p0.x + p0.y;
     tp[1] = p1.x + p1.y;
+  };
+  auto partials = [&](const uint32_t (&q)[8], int k, float (&tp)[2]) {
+    uint32_t afr[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) afr[r] = (q[kPairLo[r]] | q[kPairLo[r] + 1]) ^ smask[r];
+    partials_afr(afr, k, tp);
   };
   auto evaluate = [&](const uint32_t (&q)[8], int k) {
     float tp[2];
@@ -418,46 +478,9 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
   // tq ^ 2 finish. Each lane tracks the best of its own candidates; the quad merges them after
   // the loop.
   const bool b0 = (tq & 1) != 0, b1 = (tq & 2) != 0;
-#pragma unroll 1
-  for (int k = kinc; k < kCand; k += 4) {
-    float hold[2], spair[2][2];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t q[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float t;
-        if (c == 0) t = lds_f32<kTabRowBytes>(addr[i]);
-        else if (c == 1) t = lds_f32<2 * kTabRowBytes>(addr[i]);
-        else if (c == 2) t = lds_f32<3 * kTabRowBytes>(addr[i]);
-        else t = lds_f32<4 * kTabRowBytes>(addr[i]);
-        addr[i] = drop_if_below(addr[i], a[i], t, static_cast<uint32_t>(kEntryBytes));
-        constexpr int kQ0 = 4, kQ1 = 8;  // byte offsets of the low- and high-half fp16 words
-        if (i & 1) {
-          if (c == 0) q[i] = lds_u32<kTabRowBytes + kQ1>(addr[i]);
-          else if (c == 1) q[i] = lds_u32<2 * kTabRowBytes + kQ1>(addr[i]);
-          else if (c == 2) q[i] = lds_u32<3 * kTabRowBytes + kQ1>(addr[i]);
-          else q[i] = lds_u32<4 * kTabRowBytes + kQ1>(addr[i]);
-        } else {
-          if (c == 0) q[i] = lds_u32<kTabRowBytes + kQ0>(addr[i]);
-          else if (c == 1) q[i] = lds_u32<2 * kTabRowBytes + kQ0>(addr[i]);
-          else if (c == 2) q[i] = lds_u32<3 * kTabRowBytes + kQ0>(addr[i]);
-          else q[i] = lds_u32<4 * kTabRowBytes + kQ0>(addr[i]);
-        }
-      }
-      float tp[2];
-      partials(q, k + c, tp);
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        if ((c & 1) == 0) {
-          hold[u] = tp[u];
-        } else {  // candidates (c - 1, c): keep the one with index bit b0, hand over the other
-          spair[c >> 1][u] = (b0 ? tp[u] : hold[u]) + __shfl_xor_sync(0xffffffffu, b0 ? hold[u] : tp[u], 1);
-        }
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) addr[i] += 4 * kTabRowBytes;
+  // One loop trip's bookkeeping after the four candidates: the reductions' second stage and the
+  // best of the lane's candidate k + tq.
+  auto finish4 = [&](int k, const float (&spair)[2][2]) {
     const int kk = k + tq;
     const float s2 = sh.s2[kk];
 #pragma unroll
@@ -468,6 +491,95 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
         best[u] = L;
         best_k[u] = kk;
       }
+    }
+  };
+  auto stage_pair = [&](int c, const float (&tp)[2], float (&hold)[2], float (&spair)[2][2]) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if ((c & 1) == 0) {
+        hold[u] = tp[u];
+      } else {  // candidates (c - 1, c): keep the one with index bit b0, hand over the other
+        spair[c >> 1][u] = (b0 ? tp[u] : hold[u]) + __shfl_xor_sync(0xffffffffu, b0 ? hold[u] : tp[u], 1);
+      }
+    }
+  };
+  // bf16 magnitudes of the A registers' element pairs (exact: the weights are bf16).
+  uint32_t a2[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+    a2[r] = (__float_as_uint(a[kPairLo[r]]) >> 16) | (__float_as_uint(a[kPairLo[r] + 1]) & 0xffff0000u);
+  if constexpr (kPair) {
+    // Pair addresses in the row of candidate kinc - 1, from the levels the direct loop left.
+    const uint32_t thr2_base = smem_u32(ps.thr2), q2_base = smem_u32(ps.q2);
+    uint32_t pa[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const uint32_t l0 = ((addr[kPairLo[r]] - tab_base) >> 4) & 7u;
+      const uint32_t l1 = ((addr[kPairLo[r] + 1] - tab_base) >> 4) & 7u;
+      pa[r] = thr2_base + static_cast<uint32_t>((kinc - 1) * kPairRowBytes) + (8u * l1 + l0) * 4u;
+    }
+    // pa - qoff is the pair's grid-value entry: qoff removes the row and the table base.
+    uint32_t qoff = thr2_base + static_cast<uint32_t>((kinc - 1) * kPairRowBytes) - q2_base;
+#pragma unroll 1
+    for (int k = kinc; k < kCand; k += 4) {
+      float hold[2], spair[2][2];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t afr[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          uint32_t t2;
+          if (c == 0) t2 = lds_u32<kPairRowBytes>(pa[r]);
+          else if (c == 1) t2 = lds_u32<2 * kPairRowBytes>(pa[r]);
+          else if (c == 2) t2 = lds_u32<3 * kPairRowBytes>(pa[r]);
+          else t2 = lds_u32<4 * kPairRowBytes>(pa[r]);
+          drop_pair(pa[r], a2[r], t2);
+          afr[r] = lds_u32<0>(pa[r] - qoff) ^ smask[r];
+        }
+        float tp[2];
+        partials_afr(afr, k + c, tp);
+        stage_pair(c, tp, hold, spair);
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r) pa[r] += 4 * kPairRowBytes;
+      qoff += 4 * kPairRowBytes;
+      finish4(k, spair);
+    }
+  } else {
+#pragma unroll 1
+    for (int k = kinc; k < kCand; k += 4) {
+      float hold[2], spair[2][2];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t q[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float t;
+          if (c == 0) t = lds_f32<kTabRowBytes>(addr[i]);
+          else if (c == 1) t = lds_f32<2 * kTabRowBytes>(addr[i]);
+          else if (c == 2) t = lds_f32<3 * kTabRowBytes>(addr[i]);
+          else t = lds_f32<4 * kTabRowBytes>(addr[i]);
+          addr[i] = drop_if_below(addr[i], a[i], t, static_cast<uint32_t>(kEntryBytes));
+          constexpr int kQ0 = 4, kQ1 = 8;  // byte offsets of the low- and high-half fp16 words
+          if (i & 1) {
+            if (c == 0) q[i] = lds_u32<kTabRowBytes + kQ1>(addr[i]);
+            else if (c == 1) q[i] = lds_u32<2 * kTabRowBytes + kQ1>(addr[i]);
+            else if (c == 2) q[i] = lds_u32<3 * kTabRowBytes + kQ1>(addr[i]);
+            else q[i] = lds_u32<4 * kTabRowBytes + kQ1>(addr[i]);
+          } else {
+            if (c == 0) q[i] = lds_u32<kTabRowBytes + kQ0>(addr[i]);
+            else if (c == 1) q[i] = lds_u32<2 * kTabRowBytes + kQ0>(addr[i]);
+            else if (c == 2) q[i] = lds_u32<3 * kTabRowBytes + kQ0>(addr[i]);
+            else q[i] = lds_u32<4 * kTabRowBytes + kQ0>(addr[i]);
+          }
+        }
+        float tp[2];
+        partials(q, k + c, tp);
+        stage_pair(c, tp, hold, spair);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) addr[i] += 4 * kTabRowBytes;
+      finish4(k, spair);
     }
   }
   // Merge the quad's bests: the smallest loss, and on equal losses the lowest candidate.
@@ -493,8 +605,11 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
     // The sign bit of element i, from the packed A-register masks (not kept live through the sweep).
     constexpr int kPairOf[8] = {0, 0, 2, 2, 1, 1, 3, 3};
     const uint32_t sbit = (smask[kPairOf[i]] >> ((i & 1) ? 31 : 15)) & 1u;
-    wqv[i] = __uint_as_float(__float_as_uint(tab_k[level_direct_tc(tab_k, a[i])].w) | (sbit << 31));
-    dwv[i] = wqv[i] - __uint_as_float(__float_as_uint(a[i]) | (sbit << 31));
+    // bf16 weights: |w| from the packed pairs, so that a[] need not stay live through the sweep.
+    constexpr int kRegOf[8] = {0, 0, 2, 2, 1, 1, 3, 3};
+    const float ai = kPair ? __uint_as_float((i & 1) ? (a2[kRegOf[i]] & 0xffff0000u) : (a2[kRegOf[i]] << 16)) : a[i];
+    wqv[i] = __uint_as_float(__float_as_uint(tab_k[level_direct_tc(tab_k, ai)].w) | (sbit << 31));
+    dwv[i] = wqv[i] - __uint_as_float(__float_as_uint(ai) | (sbit << 31));
   }
 #pragma unroll 1
   for (int u = 0; u < 2; ++u) {
@@ -567,11 +682,21 @@ lhcal_status launch_sweep_tc(lhcal_mode mode, lhcal_dtype dtype, const void* w, 
   const dim3 grid(static_cast<unsigned>(cin / kBlock), static_cast<unsigned>(ceil_div(rows, kUnitsPerCta)),
                   static_cast<unsigned>(groups));
   if (dtype == LHCAL_BF16) {
+    // The pair tables live in dynamic shared memory; with the static part a CTA holds about 69 KB,
+    // three per SM. Set on every call with the same values: cheap, and right for any device.
+    constexpr int kDyn = static_cast<int>(sizeof(TcPairShared));
+    for (const void* fn : {reinterpret_cast<const void*>(sweep_tc_kernel<true, __nv_bfloat16>),
+                           reinterpret_cast<const void*>(sweep_tc_kernel<false, __nv_bfloat16>)}) {
+      cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kDyn);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+      if (e != cudaSuccess) return fail(LHCAL_ERR_CUDA, "scale sweep: %s", cudaGetErrorString(e));
+    }
     if (mode == LHCAL_ACT_AWARE)
-      sweep_tc_kernel<true, __nv_bfloat16><<<grid, kTcThreads, 0, stream>>>(
+      sweep_tc_kernel<true, __nv_bfloat16><<<grid, kTcThreads, kDyn, stream>>>(
           static_cast<const __nv_bfloat16*>(w), rows, cin, h, p, g, codes, wq, loss);
     else
-      sweep_tc_kernel<false, __nv_bfloat16><<<grid, kTcThreads, 0, stream>>>(
+      sweep_tc_kernel<false, __nv_bfloat16><<<grid, kTcThreads, kDyn, stream>>>(
           static_cast<const __nv_bfloat16*>(w), rows, cin, h, p, g, codes, wq, loss);
   } else {
     if (mode == LHCAL_ACT_AWARE)
