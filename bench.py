@@ -75,9 +75,9 @@ WORKLOAD_TEXT = {
 # counters). The fused-MoE sweep was captured with 128 rows per expert and is scaled to the
 # 1280 rows of the workload (its traffic, W in and Wq out, grows with the rows).
 PROFILED_TRAFFIC = {
-    ("dense", "sweep_tc_kernel"): {"bytes": 33_872_128 + 23_449_856},
-    ("act", "sweep_tc_kernel"): {"bytes": 101_289_216 + 171_041_792},
-    ("moe", "sweep_tc_kernel"): {"bytes": 10 * (420_447_488 + 678_123_264), "scaled": "x10 from 128 rows per expert"},
+    ("dense", "sweep_tc_kernel"): {"bytes": 33_860_608 + 27_109_120},
+    ("act", "sweep_tc_kernel"): {"bytes": 101_325_824 + 171_952_384},
+    ("moe", "sweep_tc_kernel"): {"bytes": 10 * (419_859_200 + 700_098_816), "scaled": "x10 from 128 rows per expert"},
     ("wmse", "sweep_diag_kernel"): {"bytes": 100_809_000 + 163_823_616},
     ("dense", "accum"): {"bytes": 134_267_904 + 3_960_064},
     ("act", "accum"): {"bytes": 268_599_552 + 3_796_736},
