@@ -324,6 +324,7 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
   float a[8], up[8];
   uint32_t sgn[8];
   float pa[2], pb[2];
+  float pwk[8];  // activation-aware: (P w)_c of each lane element, kept for the epilogue
 #pragma unroll
   for (int u = 0; u < 2; ++u) {
     // The unit's 16 weights and their signs (+-1), then per lane column c of the unit:
@@ -363,6 +364,7 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
       a[i] = fabsf(x);
       sgn[i] = __float_as_uint(x) >> 31;
       up[i] = hw - pw;  // U'_c
+      pwk[i] = pw;
       qa = fmaf(sc, hsg, qa);
       qb = fmaf(sc, up[i], qb);
     }
@@ -376,6 +378,16 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
     }
     pa[u] = 36.f * qa;
     pb[u] = -12.f * qb;
+  }
+  if (ACT && kPair) {
+    // The epilogue needs (P w)_c again. Rather than keep it in registers through the sweep, each
+    // lane stores its eight values over the staged weights of its own units' rows, once every
+    // lane of the warp has read those rows (only this warp reads them, and after this only the
+    // writing lane reads the entries it wrote). fp32 weights recompute it in the epilogue (the
+    // stored form measured a large spill in that build).
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) sh.wall[sh.perm[warp * kUnitsPerWarp + gq + 8 * (i >> 2)]][col_of(i & 3)] = pwk[i];
   }
   // Sign masks of the four packed A registers: a0 = (elems 0,1), a1 = (4,5), a2 = (2,3), a3 = (6,7).
   constexpr int kPairLo[4] = {0, 4, 2, 6};
@@ -642,17 +654,21 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
         hd = fmaf(hq.z, dfull[k + 2], hd);
         hd = fmaf(hq.w, dfull[k + 3], hd);
       }
-      if (ACT) {  // + 2 (P w)_c, with w from the CTA's shared copy
+      if (ACT) {  // + 2 (P w)_c
         const float* wr = sh.wall[sh.perm[warp * kUnitsPerWarp + gq + 8 * u]];
         float pw = 0.f;
+        if (kPair) {
+          pw = wr[c];  // as the set-up computed it, stored over the unit's staged row
+        } else {  // from the staged weights, in the set-up's order
 #pragma unroll
-        for (int k = 0; k < 16; k += 4) {
-          const float4 pq = *reinterpret_cast<const float4*>(sh.p + c * 16 + k);
-          const float4 wq4v = *reinterpret_cast<const float4*>(wr + k);
-          pw = fmaf(pq.x, wq4v.x, pw);
-          pw = fmaf(pq.y, wq4v.y, pw);
-          pw = fmaf(pq.z, wq4v.z, pw);
-          pw = fmaf(pq.w, wq4v.w, pw);
+          for (int k = 0; k < 16; k += 4) {
+            const float4 pq = *reinterpret_cast<const float4*>(sh.p + c * 16 + k);
+            const float4 wq4v = *reinterpret_cast<const float4*>(wr + k);
+            pw = fmaf(pq.x, wq4v.x, pw);
+            pw = fmaf(pq.y, wq4v.y, pw);
+            pw = fmaf(pq.z, wq4v.z, pw);
+            pw = fmaf(pq.w, wq4v.w, pw);
+          }
         }
         hd = fmaf(2.f, pw, hd);
       }
