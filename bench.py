@@ -76,7 +76,7 @@ WORKLOAD_TEXT = {
 # 1280 rows of the workload (its traffic, W in and Wq out, grows with the rows).
 PROFILED_TRAFFIC = {
     ("dense", "sweep_tc_kernel"): {"bytes": 33_860_608 + 27_109_120},
-    ("act", "sweep_tc_kernel"): {"bytes": 101_325_824 + 171_952_384},
+    ("act", "sweep_tc_kernel"): {"bytes": 101_307_648 + 172_282_880},
     ("moe", "sweep_tc_kernel"): {"bytes": 10 * (419_859_200 + 700_098_816), "scaled": "x10 from 128 rows per expert"},
     ("wmse", "sweep_diag_kernel"): {"bytes": 100_809_000 + 163_823_616},
     ("dense", "accum"): {"bytes": 134_267_904 + 3_960_064},

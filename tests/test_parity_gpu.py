@@ -141,10 +141,11 @@ def test_fp32_inputs_all_modes(mode, grouped):
 
 # ----------------------------------------------------------------------------- sweep special cases
 
-def _sweep_gpu(mode, w, h, p, g):
-    """w fp32 [G,R,C]; h/p/g from the oracle side (fp32-rounded) -> GPU outputs (numpy)."""
+def _sweep_gpu(mode, w, h, p, g, w_bf16=False):
+    """w fp32 [G,R,C] (bf16-exact values when w_bf16: the kernel then reads bf16 weights); h/p/g
+    from the oracle side (fp32-rounded) -> GPU outputs (numpy)."""
     G, R, C = w.shape
-    dw = P.to_device(w, "f32")
+    dw = P.to_device((w.view(np.uint32) >> 16).astype(np.uint16), "bf16") if w_bf16 else P.to_device(w, "f32")
     dh = P.to_device(np.asarray(h, np.float32), "f32")
     dp = None if p is None else P.to_device(np.asarray(p, np.float32), "f32")
     dg = P.to_device(g, "f32")
@@ -208,6 +209,72 @@ def test_sweep_special_weights_with_oracle_hessians(mode):
     # Degenerate units: every candidate ties, the lowest code wins, outputs are signed zeros.
     assert np.all(codes[2] == 1) and np.all(codes[0, 0] == 1)
     assert np.all(wq[2] == 0) and np.all(wq[0, 1, 16:32].view(np.int32) == np.float32(-0.0).view(np.int32))
+
+
+def _bf16_step(t: np.ndarray, up: bool) -> np.ndarray:
+    """The neighbouring bf16 value of positive bf16 values t (as fp32), above or below."""
+    b = (t.view(np.uint32) >> 16).astype(np.int64) + (1 if up else -1)
+    return (b.astype(np.uint32) << 16).view(np.float32)
+
+
+def _bf16_tie_weights(seed=12):
+    """bf16 weights whose group 0 has the global scale 2^-12 (its largest |w| is 2688 * 2^-12), so
+    that every E2M1 midpoint times a candidate scale (at most 7 significant bits) is a bf16 value:
+    rows of exact ties, their bf16 neighbours above and below, and ordinary weights. Group 1 has
+    an arbitrary global scale, where the rounded midpoints are near-ties."""
+    rng = np.random.default_rng(seed)
+    G, R, C = 2, 48, 64
+    w = rng.normal(0, 0.02, (G, R, C)).astype(np.float32)
+    w = ((w.view(np.uint32) >> 16) << 16).view(np.float32)  # bf16 values
+    w[0, 0, 0] = np.float32(2688.0 * 2.0 ** -12)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    for e in range(G):
+        s = O.candidate_scales(O.global_scale(w[e]))
+        for r in range(1, 41):
+            k = rng.integers(0, 126)
+            t = (mids[rng.integers(0, 7, 16)] * np.float64(s[k])).astype(np.float32)
+            t = ((t.view(np.uint32) >> 16) << 16).view(np.float32)  # exact in group 0
+            sign = np.where(rng.random(16) < 0.5, -1, 1).astype(np.float32)
+            w[e, r, :16] = t * sign
+            w[e, r, 16:32] = _bf16_step(t, True) * sign
+            w[e, r, 32:48] = _bf16_step(t, False) * sign
+    return w
+
+
+@pytest.mark.parametrize("mode", ["full", "act"])
+def test_sweep_bf16_weights_at_exact_ties(mode):
+    """The bf16 weight path decides E2M1 levels on bf16 thresholds, two elements per packed
+    compare: exact ties (round half to even) and their bf16 neighbours against the oracle."""
+    w = _bf16_tie_weights()
+    G, R, C = w.shape
+    g = np.array([O.global_scale(w[e]) for e in range(G)], np.float32)
+    assert g[0] == np.float32(2.0 ** -12)
+    s0 = O.candidate_scales(g[0]).astype(np.float64)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    a = np.abs(w[0, 1:41, :16]).astype(np.float64)
+    assert np.isin(a, np.outer(mids, s0)).all()  # every one an exact tie for some candidate
+    nblk = C // 16
+    rng = np.random.default_rng(13)
+    x = (rng.normal(size=(200, C)) * rng.lognormal(0, 1, C)).astype(np.float32)
+    if mode == "act":
+        xq = (x * 0.95 + rng.normal(0, 0.05, x.shape)).astype(np.float32)
+        hs, ps = O.hessian_sum_act(x, xq)
+        h = np.broadcast_to(hs / 200, (G, nblk, 16, 16)).astype(np.float32)
+        p = np.broadcast_to(ps / 200, (G, nblk, 16, 16)).astype(np.float32)
+    else:
+        h = np.broadcast_to(O.hessian_sum_full(x) / 200, (G, nblk, 16, 16)).astype(np.float32)
+        p = None
+    codes, wq, loss = _sweep_gpu(L.MODE_IDS[mode], w, h, p, g, w_bf16=True)
+    units = P.all_units(G, R, nblk)
+    ref = P.oracle_sweep(mode, w, h.astype(np.float64), None if p is None else p.astype(np.float64), g, units)
+    gc, gw, gl = P.gather_gpu_units(codes, wq, loss, units)
+    rep = P.check_sweep(gc, gw, gl, ref, f"bf16 ties {mode}")
+    assert rep["units"] == G * R * nblk
+    # The same weights as fp32 take the fp32 thresholds: identical codes, weights and losses.
+    c32, w32, l32 = _sweep_gpu(L.MODE_IDS[mode], w, h, p, g)
+    assert np.array_equal(codes, c32)
+    assert np.array_equal(wq.view(np.int32), w32.view(np.int32))
+    assert np.array_equal(loss.view(np.int32), l32.view(np.int32))
 
 
 def test_sweep_identity_hessian_is_plain_mse():
