@@ -524,6 +524,7 @@ def measure_workload(name, args, rank, world, dev, flusher):
         "clocks": clk,
     }
     rec.update(e2e)
+    rec["searches"] = measure_searches(L, mode, layer, d, buf, units, stream, dev, peak_ops, events, rank_max, flusher)
     if small:
         rec["latency_bound"] = True
     if two_tensor is not None:
@@ -540,6 +541,55 @@ def measure_workload(name, args, rank, world, dev, flusher):
     del d, buf, hx, hxq, hw, hoffs, hids
     torch.cuda.empty_cache()
     return rec
+
+
+# The amax-multiplier search's multipliers: the pages name a step size and multipliers but give no
+# values, so the bench takes 38 of them, 0.25 + 0.1 i (an amax range of 0.25x to 3.95x).
+SEARCH_MULTIPLIERS = [0.25 + 0.1 * i for i in range(38)]
+
+
+def measure_searches(L, mode, layer, d, buf, units, stream, dev, peak_ops, events, rank_max, flusher):
+    """The non-sweep searches on the workload's finalized statistics, timed alone: the
+    amax-multiplier search in the workload's mode, and (one-group layers) the plain MSE sweep
+    (H = I). Each is the median of 5 launches after one untimed launch and an L2 flush before
+    each; the fraction is the FP32 lane peak against the direct method's lane-ops per evaluated
+    scale (the search evaluates at most one scale per multiplier and skips repeated codes)."""
+    import torch
+
+    out = {}
+    mult = torch.tensor(SEARCH_MULTIPLIERS, dtype=torch.float32, device=dev)
+    codes = torch.empty_like(buf.codes)
+
+    def timed(fn, reps=5):
+        fn()
+        torch.cuda.synchronize()
+        evs = [events(2) for _ in range(reps)]
+        for a, b in evs:
+            flusher()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        (ms,) = rank_max([median(a.elapsed_time(b) for a, b in evs)], dev)
+        return ms
+
+    ms = timed(lambda: L.lhcal_multiplier_search(mode, d["w"], buf.h, buf.g, mult, codes, p=buf.p))
+    ops = units * len(SEARCH_MULTIPLIERS) * OPS_PER_CANDIDATE[layer.mode]
+    out["multiplier_search"] = {
+        "kernel": "msearch_kernel", "mode": layer.mode, "multipliers": len(SEARCH_MULTIPLIERS), "ms": ms,
+        "units_per_s": units / (ms / 1e3), "bound": "alu", "achieved": ops / (ms / 1e3) / 1e12,
+        "peak": peak_ops / 1e12, "unit": "Tops/s", "frac": ops / (ms / 1e3) / peak_ops,
+        "note": "multipliers 0.25 + 0.1 i, i < 38; outputs: codes only"}
+    if layer.groups == 1 and layer.mode != "diag":
+        g = torch.empty_like(buf.g)
+        L.lhcal_global_scale(d["w"], g)
+        ms2 = timed(lambda: L.lhcal_scale_sweep("mse", d["w"], None, g, codes))
+        ops2 = units * 126 * OPS_PER_CANDIDATE["diag"]
+        out["mse_sweep"] = {
+            "kernel": "sweep_diag_kernel (importance 1)", "ms": ms2, "units_per_s": units / (ms2 / 1e3),
+            "bound": "alu", "achieved": ops2 / (ms2 / 1e3) / 1e12, "peak": peak_ops / 1e12, "unit": "Tops/s",
+            "frac": ops2 / (ms2 / 1e3) / peak_ops, "note": "126 candidates, H = I; outputs: codes only"}
+    return out
 
 
 def measure_sharded(name, args, rank, world, dev):

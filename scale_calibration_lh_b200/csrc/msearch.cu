@@ -21,8 +21,8 @@ namespace {
 
 constexpr int kMsThreads = 128;
 
-struct MsShared {
-  float h[256];  // FULL/ACT: H of the block; DIAG: Imp in the first 16
+struct __align__(16) MsShared {
+  float h[256];  // FULL/ACT: H of the block; DIAG: Imp in the first 16 (rows read 16 bytes at a time)
   float p[256];  // ACT: P of the block
   float mult[kMaxMultipliers];
 };
@@ -48,6 +48,17 @@ __device__ __forceinline__ int e4m3_code_of(float a, float g) {
   while (c < 126 && reaches_code(a, c + 1, g6)) ++c;
   while (c > 0 && !reaches_code(a, c, g6)) --c;
   return c;
+}
+
+// Four entries of a shared-memory row. volatile: H is read again for every evaluated scale
+// rather than hoisted out of the multiplier loop into 256 registers (which left one CTA's worth
+// of warps per SM).
+__device__ __forceinline__ float4 lds_row4(const float* p) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];\n"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
+  return v;
 }
 
 template <int MODE>
@@ -81,7 +92,13 @@ __device__ __forceinline__ float unit_loss(const float (&w)[16], const float (&p
     for (int i = 0; i < 16; ++i) {
       float r = 0.f;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) r = fmaf(sh.h[i * 16 + j], dw[j], r);
+      for (int j = 0; j < 16; j += 4) {  // row i of H, in column order
+        const float4 hq = lds_row4(sh.h + i * 16 + j);
+        r = fmaf(hq.x, dw[j], r);
+        r = fmaf(hq.y, dw[j + 1], r);
+        r = fmaf(hq.z, dw[j + 2], r);
+        r = fmaf(hq.w, dw[j + 3], r);
+      }
       L = fmaf(dw[i], r, L);
       if (MODE == LHCAL_ACT_AWARE) L = fmaf(2.f * dw[i], pw[i], L);
     }
