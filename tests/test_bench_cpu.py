@@ -177,3 +177,17 @@ def test_headline_is_the_largest_workload_and_all_run_by_default():
 
 def test_median_of_stage_times():
     assert bench.median([3, 1, 2]) == 2 and bench.median([4, 1, 3, 2]) == 2.5
+
+
+def test_search_multipliers_are_the_stated_grid():
+    # 38 multipliers 0.25 + 0.1 i: an amax range of 0.25x to 3.95x, ascending (so that the search's
+    # first-best rule and the lowest-code rule agree).
+    m = np.array(bench.SEARCH_MULTIPLIERS)
+    assert len(m) == 38 and np.all(np.diff(m) > 0)
+    np.testing.assert_allclose(m, 0.25 + 0.1 * np.arange(38))
+
+
+def test_search_fractions_count_38_direct_evaluations_per_unit():
+    # The multiplier search's numerator: units x 38 x the direct method's lane-ops per candidate.
+    units = 1_048_576
+    assert units * len(bench.SEARCH_MULTIPLIERS) * bench.OPS_PER_CANDIDATE["full"] == 7_331_643_392
