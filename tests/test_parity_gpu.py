@@ -146,7 +146,7 @@ def _sweep_gpu(mode, w, h, p, g, w_bf16=False):
     from the oracle side (fp32-rounded) -> GPU outputs (numpy)."""
     G, R, C = w.shape
     dw = P.to_device((w.view(np.uint32) >> 16).astype(np.uint16), "bf16") if w_bf16 else P.to_device(w, "f32")
-    dh = P.to_device(np.asarray(h, np.float32), "f32")
+    dh = None if h is None else P.to_device(np.asarray(h, np.float32), "f32")
     dp = None if p is None else P.to_device(np.asarray(p, np.float32), "f32")
     dg = P.to_device(g, "f32")
     codes = torch.empty((G, R, C // 16), dtype=torch.uint8, device="cuda")
@@ -241,10 +241,11 @@ def _bf16_tie_weights(seed=12):
     return w
 
 
-@pytest.mark.parametrize("mode", ["full", "act"])
+@pytest.mark.parametrize("mode", ["full", "act", "diag", "mse"])
 def test_sweep_bf16_weights_at_exact_ties(mode):
-    """The bf16 weight path decides E2M1 levels on bf16 thresholds, two elements per packed
-    compare: exact ties (round half to even) and their bf16 neighbours against the oracle."""
+    """bf16 weights at exact E2M1 ties (round half to even) and their bf16 neighbours against the
+    oracle, in every sweep mode; the tensor-core sweep decides their levels on bf16 thresholds,
+    two elements per packed compare."""
     w = _bf16_tie_weights()
     G, R, C = w.shape
     g = np.array([O.global_scale(w[e]) for e in range(G)], np.float32)
@@ -256,21 +257,27 @@ def test_sweep_bf16_weights_at_exact_ties(mode):
     nblk = C // 16
     rng = np.random.default_rng(13)
     x = (rng.normal(size=(200, C)) * rng.lognormal(0, 1, C)).astype(np.float32)
+    p = None
     if mode == "act":
         xq = (x * 0.95 + rng.normal(0, 0.05, x.shape)).astype(np.float32)
         hs, ps = O.hessian_sum_act(x, xq)
         h = np.broadcast_to(hs / 200, (G, nblk, 16, 16)).astype(np.float32)
         p = np.broadcast_to(ps / 200, (G, nblk, 16, 16)).astype(np.float32)
+    elif mode == "diag":
+        h = np.broadcast_to(O.importance_sum(x), (G, nblk, 16)).astype(np.float32)
+    elif mode == "mse":
+        h = None  # every importance 1
     else:
         h = np.broadcast_to(O.hessian_sum_full(x) / 200, (G, nblk, 16, 16)).astype(np.float32)
-        p = None
     codes, wq, loss = _sweep_gpu(L.MODE_IDS[mode], w, h, p, g, w_bf16=True)
     units = P.all_units(G, R, nblk)
-    ref = P.oracle_sweep(mode, w, h.astype(np.float64), None if p is None else p.astype(np.float64), g, units)
+    href = None if h is None else h.astype(np.float64)
+    ref = P.oracle_sweep(mode, w, href, None if p is None else p.astype(np.float64), g, units)
     gc, gw, gl = P.gather_gpu_units(codes, wq, loss, units)
     rep = P.check_sweep(gc, gw, gl, ref, f"bf16 ties {mode}")
     assert rep["units"] == G * R * nblk
-    # The same weights as fp32 take the fp32 thresholds: identical codes, weights and losses.
+    # The same weights as fp32: identical codes, weights and losses (the FULL and activation-aware
+    # bf16 paths decide on bf16 thresholds, the others share the fp32 code).
     c32, w32, l32 = _sweep_gpu(L.MODE_IDS[mode], w, h, p, g)
     assert np.array_equal(codes, c32)
     assert np.array_equal(wq.view(np.int32), w32.view(np.int32))
