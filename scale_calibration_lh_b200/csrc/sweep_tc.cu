@@ -29,9 +29,12 @@
 //
 // Quantization. As in the FP32 sweep: per-candidate threshold tables built from exact
 // residuals decide the E2M1 level of every element exactly as on the exact quotient, and
-// each element's level falls by at most one per candidate from the 4th on. Each table entry
-// also carries the fp16 bits of its grid value, pre-placed for the low or the high half of
-// a packed pair, so building the A fragment is one OR (and a sign XOR) per pair.
+// each element's level falls by at most one per candidate from the 4th on. fp32 weights: each
+// table entry also carries the fp16 bits of its grid value, pre-placed for the low or the high
+// half of a packed pair, so building the A fragment is one OR (and a sign XOR) per pair. bf16
+// weights: the levels are tracked per pair (the two halves of an A register) on bf16 copies of
+// the thresholds, which decide exactly as the fp32 ones for bf16 magnitudes: one load of the
+// pair's two thresholds, one packed compare, one load of the pair's two grid values.
 //
 // Work per candidate. Candidates below the warp's first unclamped one take a closed form;
 // the rest go four per loop trip, and the quad's four lanes share the reduction of four
