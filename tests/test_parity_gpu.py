@@ -118,6 +118,26 @@ def test_moe_grouped_full_rank_experts():
     assert r["sweep"]["exempt"] < 0.05 * r["sweep"]["units"]
 
 
+@pytest.mark.parametrize("variant", ["full", "act", "act_fused"])
+def test_moe_grouped_tile_boundaries(variant):
+    """Experts with 0, 1, 63, 64, 65, 127, 128, 129 and 200 routed rows (the 64-row tiles of the
+    grouped accumulation full, ragged and empty) over cin = 160 (one full 128-column slab and a
+    partial one): the loader's unpredicated copies for full tiles and predicated ones for ragged
+    tiles and out-of-range columns, against the oracle."""
+    counts = [0, 1, 63, 64, 65, 127, 128, 129, 200]
+    T = 300
+    layer = synth.make_layer("moe", 41, tokens=T, cin=160, rows=20, groups=len(counts), top_k=2)
+    rng = np.random.default_rng(42)
+    ids = [np.sort(rng.choice(T, size=c, replace=False)) for c in counts]
+    layer.group_offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    layer.token_ids = np.concatenate(ids).astype(np.int32)
+    if variant != "full":
+        layer.mode = "act"
+        P.act_inputs(layer)
+    assert np.array_equal(np.diff(layer.group_offsets), counts)
+    _run_and_check(layer, fused=variant == "act_fused")
+
+
 def test_moe_grouped_diag_bf16_generic_path():
     layer = P.make_layer("moe", 5, tokens=50, cin=48, rows=20, groups=8, top_k=2)
     layer.mode = "diag"
