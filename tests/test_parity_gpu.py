@@ -384,14 +384,16 @@ def test_accumulate_add_equals_one_pass_and_is_deterministic():
     assert torch.equal(p2.view(torch.int32), p3.view(torch.int32))
 
 
+@pytest.mark.parametrize("cin", [4096, 4000])
 @pytest.mark.parametrize("name", ["dense", "act"])
-def test_accumulate_cluster_path_overwrite_and_add(name):
-    """Wide layers (32 column slabs) reduce token splits inside CTA clusters, with no workspace."""
-    layer = P.make_layer(name, 14, tokens=3001, cin=4096, rows=2)
+def test_accumulate_cluster_path_overwrite_and_add(name, cin):
+    """Wide layers (32 column slabs; with cin = 4000 the last holds 32 columns) reduce token
+    splits inside CTA clusters, with no workspace."""
+    layer = P.make_layer(name, 14, tokens=3001, cin=cin, rows=2)
     mode = layer.mode
     assert L.lhcal_accumulate_workspace(mode, L.BF16, layer.tokens, layer.cin, 1) == 0
     d = P.layer_to_device(layer)
-    shape = (1, 256, 16, 16)
+    shape = (1, cin // 16, 16, 16)
     h = torch.full(shape, 3.0, dtype=torch.float32, device="cuda")
     p = torch.full(shape, 3.0, dtype=torch.float32, device="cuda") if mode == "act" else None
     L.lhcal_accumulate(mode, d["x"], h, xq=d["xq"], p=p, flags=L.ACCUM_OVERWRITE)
