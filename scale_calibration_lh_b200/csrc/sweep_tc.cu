@@ -52,6 +52,8 @@
 #include <cstddef>
 #include <type_traits>
 
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 #include "quant_tables.cuh"
 #include "row_order.cuh"
@@ -455,18 +457,43 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
     }
   };
 
-  // Candidates below kstart: every unit of the warp is fully clamped; closed-form losses.
-#pragma unroll 1
-  for (int k = 0; k < kstart; ++k) {
-    const float sk = sh.tab[kLev * k + 2].w;  // grid value 1 times s_k
+  // Candidates below kstart: every unit of the warp is fully clamped, and its loss is the
+  // parabola f(k) = (pa s_k + pb) s_k, evaluated in fp32 exactly as written. For pa > 0 its
+  // minimum over the prefix (lowest k on equal values) is at one of the two candidates that
+  // bracket the vertex s* = -pb / (2 pa), up to rounding: consecutive candidate scales differ by
+  // at least 1/16 (relative), so a candidate two or more places beyond the bracket exceeds the
+  // bracket's better one by at least about 0.6% of pa s*^2, against rounding errors of a few
+  // 2^-24 of the same. The E4M3 code of s*/g, rounded to nearest, is one of the bracketing
+  // candidates' codes or next to them, so the candidates within three places of it find the
+  // same minimum and index as all of them. Short prefixes, pa <= 0 and values near the ends of
+  // the fp32 range take every candidate.
+  constexpr int kPrefixWin = 3;
+  const float s0 = sh.tab[2].w;  // the smallest candidate scale (grid value 1 times s_0)
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const float L = fmaf(pa[u], sk, pb[u]) * sk;
-      if (L < best[u]) {
-        best[u] = L;
-        best_k[u] = k;
+  for (int u = 0; u < 2; ++u) {
+    int lo = 0, hi = kstart;
+    const float a = pa[u], b = pb[u];
+    if (kstart > 2 * kPrefixWin + 1 && s0 > 0.f && a > 0.f && a < 0x1p100f && fabsf(b) < 0x1p100f &&
+        a * s0 * s0 >= 0x1p-100f && sh.tab[kLev * (kstart - 1) + 2].w < 0x1p40f) {
+      const float q = fmaxf(-b / (2.f * a), 0.f) / __ldg(g + e);  // s*/g, or 0 if the vertex is at s <= 0
+      const int c = static_cast<int>(__nv_cvt_float_to_fp8(q, __NV_SATFINITE, __NV_E4M3) & 0x7F);
+      const int k0 = min(max(c - 1, 0), kstart - 1);  // candidate k has code k + 1
+      lo = max(0, k0 - kPrefixWin);
+      hi = min(kstart, k0 + kPrefixWin + 1);
+    }
+    float bu = best[u];
+    int bk = best_k[u];
+#pragma unroll 1
+    for (int k = lo; k < hi; ++k) {
+      const float sk = sh.tab[kLev * k + 2].w;  // grid value 1 times s_k
+      const float L = fmaf(a, sk, b) * sk;
+      if (L < bu) {
+        bu = L;
+        bk = k;
       }
     }
+    best[u] = bu;
+    best_k[u] = bk;
   }
   // From kstart: levels by counting thresholds until the 4th candidate and until the rest is a
   // multiple of four, then by single-step drops (consecutive scales differ by at most 4/3).
