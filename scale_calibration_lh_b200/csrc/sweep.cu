@@ -25,6 +25,8 @@
 //  * Loss: packed f32x2 products, L = sum_i Imp_i (|wq_i| - |w_i|)^2.
 #include <cstddef>
 
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 #include "quant_tables.cuh"
 #include "row_order.cuh"
@@ -72,7 +74,7 @@ __device__ __forceinline__ void load_w16(const WT* src, float* w) {
 }
 
 template <typename WT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 7)  // seven CTAs (28 warps) per SM: 72 registers
 sweep_diag_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float* __restrict__ imp,  // NULL: all 1
                   const float* __restrict__ g, uint8_t* __restrict__ codes, float* __restrict__ wq,
                   float* __restrict__ loss) {
@@ -177,8 +179,30 @@ sweep_diag_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const flo
   // Clamped prefix: the warp's first full candidate is the smallest kfirst of its 32 rows, the
   // first of its sorted range.
   const int kstart = sh.kf_sorted[threadIdx.x & ~31];
+  // The parabola's minimum over the prefix (lowest k on equal values) is at one of the two
+  // candidates that bracket its vertex s* = -pb / (2 pa), up to rounding: consecutive candidate
+  // scales differ by at least 1/16 (relative), so a candidate two or more places beyond the
+  // bracket exceeds the bracket's better one by at least about 0.6% of pa s*^2. With the constant
+  // pc in the sum, rounding errors are a few 2^-24 of pc, so the window is taken only where
+  // pa s*^2 = pb^2 / (4 pa) is at least 2^-12 pc; the candidates within three places of the E4M3
+  // code of s*/g (one of the bracket's codes or next to them) then find the same minimum and
+  // index as all of them. Otherwise every candidate of the prefix is evaluated.
+  constexpr int kPrefixWin = 3;
+  int lo = 0, hi = kstart;
+  {
+    const float s0 = sh.tab[2].y;  // the smallest candidate scale
+    if (kstart > 2 * kPrefixWin + 1 && s0 > 0.f && pa > 0.f && pa < 0x1p100f && fabsf(pb) < 0x1p100f &&
+        pc < 0x1p100f && pa * s0 * s0 >= 0x1p-100f && sh.tab[kLev * (kstart - 1) + 2].y < 0x1p40f &&
+        pb * pb >= 0x1p-10f * pa * pc) {
+      const float q = fmaxf(-pb / (2.f * pa), 0.f) / __ldg(g + e);  // s*/g (0 if the vertex is at s <= 0)
+      const int c = static_cast<int>(__nv_cvt_float_to_fp8(q, __NV_SATFINITE, __NV_E4M3) & 0x7F);
+      const int k0 = min(max(c - 1, 0), kstart - 1);  // candidate k has code k + 1
+      lo = max(0, k0 - kPrefixWin);
+      hi = min(kstart, k0 + kPrefixWin + 1);
+    }
+  }
 #pragma unroll 1
-  for (int k = 0; k < kstart; ++k) {
+  for (int k = lo; k < hi; ++k) {
     const float sk = sh.tab[kLev * k + 2].y;  // grid value 1 times s_k
     const float L = fmaf(fmaf(pa, sk, pb), sk, pc);
     if (L < best) {
