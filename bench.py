@@ -75,10 +75,10 @@ WORKLOAD_TEXT = {
 # counters). The fused-MoE sweep was captured with 128 rows per expert and is scaled to the
 # 1280 rows of the workload (its traffic, W in and Wq out, grows with the rows).
 PROFILED_TRAFFIC = {
-    ("dense", "sweep_tc_kernel"): {"bytes": 33_860_608 + 27_109_120},
-    ("act", "sweep_tc_kernel"): {"bytes": 101_307_648 + 172_282_880},
-    ("moe", "sweep_tc_kernel"): {"bytes": 10 * (419_859_200 + 700_098_816), "scaled": "x10 from 128 rows per expert"},
-    ("wmse", "sweep_diag_kernel"): {"bytes": 100_809_000 + 163_823_616},
+    ("dense", "sweep_tc_kernel"): {"bytes": 33_956_352 + 28_585_216},
+    ("act", "sweep_tc_kernel"): {"bytes": 101_255_168 + 177_749_248},
+    ("moe", "sweep_tc_kernel"): {"bytes": 10 * (420_230_912 + 702_877_440), "scaled": "x10 from 128 rows per expert"},
+    ("wmse", "sweep_diag_kernel"): {"bytes": 100_873_216 + 163_058_176},
     ("dense", "accum"): {"bytes": 134_267_904 + 3_960_064},
     ("act", "accum"): {"bytes": 268_599_552 + 3_796_736},
     ("moe", "accum"): {"bytes": 84_716_032 + 49_333_248},
