@@ -39,8 +39,8 @@
 // Work per candidate. Candidates below the warp's first unclamped one take a closed form;
 // the rest go four per loop trip, and the quad's four lanes share the reduction of four
 // candidates (a transposed reduction: lane t ends with candidate k + t) and keep their own
-// bests, merged after the loop. The argmin compares L - C' (C' is the same for all of a
-// unit's candidates); the winner's loss is then recomputed by its definition.
+// bests, merged after the loop. The argmin compares 2^eH (L - C') (C' and 2^eH are the same for
+// all of a unit's candidates); the winner's loss is then recomputed by its definition.
 //
 // Set-up per CTA (128 rows of one block). The rows' weights are staged in shared memory once;
 // each row's first unclamped candidate kfirst comes from a binary search of the top-level
@@ -90,7 +90,7 @@ struct __align__(16) TcShared {
   // warp's lane groups read at once with 16-byte loads then fall in distinct banks.
   alignas(16) float wall[kUnitsPerCta][kWStride];
   float rho[kCand];  // -2 / (s_k * 2^eH): scale of U' in the MMA accumulator
-  float s2[kCand];   // s_k^2 * 2^eH
+  float s2[kCand];   // s_k^2 (losses are compared in H' units, 2^eH times the true ones)
   float hscale;  // 2^-eH: H' = H * hscale lies below 2^15
   int kfirst[kUnitsPerCta];     // per row: first candidate with an element below the top level
   int perm[kUnitsPerCta];       // the CTA's rows in ascending kfirst (row_order.cuh)
@@ -292,11 +292,10 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
     row_order_scan(sh.hist, sh.base);
   } else if (warp == 1) {
     const float hscale = sh.hscale;
-    const float inv_hscale = 1.0f / hscale;  // exact: a power of two
     for (int k = lane; k < kCand; k += 32) {
       const float s = candidate_scale(k, gs);
       sh.rho[k] = -2.f * hscale / s;
-      sh.s2[k] = (s * s) * inv_hscale;
+      sh.s2[k] = s * s;
     }
   }
   __syncthreads();
@@ -381,8 +380,9 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
       qa += __shfl_xor_sync(0xffffffffu, qa, o);
       qb += __shfl_xor_sync(0xffffffffu, qb, o);
     }
-    pa[u] = 36.f * qa;
-    pb[u] = -12.f * qb;
+    // In H' units, as the candidate loop compares: times 2^eH (exact, a power of two).
+    pa[u] = 36.f * (qa * hscale);
+    pb[u] = -12.f * (qb * hscale);
   }
   if (ACT && kPair) {
     // The epilogue needs (P w)_c again. Rather than keep it in registers through the sweep, each
@@ -409,9 +409,10 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
 
   // One candidate: A fragment from the elements' packed fp16 grid values; the accumulator starts
   // at rho_k U', so after the 4 MMAs D = v^T H' + rho_k U' and
-  //   L - C' = s2_k * sum_n v_n D_n = s^2 v^T H v - 2 s v^T U'.
-  // C' is the same for every candidate of a unit, so the argmin compares L - C'; the winner's
-  // loss is recomputed by its definition after the sweep.
+  //   s2_k * sum_n v_n D_n = 2^eH (s^2 v^T H v - 2 s v^T U') = 2^eH (L - C').
+  // C' and 2^eH are the same for every candidate of a unit, so the argmin compares these values
+  // (normalised to H', they stay in range whatever H's magnitude); the winner's loss is
+  // recomputed by its definition after the sweep.
   // The lane's share of t for units 0 and 1 (its 4 columns), before the reduction over the quad.
   auto partials_afr = [&](const uint32_t (&afr)[4], int k, float (&tp)[2]) {
     const float rk = sh.rho[k];
