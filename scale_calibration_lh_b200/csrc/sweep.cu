@@ -184,10 +184,10 @@ sweep_diag_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const flo
   // scales differ by at least 1/16 (relative), so a candidate two or more places beyond the
   // bracket exceeds the bracket's better one by at least about 0.6% of pa s*^2. With the constant
   // pc in the sum, rounding errors are a few 2^-24 of pc, so the window is taken only where
-  // pa s*^2 = pb^2 / (4 pa) is at least 2^-12 pc; the candidates within three places of the E4M3
+  // pa s*^2 = pb^2 / (4 pa) is at least 2^-12 pc; the candidates within two places of the E4M3
   // code of s*/g (one of the bracket's codes or next to them) then find the same minimum and
   // index as all of them. Otherwise every candidate of the prefix is evaluated.
-  constexpr int kPrefixWin = 3;
+  constexpr int kPrefixWin = 2;
   int lo = 0, hi = kstart;
   {
     const float s0 = sh.tab[2].y;  // the smallest candidate scale

@@ -465,10 +465,10 @@ sweep_tc_kernel(const WT* __restrict__ w, int64_t rows, int64_t cin, const float
   // at least 1/16 (relative), so a candidate two or more places beyond the bracket exceeds the
   // bracket's better one by at least about 0.6% of pa s*^2, against rounding errors of a few
   // 2^-24 of the same. The E4M3 code of s*/g, rounded to nearest, is one of the bracketing
-  // candidates' codes or next to them, so the candidates within three places of it find the
+  // candidates' codes or next to them, so the candidates within two places of it find the
   // same minimum and index as all of them. Short prefixes, pa <= 0 and values near the ends of
   // the fp32 range take every candidate.
-  constexpr int kPrefixWin = 3;
+  constexpr int kPrefixWin = 2;
   const float s0 = sh.tab[2].w;  // the smallest candidate scale (grid value 1 times s_0)
 #pragma unroll
   for (int u = 0; u < 2; ++u) {

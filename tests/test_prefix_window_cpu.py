@@ -3,7 +3,7 @@
 While all weights of a unit sit at the top E2M1 level, its loss over the candidate scales s_k is
 a parabola, f(k) = (pa s_k + pb) s_k (FULL / activation-aware, L - C') or ((pa s_k + pb) s_k + pc)
 (WMSE / MSE), evaluated in fp32 with fused multiply-adds. The sweeps evaluate f only at the
-candidates within three places of the E4M3 code of s*/g, s* = -pb / (2 pa) the vertex, under the
+candidates within two places of the E4M3 code of s*/g, s* = -pb / (2 pa) the vertex, under the
 conditions they test, and rely on the minimum over the whole prefix (lowest k on equal values)
 lying in that window. Here that claim is tested directly: random parabolas, global scales and
 prefix lengths; f evaluated at every candidate of the prefix with the kernels' arithmetic
@@ -15,7 +15,7 @@ import torch
 
 from oracle import lhcal_oracle as O
 
-WIN = 3
+WIN = 2
 
 
 def _f32(x):
@@ -103,7 +103,7 @@ def test_centre_is_the_nearest_candidate_up_to_rounding():
     # The parabola is symmetric about s*, so the candidate nearest s* (in value) is the discrete
     # minimum, and rounding s*/g to the nearest E4M3 value finds it: the window's centre is the
     # minimum, or next to it where s*/g falls on a midpoint or the fp32 evaluation rounds a near
-    # tie. The kernels' window of three places each side is the margin for those cases.
+    # tie. The kernels' window of two places each side is the margin for those cases.
     rng = np.random.default_rng(22)
     checked = 0
     for g, s, kstart, pa, pb in _cases(rng, 3000):
